@@ -1,0 +1,356 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test checks the oracle (oracle.cpp) against brute force on tiny inputs, a
+library routine in a special case the method reduces to, a closed form or an
+invariant, so that a dropped term, a wrong sign, index or transposed operand in
+the oracle fails at least one of them.
+
+Pages: [HSA] "Hybrid Sparse Attention for Long-Context LLMs: How Linear Attention
+and Indexer + Top-K Work Together", section "Indexer + Top-K: How Fine-Grained
+Sparse Attention Works" (steps 1-4 and pseudocode); [GSA] "From Linear Attention
+to Gated Sparse Attention: Dissecting a Hybrid LLM Architecture Trade-off",
+section "2. The Core Change" (masked formulation and gate).
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import dsa_synth as S
+import oracle as O
+
+
+def _bf16(x):
+    return S.f32_to_bf16_bits(np.asarray(x, dtype=np.float32))
+
+
+def _val(bits):
+    return S.bf16_bits_to_f32(bits).astype(np.float64)
+
+
+def _problem(arrays, **kw):
+    base = dict(top_k=4, n_idx_heads=1, idx_dim=1, n_q_heads=1, n_kv_heads=1, head_dim=1)
+    base.update(kw)
+    return O.Oracle(arrays, **base)
+
+
+def _rand_layer(seed, q_lens, kv_lens, Hi=3, Di=8, Hq=4, Hkv=2, d=8, nonneg_idx=False,
+                scale=0.5, gate=True):
+    rng = np.random.default_rng(seed)
+    tq, tk = sum(q_lens), sum(kv_lens)
+    grid = lambda shape: (rng.integers(-4, 5, size=shape) / 8.0)
+    qi, ki = grid((tq, Hi, Di)), grid((tk, Hi, Di))
+    if nonneg_idx:
+        qi, ki = np.abs(qi), np.abs(ki)
+    a = {
+        "q_idx": _bf16(qi), "k_idx": _bf16(ki),
+        "w": np.array([0.25, 0.5, 1.0, 2.0][:Hi], dtype=np.float32),
+        "q": _bf16(rng.normal(size=(tq, Hq, d)) * scale),
+        "k": _bf16(rng.normal(size=(tk, Hkv, d)) * scale),
+        "v": _bf16(rng.normal(size=(tk, Hkv, d))),
+        "q_offsets": np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int64),
+        "kv_offsets": np.concatenate([[0], np.cumsum(kv_lens)]).astype(np.int64),
+    }
+    if gate:
+        a["gate"] = _bf16(rng.normal(size=(tq, Hq, d)))
+    return a
+
+
+# ----------------------------------------------------------------------------- indexer
+
+def test_indexer_nonnegative_reduces_to_one_matmul():
+    """With q, k >= 0 every per-head dot is >= 0, so ReLU is the identity and
+    s = sum_h w_h q_h k_h^T is one matmul over the concatenated (head, dim) axis."""
+    q_lens, kv_lens = [5, 1, 7], [9, 4, 7]
+    a = _rand_layer(1, q_lens, kv_lens, Hi=3, Di=8, nonneg_idx=True)
+    orc = _problem(a, n_idx_heads=3, idx_dim=8)
+    qo, ko = a["q_offsets"], a["kv_offsets"]
+    w = torch.tensor(a["w"], dtype=torch.float64)
+    for b in range(3):
+        qb = torch.tensor(_val(a["q_idx"][qo[b]:qo[b + 1]]))            # [Q, H, D]
+        kb = torch.tensor(_val(a["k_idx"][ko[b]:ko[b + 1]]))            # [L, H, D]
+        lib = torch.matmul((qb * w[None, :, None]).reshape(len(qb), -1),
+                           kb.reshape(len(kb), -1).T).numpy()           # [Q, L]
+        for i in range(q_lens[b]):
+            r = int(qo[b]) + i
+            p = kv_lens[b] - q_lens[b] + i
+            s = orc.index_scores_row(r)
+            assert len(s) == p + 1
+            np.testing.assert_array_equal(s, lib[i, : p + 1])
+
+
+def test_indexer_relu_and_weights_closed_form():
+    """q_h = sign_h * e_0; then s[j] = sum_h w_h max(0, sign_h k[j,h,0]).  A dropped
+    ReLU, a wrong head weight or a sign slip changes the value."""
+    Hi, Di, L = 4, 3, 6
+    signs = np.array([1, -1, 1, -1], dtype=np.float64)
+    q = np.zeros((1, Hi, Di))
+    q[0, :, 0] = signs
+    rng = np.random.default_rng(2)
+    k = rng.integers(-4, 5, size=(L, Hi, Di)) / 8.0
+    w = np.array([0.25, 0.5, 1.0, 2.0], dtype=np.float32)
+    a = {"q_idx": _bf16(q), "k_idx": _bf16(k), "w": w,
+         "q_offsets": np.array([0, 1]), "kv_offsets": np.array([0, L])}
+    s = _problem(a, n_idx_heads=Hi, idx_dim=Di).index_scores_row(0)
+    expect = [sum(float(w[h]) * max(0.0, signs[h] * k[j, h, 0]) for h in range(Hi))
+              for j in range(L)]
+    np.testing.assert_array_equal(s, expect)
+
+
+def test_indexer_row_sees_itself_and_not_the_future():
+    """Query at position p scores positions 0..p inclusive and no later one."""
+    L = 8
+    q = np.ones((3, 1, 1)) * 0.5
+    k = (np.arange(L, dtype=np.float64) / 8.0).reshape(L, 1, 1)
+    a = {"q_idx": _bf16(q), "k_idx": _bf16(k), "w": np.array([1.0], np.float32),
+         "q_offsets": np.array([0, 3]), "kv_offsets": np.array([0, L])}
+    orc = _problem(a)
+    for i in range(3):
+        p = L - 3 + i
+        s = orc.index_scores_row(i)
+        np.testing.assert_array_equal(s, 0.5 * np.arange(p + 1) / 8.0)
+
+
+def test_indexer_fp8_e4m3_decoding_matches_torch():
+    """All 256 e4m3 codes: q = +1 gives relu(value), q = -1 gives relu(-value); the
+    decoded values are compared with torch's float8_e4m3fn conversion."""
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    L = len(codes)
+    ref = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for qcode, sign in ((0x38, 1.0), (0xB8, -1.0)):
+        a = {"q_idx": np.array([[[qcode]]], np.uint8), "k_idx": codes.reshape(L, 1, 1),
+             "w": np.array([1.0], np.float32),
+             "q_offsets": np.array([0, 1]), "kv_offsets": np.array([0, L])}
+        s = _problem(a, idx_fp8=True).index_scores_row(0)
+        np.testing.assert_array_equal(s, np.maximum(0.0, sign * ref))
+
+
+# ----------------------------------------------------------------------------- top-k
+
+def _is_valid_topk(s, K, idx):
+    """The selection is valid iff it has min(K, n) distinct ascending positions and
+    every selected i beats every unselected j: s_i > s_j, or equal with i < j."""
+    n = len(s)
+    take = min(K, n)
+    sel = idx[:take]
+    if not np.all(idx[take:] == -1):
+        return False
+    if len(set(sel.tolist())) != take or not np.all(np.diff(sel) > 0):
+        return False
+    chosen = set(sel.tolist())
+    for i in chosen:
+        for j in range(n):
+            if j in chosen:
+                continue
+            if not (s[i] > s[j] or (s[i] == s[j] and i < j)):
+                return False
+    return True
+
+
+def test_topk_exhaustive_tiny_rows():
+    """Every row over {0, 1, 2}^n for n <= 6 and every K in 1..7 (brute force)."""
+    for n in range(1, 7):
+        for vals in itertools.product([0.0, 1.0, 2.0], repeat=n):
+            s = np.array(vals)
+            for K in range(1, 8):
+                idx = O.topk_row(s, K)
+                assert _is_valid_topk(s, K, idx), (vals, K, idx)
+
+
+def test_topk_matches_stable_descending_sort():
+    """Library routine: a stable descending sort keeps lower positions first among
+    equal scores, so its first K positions are the selection."""
+    rng = np.random.default_rng(3)
+    for trial in range(200):
+        n = int(rng.integers(1, 700))
+        K = int(rng.integers(1, 300))
+        kind = trial % 4
+        if kind == 0:
+            s = rng.integers(0, 4, size=n).astype(np.float64)           # heavy ties
+        elif kind == 1:
+            s = rng.normal(size=n).astype(np.float32).astype(np.float64)
+        elif kind == 2:
+            s = np.zeros(n)                                             # all equal
+        else:
+            s = (rng.integers(0, 64 * 256, size=n) / 256.0)             # dyadic scores
+        order = torch.sort(torch.tensor(s), descending=True, stable=True).indices.numpy()
+        expect = np.sort(order[:K]).astype(np.int32)
+        idx = O.topk_row(s, K)
+        np.testing.assert_array_equal(idx[: len(expect)], expect)
+        assert np.all(idx[len(expect):] == -1)
+
+
+def test_topk_negative_zero_ties_with_zero():
+    s = np.array([0.0, -0.0, 1.0, -0.0, 0.0])
+    np.testing.assert_array_equal(O.topk_row(s, 3), [0, 1, 2])
+    s = np.array([-0.0, 0.0, -1.0])
+    np.testing.assert_array_equal(O.topk_row(s, 1), [0])
+
+
+def test_topk_short_row_takes_everything():
+    idx = O.topk_row(np.array([3.0, 1.0, 2.0]), 5)
+    np.testing.assert_array_equal(idx, [0, 1, 2, -1, -1])
+
+
+# ----------------------------------------------------------------------------- attention
+
+def _dense_causal_reference(a, q_lens, kv_lens, Hq, Hkv, d, mask_rows=None, gate=True):
+    """torch SDPA (fp64, CPU) per sequence, GQA by repeating KV heads, times sigmoid(gate)."""
+    G = Hq // Hkv
+    outs = []
+    qo, ko = a["q_offsets"], a["kv_offsets"]
+    for b in range(len(q_lens)):
+        q = torch.tensor(_val(a["q"][qo[b]:qo[b + 1]])).permute(1, 0, 2)       # [Hq, Q, d]
+        k = torch.tensor(_val(a["k"][ko[b]:ko[b + 1]])).permute(1, 0, 2)       # [Hkv, L, d]
+        v = torch.tensor(_val(a["v"][ko[b]:ko[b + 1]])).permute(1, 0, 2)
+        k, v = k.repeat_interleave(G, 0), v.repeat_interleave(G, 0)
+        Q, L = q_lens[b], kv_lens[b]
+        if mask_rows is None:
+            pos = torch.arange(L - Q, L)[:, None]
+            mask = torch.arange(L)[None, :] <= pos                               # causal
+        else:
+            mask = torch.zeros(Q, L, dtype=torch.bool)
+            for i in range(Q):
+                sel = mask_rows[int(qo[b]) + i]
+                mask[i, sel[sel >= 0]] = True
+        o = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=mask)
+        o = o.permute(1, 0, 2)
+        if gate:
+            g = torch.tensor(_val(a["gate"][qo[b]:qo[b + 1]]))
+            o = o * torch.sigmoid(g)
+        outs.append(o.numpy())
+    return np.concatenate(outs, 0)
+
+
+def test_full_history_reduces_to_dense_causal_attention():
+    """K >= history: the selection is every causal position, and the layer is
+    dense causal softmax attention (library SDPA) times the sigmoid gate."""
+    q_lens, kv_lens = [6, 1, 4], [6, 9, 13]
+    Hq, Hkv, d = 4, 2, 8
+    a = _rand_layer(4, q_lens, kv_lens, Hq=Hq, Hkv=Hkv, d=d)
+    orc = _problem(a, top_k=16, n_idx_heads=3, idx_dim=8, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d)
+    rows = list(range(sum(q_lens)))
+    idx, out, lse = orc.layer_rows(rows, nthreads=2)
+    ref = _dense_causal_reference(a, q_lens, kv_lens, Hq, Hkv, d)
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-14)
+    for r in rows:
+        p = orc.position(r)
+        np.testing.assert_array_equal(idx[r, : p + 1], np.arange(p + 1))
+
+
+def test_sparse_selection_matches_masked_dense_attention():
+    """K < history: attention over the gathered rows equals dense attention with a
+    mask that keeps exactly the selected positions ([GSA] masked formulation)."""
+    q_lens, kv_lens = [7, 5], [20, 11]
+    Hq, Hkv, d = 4, 1, 8
+    a = _rand_layer(5, q_lens, kv_lens, Hq=Hq, Hkv=Hkv, d=d)
+    orc = _problem(a, top_k=5, n_idx_heads=3, idx_dim=8, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d)
+    rows = list(range(sum(q_lens)))
+    idx, out, lse = orc.layer_rows(rows, nthreads=1)
+    ref = _dense_causal_reference(a, q_lens, kv_lens, Hq, Hkv, d, mask_rows=idx)
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-14)
+    # the selection itself is the top-K of the oracle's own scores, checked by brute force
+    for r in rows:
+        assert _is_valid_topk(orc.index_scores_row(r), 5, idx[r])
+
+
+def test_attention_invariants():
+    """v = 1 without gate gives exactly 1 (softmax rows sum to 1); q = 0 gives the mean
+    of the selected v rows; one-hot v recovers the softmax weights; gate = 0 halves."""
+    L, Hq, Hkv, d, K = 12, 2, 1, 12, 5
+    rng = np.random.default_rng(6)
+    base = {"q": _bf16(rng.normal(size=(1, Hq, d))), "k": _bf16(rng.normal(size=(L, Hkv, d))),
+            "v": _bf16(np.ones((L, Hkv, d))), "q_offsets": np.array([0, 1]),
+            "kv_offsets": np.array([0, L])}
+    kw = dict(top_k=K, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d)
+    idx = np.array([1, 3, 4, 8, 11], dtype=np.int32)
+    out, lse = _problem(base, **kw).sparse_attn_row(0, idx)
+    np.testing.assert_allclose(out, 1.0, rtol=0, atol=1e-15)
+    # q = 0: uniform weights -> mean of selected v
+    vv = rng.normal(size=(L, Hkv, d))
+    a = dict(base, q=_bf16(np.zeros((1, Hq, d))), v=_bf16(vv))
+    out, lse = _problem(a, **kw).sparse_attn_row(0, idx)
+    np.testing.assert_allclose(out[0], _val(a["v"])[idx, 0].mean(0), rtol=1e-13)
+    np.testing.assert_allclose(lse, math.log(K), rtol=1e-14)
+    # one-hot v: out[h, e] = P_h[position e]; compare with torch.softmax / logsumexp
+    a = dict(base, v=_bf16(np.eye(L, d).reshape(L, 1, d)))
+    out, lse = _problem(a, **kw).sparse_attn_row(0, idx)
+    qf, kf = _val(a["q"])[0], _val(a["k"])[:, 0]
+    logits = torch.tensor(qf @ kf[idx].T / math.sqrt(d))                 # [Hq, K]
+    P = torch.softmax(logits, -1).numpy()
+    for h in range(Hq):
+        np.testing.assert_allclose(out[h, idx], P[h], rtol=1e-13)
+        mask = np.ones(d, bool)
+        mask[idx] = False
+        assert np.all(out[h, mask] == 0)
+    np.testing.assert_allclose(lse, torch.logsumexp(logits, -1).numpy(), rtol=1e-14)
+    # gate = 0: sigmoid(0) = 1/2 exactly
+    a2 = dict(a, gate=_bf16(np.zeros((1, Hq, d))))
+    out2, _ = _problem(a2, **kw).sparse_attn_row(0, idx)
+    np.testing.assert_array_equal(out2, out * 0.5)
+
+
+def test_padding_entries_are_ignored():
+    L, Hq, d = 9, 1, 4
+    rng = np.random.default_rng(7)
+    a = {"q": _bf16(rng.normal(size=(1, Hq, d))), "k": _bf16(rng.normal(size=(L, 1, d))),
+         "v": _bf16(rng.normal(size=(L, 1, d))), "q_offsets": np.array([0, 1]),
+         "kv_offsets": np.array([0, L])}
+    o1, _ = _problem(a, top_k=3, n_q_heads=1, n_kv_heads=1, head_dim=d).sparse_attn_row(
+        0, np.array([2, 5, 7], np.int32))
+    o2, _ = _problem(a, top_k=5, n_q_heads=1, n_kv_heads=1, head_dim=d).sparse_attn_row(
+        0, np.array([2, 5, 7, -1, -1], np.int32))
+    np.testing.assert_array_equal(o1, o2)
+
+
+# ----------------------------------------------------------------------------- whole layer
+
+def test_planted_needles_are_selected():
+    """The planted-needle recipe (reduced length): every designated query row selects
+    all 16 needle positions."""
+    w = S.workload("prefill_t131072_needles", scale_down=64)
+    arrays = S.make_host_inputs(w)
+    orc = O.Oracle.for_workload(w, arrays)
+    rows = w.needle_rows[::16] + [w.needle_rows[-1]]
+    idx, _, _ = orc.layer_rows(rows)
+    for r in range(len(rows)):
+        assert set(w.needle_pos) <= set(idx[r].tolist())
+
+
+def test_golden_tiny_layer():
+    """Hand-worked example in tests/golden/tiny_layer.txt (derivation in the file)."""
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "tiny_layer.txt")
+    g = {}
+    for line in open(path):
+        line = line.split("#", 1)[0].strip()
+        if line:
+            key, val = line.split("=", 1)
+            g[key.strip()] = [float(x) for x in val.split()]
+    L = 4
+    a = {"q_idx": _bf16(np.array(g["q_idx"]).reshape(1, 1, 2)),
+         "k_idx": _bf16(np.array(g["k_idx"]).reshape(L, 1, 2)),
+         "w": np.array([1.0], np.float32),
+         "q": _bf16(np.array(g["q"]).reshape(1, 1, 2)),
+         "k": _bf16(np.array(g["k"]).reshape(L, 1, 2)),
+         "v": _bf16(np.array(g["v"]).reshape(L, 1, 2)),
+         "gate": _bf16(np.array(g["gate"]).reshape(1, 1, 2)),
+         "q_offsets": np.array([0, 1]), "kv_offsets": np.array([0, L])}
+    orc = _problem(a, top_k=2, n_idx_heads=1, idx_dim=2, n_q_heads=1, n_kv_heads=1, head_dim=2,
+                   attn_scale=1.0)
+    np.testing.assert_array_equal(orc.index_scores_row(0), g["scores"])
+    idx, out, lse = orc.layer_rows([0])
+    np.testing.assert_array_equal(idx[0], [int(x) for x in g["topk"]])
+    # closed form: logits l1, l2 over the two selected rows, then sigmoid gate
+    l1, l2 = g["logits"]
+    p1 = 1.0 / (1.0 + math.exp(l2 - l1))
+    v1, v2 = np.array(g["v_sel"][:2]), np.array(g["v_sel"][2:])
+    gate = np.array(g["gate"])
+    expect = (p1 * v1 + (1 - p1) * v2) / (1 + np.exp(-gate))
+    np.testing.assert_allclose(out[0, 0], expect, rtol=1e-15)
+    np.testing.assert_allclose(lse[0, 0], math.log(math.exp(l1) + math.exp(l2)), rtol=1e-15)
+    # the hand-derived numbers printed in the fixture
+    np.testing.assert_allclose(out[0, 0], g["out"], rtol=1e-15)
+    np.testing.assert_allclose(lse[0, 0], g["lse"][0], rtol=1e-15)
