@@ -1,0 +1,222 @@
+/*
+ * dsa.h - C ABI of the B200 (sm_100a) gated Indexer + Top-K sparse-attention layer.
+ *
+ * The layer, for every query row t of a ragged batch:
+ *   1. indexer  s[t,j] = sum_h w_h * max(0, c * q_idx[t,h,:] . k_idx[j,h,:]),  j = 0..p(t)
+ *   2. Top-K    the K positions with the largest s[t,j] (ties: lower j wins), or all
+ *               p(t)+1 positions when there are no more than K
+ *   3. attention o[t,h] = softmax_j(scale * q[t,h] . k[j,g(h)]) . v[j,g(h)] over the
+ *               selected j only (exact softmax over the subset)
+ *   4. gate     out[t,h,e] = sigmoid(gate[t,h,e]) * o[t,h,e]
+ *
+ * Pages this interface follows (web articles on one model release):
+ *   [HSA] "Hybrid Sparse Attention for Long-Context LLMs: How Linear Attention and
+ *          Indexer + Top-K Work Together": section "Indexer + Top-K: How Fine-Grained
+ *          Sparse Attention Works", steps 1-4 and the pseudocode below them.
+ *   [ITK] "Optimizing LLM Long-Context Inference with Indexed Top-K Sparse Attention":
+ *          sections "Introducing Indexed Top-K Sparse Attention" (indexing stage, Top-K
+ *          stage, K = 2048) and "Interface Design for Practical Implementation"
+ *          (sparse_attn_forward(query, key, value, top_k); index consistency across
+ *          heads; variable sequence lengths across a batch).
+ *   [FGS] "How Fine-Grained Sparse Attention Reshapes Long-Context Architecture in Large
+ *          Models": section "How Indexer + Top-K Works at Runtime" (retrieve, read
+ *          precisely, fuse; one index set per query over the KV cache).
+ *   [SAE] "Sparse Attention in Long-Context LLM Inference: Engineering Trade-offs and
+ *          Architecture Choices": section "5. Abstract Implementation Sketch of
+ *          Indexer + Top-K" (scale 1/sqrt(dim); cross-head sharing).
+ *   [GSA] "From Linear Attention to Gated Sparse Attention: Dissecting a Hybrid LLM
+ *          Architecture Trade-off": sections "2. The Core Change" (gate(q) * out) and
+ *          "4. The Role of Gating and Engineering Considerations" (indexer precision,
+ *          fused Top-K).
+ * The pages give no indexer formula; the per-head ReLU dot product with a weighted head
+ * sum in step 1 is the reading this library implements.  One score row and one index
+ * set per query are shared by all attention heads.
+ *
+ * Conventions for every entry point
+ *  - Ownership: the caller owns every buffer and the stream.  The library never
+ *    allocates device memory; scratch comes from a caller-provided workspace.  The
+ *    library keeps no per-call state and may be called from several host threads.
+ *  - Synchrony: every compute call is asynchronous on `stream` (a cudaStream_t; NULL
+ *    is the legacy default stream).  Argument errors are returned before anything is
+ *    launched; a failed launch returns DSA_ERR_CUDA.  No exception crosses the ABI.
+ *  - Device pointers: all tensor arguments are device pointers unless a field says
+ *    "host".  Tensors are row-major and packed ragged: query-side tensors have
+ *    total_q rows (sequence b owns rows q_offsets[b] .. q_offsets[b+1]-1), cache-side
+ *    tensors have total_kv rows (sequence b owns rows kv_offsets[b] ..).
+ *  - Positions: sequence b has L_b = kv_offsets[b+1]-kv_offsets[b] cache positions and
+ *    Q_b = q_offsets[b+1]-q_offsets[b] <= L_b queries, the last Q_b positions: query i
+ *    of b sits at p = L_b - Q_b + i and sees positions 0..p (itself included).  Index
+ *    values are positions within the sequence (0-based).
+ *  - Bad device data is never trapped: index entries < 0 are padding; entries > p are
+ *    skipped and counted in `err_count` when one is given.  A bounded wait inside a
+ *    kernel that runs out records DSA_ERR_TIMEOUT in the device status word
+ *    (dsa_device_status) and the kernel returns.
+ */
+#ifndef DSA_H
+#define DSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1, /* a pointer, size, stride or alignment is invalid     */
+  DSA_ERR_UNSUPPORTED = 2, /* valid but outside what this build implements        */
+  DSA_ERR_WORKSPACE = 3,   /* workspace missing, too small or misaligned          */
+  DSA_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed         */
+  DSA_ERR_TIMEOUT = 5      /* (device status only) a bounded in-kernel wait ended */
+} dsa_status;
+
+typedef enum {
+  DSA_BF16 = 0,     /* bfloat16                                  */
+  DSA_FP8_E4M3 = 1  /* OCP fp8 e4m3 (indexer tensors only)       */
+} dsa_dtype;
+
+/* Ragged batch description. */
+typedef struct {
+  int32_t batch;              /* B >= 1                                            */
+  const int32_t* q_offsets;   /* device [B+1], q_offsets[0] = 0, non-decreasing    */
+  const int32_t* kv_offsets;  /* device [B+1], kv_offsets[0] = 0, non-decreasing   */
+  int32_t max_q_len;          /* host: >= max_b Q_b                                */
+  int32_t max_kv_len;         /* host: >= max_b L_b                                */
+  int64_t total_q;            /* host: q_offsets[B]                                */
+  int64_t total_kv;           /* host: kv_offsets[B]                               */
+} dsa_ragged;
+
+/* Layer shape and numerics.  Supported by this build: idx_dim = 64,
+ * 1 <= n_idx_heads <= 4, head_dim = 128, n_kv_heads divides n_q_heads with
+ * n_q_heads / n_kv_heads <= 16, 1 <= top_k <= 16384. */
+typedef struct {
+  int32_t n_idx_heads;   /* H_i: indexer heads                                        */
+  int32_t idx_dim;       /* D_i: indexer head dimension                               */
+  int32_t n_q_heads;     /* Hq: attention query heads                                 */
+  int32_t n_kv_heads;    /* Hkv: attention KV heads; query head h reads KV head h/(Hq/Hkv) */
+  int32_t head_dim;      /* d                                                         */
+  int32_t top_k;         /* K                                                         */
+  int32_t idx_dtype;     /* dsa_dtype of q_idx and k_idx                              */
+  float idx_scale_q;     /* dequantisation scale of q_idx (1 for bf16)                */
+  float idx_scale_k;     /* dequantisation scale of k_idx (1 for bf16); c = scale_q*scale_k */
+  float attn_scale;      /* softmax logit scale; 0 selects 1/sqrt(head_dim)           */
+  int32_t w_row_stride;  /* 0: w is [H_i], shared by all rows; else w[row*stride + h] */
+} dsa_params;
+
+/* Human-readable name of a status code (static string). */
+const char* dsa_status_string(dsa_status s);
+
+/* Library ABI version (major*10000 + minor*100 + patch). */
+int32_t dsa_version(void);
+
+/*
+ * Step 1 - indexer scores ([HSA] step 1; [ITK] "Two Engineering Considerations",
+ * 1. Indexer Computational Cost: low-dimensional and cheap).
+ *   q_idx  [total_q, H_i, D_i]  bf16 or e4m3 (params->idx_dtype)
+ *   k_idx  [total_kv, H_i, D_i] same dtype
+ *   w      fp32, [H_i] or [total_q, w_row_stride] (see dsa_params)
+ *   scores fp32 [q_count, ld_scores]: row i belongs to packed query row q_begin+i and
+ *          receives s[j] for j = 0..p of that row.  Entries beyond p are not written.
+ * Requirements: 0 <= q_begin, q_begin+q_count <= total_q; ld_scores >= max_kv_len and a
+ * multiple of 4; q_idx, k_idx 16-byte aligned; row strides H_i*D_i*elem a multiple of
+ * 16 bytes.  Runs on tcgen05 tensor cores fed by TMA.
+ */
+dsa_status dsa_index_scores(const dsa_params* params, const dsa_ragged* ragged,
+                            const void* q_idx, const void* k_idx, const float* w,
+                            int64_t q_begin, int64_t q_count, float* scores, int64_t ld_scores,
+                            void* stream);
+
+/*
+ * Step 2 - Top-K selection ([HSA] step 2; [ITK] "Introducing Indexed Top-K Sparse
+ * Attention", Top-K Selection Stage).
+ *   scores fp32 [q_count, ld_scores] as written by dsa_index_scores (only 0..p read)
+ *   idx    int32 [q_count, ld_idx]: the selected positions of row i in ascending order,
+ *          min(K, p+1) of them, then -1 up to K.  Ties at the threshold keep the lower
+ *          positions; -0.0 equals +0.0.  NaN scores are not supported.
+ *   cnt    int32 [q_count] or NULL: number selected per row.
+ * Requirements: ld_scores a multiple of 4 and scores 16-byte aligned; ld_idx >= K.
+ */
+dsa_status dsa_topk(const dsa_params* params, const dsa_ragged* ragged, const float* scores,
+                    int64_t ld_scores, int64_t q_begin, int64_t q_count, int32_t* idx,
+                    int64_t ld_idx, int32_t* cnt, void* stream);
+
+/*
+ * Steps 3-4 - exact softmax attention over the selected rows with the sigmoid output
+ * gate fused in ([HSA] steps 3-4 and pseudocode; [SAE] section 5; [GSA] section 2).
+ *   q        bf16 [total_q, Hq, d]
+ *   k_cache  bf16 [total_kv, Hkv, d]; v_cache likewise
+ *   idx      int32 [q_count, ld_idx], row i for packed query row q_begin+i: positions
+ *            within the sequence, any order; entries < 0 are padding
+ *   gate     bf16 [total_q, Hq, d] gate logits, or NULL for no gate
+ *   out      bf16 [total_q, Hq, d] (rows q_begin..q_begin+q_count-1 written)
+ *   lse      fp32 [q_count, Hq] or NULL: log(sum_j exp(scale * q.k_j)) over the
+ *            selected j (natural log; -inf for a row with nothing selected)
+ *   err_count int32 [1] or NULL: incremented once per index entry > p (skipped)
+ * A row with nothing selected gets out = 0.  All rows read the same index set for all
+ * heads; the gather of a KV head is shared by the query heads of its group.
+ * Requirements: q, k_cache, v_cache, gate, out 16-byte aligned.
+ */
+dsa_status dsa_sparse_attn_gated(const dsa_params* params, const dsa_ragged* ragged,
+                                 const void* q, const void* k_cache, const void* v_cache,
+                                 const int32_t* idx, int64_t ld_idx, int64_t q_begin,
+                                 int64_t q_count, const void* gate, void* out, float* lse,
+                                 int32_t* err_count, void* stream);
+
+/*
+ * Workspace for dsa_prefill / dsa_decode.  *min_bytes: the least that works (one query
+ * row of scores per pass); *rec_bytes: the size this build recommends for throughput
+ * (bounded; fewer, larger passes).  Either pointer may be NULL.
+ */
+dsa_status dsa_workspace_size(const dsa_params* params, const dsa_ragged* ragged, int is_decode,
+                              size_t* min_bytes, size_t* rec_bytes);
+
+/*
+ * Whole layer for a ragged batch of prefill chunks (any Q_b <= L_b): steps 1-4 in
+ * passes over the query rows, each pass sized to the workspace (scores and, when
+ * idx_out is NULL, index rows live there).  Fused Top-K and gather per [HSA]
+ * "Engineering and Evaluation Recommendations" (inference side) and chunked prefill.
+ *   idx_out  int32 [total_q, K] or NULL: the selected positions (as dsa_topk).
+ *   err_count int32 [1] or NULL (as dsa_sparse_attn_gated).
+ *   workspace device, 256-byte aligned, ws_bytes >= the minimum of dsa_workspace_size.
+ */
+dsa_status dsa_prefill(const dsa_params* params, const dsa_ragged* ragged, const void* q_idx,
+                       const void* k_idx, const float* w, const void* q, const void* k_cache,
+                       const void* v_cache, const void* gate, void* out, int32_t* idx_out,
+                       int32_t* err_count, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Whole layer for one new token per sequence (every Q_b = 1, so max_q_len must be 1 and
+ * total_q = batch).  Same arguments and outputs as dsa_prefill; tiles are sized for a
+ * single query per sequence (the indexer becomes a bandwidth-bound scan of k_idx).
+ */
+dsa_status dsa_decode(const dsa_params* params, const dsa_ragged* ragged, const void* q_idx,
+                      const void* k_idx, const float* w, const void* q, const void* k_cache,
+                      const void* v_cache, const void* gate, void* out, int32_t* idx_out,
+                      int32_t* err_count, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Device status word of the current device: synchronises `stream`, stores the status
+ * recorded by kernels since the last clear (DSA_OK or DSA_ERR_TIMEOUT) in *status (host),
+ * and clears it when clear != 0.
+ */
+dsa_status dsa_device_status(void* stream, int32_t* status, int clear);
+
+/* Number of kernels this library has launched from the calling host thread. */
+int64_t dsa_launch_count(void);
+
+/*
+ * Per-stage device timing, for measurement.  While enabled, each stage launch made
+ * from the calling host thread is bracketed by CUDA events on its stream.
+ * dsa_stage_times synchronises those events and returns, per stage (0 indexer,
+ * 1 Top-K, 2 attention), the summed milliseconds and launch counts since the last
+ * reset; the arrays are host [3].
+ */
+dsa_status dsa_stage_timing(int enable);
+dsa_status dsa_stage_times(double* ms, int64_t* launches, int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H */

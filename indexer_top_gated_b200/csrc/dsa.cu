@@ -1,0 +1,497 @@
+// dsa.cu - C ABI of the gated Indexer + Top-K sparse-attention layer (include/dsa.h):
+// argument validation, launch configuration, TMA tensor maps, the fused prefill and
+// decode drivers, per-stage timing and the device status word.  All kernels live in
+// the headers included here, so the library is one translation unit.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "dsa.h"
+#include "common.cuh"
+#include "idx_scores.cuh"
+#include "sparse_attn.cuh"
+#include "topk.cuh"
+
+namespace dsa {
+
+// Device status word: kernels record DSA_ERR_TIMEOUT here when a bounded wait ends.
+__device__ int g_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxTopK = 16384;
+
+thread_local int64_t t_launches = 0;
+
+// ---------------------------------------------------------------- stage timing
+struct StageRec {
+  int stage;
+  cudaEvent_t start, stop;
+};
+thread_local bool t_timing = false;
+thread_local std::vector<StageRec> t_pending;
+thread_local std::vector<cudaEvent_t> t_free_events;
+thread_local double t_stage_ms[3] = {0, 0, 0};
+thread_local int64_t t_stage_launches[3] = {0, 0, 0};
+
+cudaEvent_t take_event() {
+  if (!t_free_events.empty()) {
+    cudaEvent_t e = t_free_events.back();
+    t_free_events.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+struct StageScope {
+  int stage;
+  cudaStream_t stream;
+  cudaEvent_t start = nullptr, stop = nullptr;
+  StageScope(int s, cudaStream_t st) : stage(s), stream(st) {
+    if (t_timing) {
+      start = take_event();
+      stop = take_event();
+      if (start) cudaEventRecord(start, stream);
+    }
+  }
+  ~StageScope() {
+    if (start && stop) {
+      cudaEventRecord(stop, stream);
+      t_pending.push_back({stage, start, stop});
+    }
+    ++t_stage_launches[stage];
+  }
+};
+
+// ---------------------------------------------------------------- per-device setup
+struct DeviceState {
+  bool ready = false;
+  int* status = nullptr;  // device address of g_status
+  int num_sms = 148;
+  size_t max_smem = 0;
+};
+DeviceState g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+template <typename K>
+cudaError_t allow_smem(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+dsa_status device_setup(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceState& d = g_dev[dev];
+  if (!d.ready) {
+    if (cudaGetSymbolAddress((void**)&d.status, g_status) != cudaSuccess) return DSA_ERR_CUDA;
+    cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    int smem_optin = 0;
+    cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    d.max_smem = (size_t)smem_optin;
+    const size_t idx_max = idx_smem_bytes(4, 64, false);
+    cudaError_t e = cudaSuccess;
+    e = e ? e : allow_smem(idx_scores_kernel<64, false>, idx_max);
+    e = e ? e : allow_smem(idx_scores_kernel<16, false>, idx_max);
+    e = e ? e : allow_smem(idx_scores_kernel<64, true>, idx_max);
+    e = e ? e : allow_smem(idx_scores_kernel<16, true>, idx_max);
+    e = e ? e : allow_smem(topk_kernel, kTopkStageCap * sizeof(uint32_t));
+    e = e ? e : allow_smem(sparse_attn_kernel<1, 1>, attn_smem_bytes());
+    e = e ? e : allow_smem(sparse_attn_kernel<2, 1>, attn_smem_bytes());
+    e = e ? e : allow_smem(sparse_attn_kernel<4, 1>, attn_smem_bytes());
+    e = e ? e : allow_smem(sparse_attn_kernel<8, 1>, attn_smem_bytes());
+    e = e ? e : allow_smem(sparse_attn_kernel<1, 2>, attn_smem_bytes());
+    e = e ? e : allow_smem(sparse_attn_kernel<2, 2>, attn_smem_bytes());
+    e = e ? e : allow_smem(sparse_attn_kernel<4, 2>, attn_smem_bytes());
+    e = e ? e : allow_smem(sparse_attn_kernel<8, 2>, attn_smem_bytes());
+    if (e != cudaSuccess) return DSA_ERR_CUDA;
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn)
+        return DSA_ERR_CUDA;
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    d.ready = true;
+  }
+  *out = &d;
+  return DSA_OK;
+}
+
+// ---------------------------------------------------------------- validation
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+dsa_status check_common(const dsa_params* P, const dsa_ragged* R) {
+  if (!P || !R) return DSA_ERR_INVALID_ARG;
+  if (R->batch < 1 || !R->q_offsets || !R->kv_offsets) return DSA_ERR_INVALID_ARG;
+  if (R->max_q_len < 0 || R->max_kv_len < 0 || R->total_q < 0 || R->total_kv < 0)
+    return DSA_ERR_INVALID_ARG;
+  if (R->total_q > INT32_MAX || R->total_kv > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  if (P->top_k < 1 || P->top_k > kMaxTopK) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+dsa_status check_indexer(const dsa_params* P) {
+  if (P->idx_dim != 64) return DSA_ERR_UNSUPPORTED;
+  if (P->n_idx_heads < 1 || P->n_idx_heads > 4) return DSA_ERR_UNSUPPORTED;
+  if (P->idx_dtype != DSA_BF16 && P->idx_dtype != DSA_FP8_E4M3) return DSA_ERR_INVALID_ARG;
+  if (P->w_row_stride < 0) return DSA_ERR_INVALID_ARG;
+  if (P->w_row_stride != 0 && P->w_row_stride < P->n_idx_heads) return DSA_ERR_INVALID_ARG;
+  if (!(P->idx_scale_q > 0.f) || !(P->idx_scale_k > 0.f)) return DSA_ERR_INVALID_ARG;
+  return DSA_OK;
+}
+
+dsa_status check_attn(const dsa_params* P) {
+  if (P->head_dim != kHeadDim) return DSA_ERR_UNSUPPORTED;
+  if (P->n_q_heads < 1 || P->n_kv_heads < 1) return DSA_ERR_INVALID_ARG;
+  if (P->n_q_heads % P->n_kv_heads != 0) return DSA_ERR_INVALID_ARG;
+  const int G = P->n_q_heads / P->n_kv_heads;
+  if (G > 16) return DSA_ERR_UNSUPPORTED;
+  const int hkv = P->n_kv_heads;
+  if (!(hkv == 1 || hkv == 2 || hkv == 4 || hkv % 8 == 0)) return DSA_ERR_UNSUPPORTED;
+  if (P->attn_scale < 0.f || !std::isfinite(P->attn_scale)) return DSA_ERR_INVALID_ARG;
+  return DSA_OK;
+}
+
+#define DSA_TRY(x)                   \
+  do {                               \
+    dsa_status _s = (x);             \
+    if (_s != DSA_OK) return _s;     \
+  } while (0)
+
+// ---------------------------------------------------------------- launches
+dsa_status make_idx_map(CUtensorMap* map, const void* base, int64_t rows, int n_heads, bool fp8,
+                        int box_rows) {
+  const int elem = fp8 ? 1 : 2;
+  cuuint64_t gdim[2] = {(cuuint64_t)(n_heads * 64), (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)(n_heads * 64 * elem)};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint32_t estride[2] = {1u, 1u};
+  CUresult r = g_encode(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                        2, const_cast<void*>(base), gdim, gstride, box, estride,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        fp8 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DSA_OK : DSA_ERR_INVALID_ARG;
+}
+
+dsa_status launch_index_scores(const DeviceState& dev, const dsa_params* P, const dsa_ragged* R,
+                               const void* q_idx, const void* k_idx, const float* w,
+                               int64_t q_begin, int64_t q_count, float* scores, int64_t ld,
+                               int bq, cudaStream_t stream) {
+  if (q_count == 0 || R->total_kv == 0) return DSA_OK;
+  const bool fp8 = P->idx_dtype == DSA_FP8_E4M3;
+  CUtensorMap mq, mk;
+  DSA_TRY(make_idx_map(&mq, q_idx, R->total_q, P->n_idx_heads, fp8, bq));
+  DSA_TRY(make_idx_map(&mk, k_idx, R->total_kv, P->n_idx_heads, fp8, kIdxKeyTile));
+  IdxArgs a;
+  a.q_offsets = R->q_offsets;
+  a.kv_offsets = R->kv_offsets;
+  a.batch = R->batch;
+  a.n_heads = P->n_idx_heads;
+  a.q_begin = q_begin;
+  a.q_count = q_count;
+  a.n_tiles = (int)((q_count + bq - 1) / bq);
+  const int max_kt = std::max(1, (R->max_kv_len + kIdxKeyTile - 1) / kIdxKeyTile);
+  // enough CTAs to fill the GPU a few times over, at least 8 key tiles per CTA
+  const int64_t target = (int64_t)dev.num_sms * 8;
+  int ysplit = (int)std::min<int64_t>((target + a.n_tiles - 1) / a.n_tiles,
+                                      std::max(1, max_kt / 8));
+  ysplit = std::max(ysplit, 1);
+  a.kt_per_split = (max_kt + ysplit - 1) / ysplit;
+  ysplit = (max_kt + a.kt_per_split - 1) / a.kt_per_split;
+  a.w = w;
+  a.w_row_stride = P->w_row_stride;
+  a.scale = P->idx_scale_q * P->idx_scale_k;
+  a.scores = scores;
+  a.ld = ld;
+  a.status = dev.status;
+  const size_t smem = idx_smem_bytes(P->n_idx_heads, bq, fp8);
+  dim3 grid((unsigned)a.n_tiles, (unsigned)ysplit);
+  StageScope scope(0, stream);
+  if (bq == 64) {
+    if (fp8) idx_scores_kernel<64, true><<<grid, kIdxThreads, smem, stream>>>(mq, mk, a);
+    else idx_scores_kernel<64, false><<<grid, kIdxThreads, smem, stream>>>(mq, mk, a);
+  } else {
+    if (fp8) idx_scores_kernel<16, true><<<grid, kIdxThreads, smem, stream>>>(mq, mk, a);
+    else idx_scores_kernel<16, false><<<grid, kIdxThreads, smem, stream>>>(mq, mk, a);
+  }
+  ++t_launches;
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+dsa_status launch_topk(const dsa_params* P, const dsa_ragged* R, const float* scores, int64_t ld,
+                       int64_t q_begin, int64_t q_count, int32_t* idx, int64_t ld_idx,
+                       int32_t* cnt, cudaStream_t stream) {
+  if (q_count == 0) return DSA_OK;
+  TopkArgs a;
+  a.q_offsets = R->q_offsets;
+  a.kv_offsets = R->kv_offsets;
+  a.batch = R->batch;
+  a.q_begin = q_begin;
+  a.q_count = q_count;
+  a.K = P->top_k;
+  a.scores = scores;
+  a.ld = ld;
+  a.idx = idx;
+  a.ld_idx = ld_idx;
+  a.cnt = cnt;
+  const size_t smem =
+      (size_t)std::min<int64_t>(kTopkStageCap, (int64_t)R->max_kv_len + 4) * sizeof(uint32_t);
+  StageScope scope(1, stream);
+  topk_kernel<<<(unsigned)q_count, kTopkThreads, smem, stream>>>(a);
+  ++t_launches;
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+dsa_status launch_attn(const dsa_params* P, const dsa_ragged* R, const void* q, const void* k,
+                       const void* v, const int32_t* idx, int64_t ld_idx, int64_t q_begin,
+                       int64_t q_count, const void* gate, void* out, float* lse,
+                       int32_t* err_count, cudaStream_t stream) {
+  if (q_count == 0) return DSA_OK;
+  AttnArgs a;
+  a.q_offsets = R->q_offsets;
+  a.kv_offsets = R->kv_offsets;
+  a.batch = R->batch;
+  a.q_begin = q_begin;
+  a.q_count = q_count;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.idx = idx;
+  a.ld_idx = ld_idx;
+  a.K = P->top_k;
+  a.gate = static_cast<const __nv_bfloat16*>(gate);
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.lse = lse;
+  a.err_count = err_count;
+  a.Hq = P->n_q_heads;
+  a.Hkv = P->n_kv_heads;
+  a.G = P->n_q_heads / P->n_kv_heads;
+  const float scale = P->attn_scale > 0.f ? P->attn_scale : 1.0f / std::sqrt((float)P->head_dim);
+  a.scale_log2 = scale * 1.4426950408889634f;
+  const int hkv_cta = std::min(P->n_kv_heads, 8);
+  const int nt = a.G > 8 ? 2 : 1;
+  dim3 grid((unsigned)q_count, (unsigned)(P->n_kv_heads / hkv_cta));
+  const size_t smem = attn_smem_bytes();
+  StageScope scope(2, stream);
+#define DSA_ATTN_CASE(H, N)                                                         \
+  if (hkv_cta == H && nt == N)                                                      \
+    sparse_attn_kernel<H, N><<<grid, kAttnThreads, smem, stream>>>(a);
+  DSA_ATTN_CASE(1, 1)
+  DSA_ATTN_CASE(2, 1)
+  DSA_ATTN_CASE(4, 1)
+  DSA_ATTN_CASE(8, 1)
+  DSA_ATTN_CASE(1, 2)
+  DSA_ATTN_CASE(2, 2)
+  DSA_ATTN_CASE(4, 2)
+  DSA_ATTN_CASE(8, 2)
+#undef DSA_ATTN_CASE
+  ++t_launches;
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+// Workspace per pass row: scores row (ld floats) plus an index row when idx_out is absent.
+int64_t scores_ld(const dsa_ragged* R) { return round_up(std::max(R->max_kv_len, 1), 32); }
+
+dsa_status run_layer(const dsa_params* P, const dsa_ragged* R, const void* q_idx,
+                     const void* k_idx, const float* w, const void* q, const void* k,
+                     const void* v, const void* gate, void* out, int32_t* idx_out,
+                     int32_t* err_count, void* ws, size_t ws_bytes, void* stream_v,
+                     bool decode) {
+  DSA_TRY(check_common(P, R));
+  DSA_TRY(check_indexer(P));
+  DSA_TRY(check_attn(P));
+  if (!q_idx || !k_idx || !w || !q || !k || !v || !out) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(q) || !aligned16(k) ||
+      !aligned16(v) || !aligned16(out) || (gate && !aligned16(gate)))
+    return DSA_ERR_INVALID_ARG;
+  if (decode && (R->max_q_len != 1 || R->total_q != R->batch)) return DSA_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return DSA_ERR_WORKSPACE;
+  if (R->total_q == 0) return DSA_OK;
+  const int64_t ld = scores_ld(R);
+  const int64_t K = P->top_k;
+  const int64_t row_bytes = ld * 4 + (idx_out ? 0 : round_up(K * 4, 16));
+  const int64_t rows = std::min<int64_t>(R->total_q, (int64_t)ws_bytes / row_bytes);
+  if (rows < 1) return DSA_ERR_WORKSPACE;
+  DeviceState* dev = nullptr;
+  DSA_TRY(device_setup(&dev));
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  float* scores = static_cast<float*>(ws);
+  int32_t* idx_ws =
+      idx_out ? nullptr : reinterpret_cast<int32_t*>(static_cast<char*>(ws) + rows * ld * 4);
+  const int bq = (decode || R->max_q_len <= 16) ? 16 : 64;
+  for (int64_t r0 = 0; r0 < R->total_q; r0 += rows) {
+    const int64_t cnt = std::min<int64_t>(rows, R->total_q - r0);
+    int32_t* idx = idx_out ? idx_out + r0 * K : idx_ws;
+    DSA_TRY(launch_index_scores(*dev, P, R, q_idx, k_idx, w, r0, cnt, scores, ld, bq, stream));
+    DSA_TRY(launch_topk(P, R, scores, ld, r0, cnt, idx, K, nullptr, stream));
+    DSA_TRY(launch_attn(P, R, q, k, v, idx, K, r0, cnt, gate, out, nullptr, err_count, stream));
+  }
+  return DSA_OK;
+}
+
+}  // namespace
+}  // namespace dsa
+
+using namespace dsa;
+
+extern "C" {
+
+const char* dsa_status_string(dsa_status s) {
+  switch (s) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARG: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case DSA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case DSA_ERR_CUDA: return "CUDA error";
+    case DSA_ERR_TIMEOUT: return "bounded device wait timed out";
+  }
+  return "unknown status";
+}
+
+int32_t dsa_version(void) { return 100; }
+
+dsa_status dsa_index_scores(const dsa_params* P, const dsa_ragged* R, const void* q_idx,
+                            const void* k_idx, const float* w, int64_t q_begin, int64_t q_count,
+                            float* scores, int64_t ld, void* stream) {
+  DSA_TRY(check_common(P, R));
+  DSA_TRY(check_indexer(P));
+  if (!q_idx || !k_idx || !w || !scores) return DSA_ERR_INVALID_ARG;
+  if (q_begin < 0 || q_count < 0 || q_begin + q_count > R->total_q) return DSA_ERR_INVALID_ARG;
+  if (ld < R->max_kv_len || ld % 4 != 0) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx)) return DSA_ERR_INVALID_ARG;
+  DeviceState* dev = nullptr;
+  DSA_TRY(device_setup(&dev));
+  const int bq = R->max_q_len <= 16 ? 16 : 64;
+  return launch_index_scores(*dev, P, R, q_idx, k_idx, w, q_begin, q_count, scores, ld, bq,
+                             static_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_topk(const dsa_params* P, const dsa_ragged* R, const float* scores, int64_t ld,
+                    int64_t q_begin, int64_t q_count, int32_t* idx, int64_t ld_idx, int32_t* cnt,
+                    void* stream) {
+  DSA_TRY(check_common(P, R));
+  if (!scores || !idx) return DSA_ERR_INVALID_ARG;
+  if (q_begin < 0 || q_count < 0 || q_begin + q_count > R->total_q) return DSA_ERR_INVALID_ARG;
+  if (ld < R->max_kv_len || ld % 4 != 0 || !aligned16(scores)) return DSA_ERR_INVALID_ARG;
+  if (ld_idx < P->top_k) return DSA_ERR_INVALID_ARG;
+  if (q_count > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  DeviceState* dev = nullptr;
+  DSA_TRY(device_setup(&dev));
+  return launch_topk(P, R, scores, ld, q_begin, q_count, idx, ld_idx, cnt,
+                     static_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_sparse_attn_gated(const dsa_params* P, const dsa_ragged* R, const void* q,
+                                 const void* k_cache, const void* v_cache, const int32_t* idx,
+                                 int64_t ld_idx, int64_t q_begin, int64_t q_count,
+                                 const void* gate, void* out, float* lse, int32_t* err_count,
+                                 void* stream) {
+  DSA_TRY(check_common(P, R));
+  DSA_TRY(check_attn(P));
+  if (!q || !k_cache || !v_cache || !idx || !out) return DSA_ERR_INVALID_ARG;
+  if (q_begin < 0 || q_count < 0 || q_begin + q_count > R->total_q) return DSA_ERR_INVALID_ARG;
+  if (ld_idx < P->top_k) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+      (gate && !aligned16(gate)))
+    return DSA_ERR_INVALID_ARG;
+  if (q_count > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  DeviceState* dev = nullptr;
+  DSA_TRY(device_setup(&dev));
+  return launch_attn(P, R, q, k_cache, v_cache, idx, ld_idx, q_begin, q_count, gate, out, lse,
+                     err_count, static_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_workspace_size(const dsa_params* P, const dsa_ragged* R, int is_decode,
+                              size_t* min_bytes, size_t* rec_bytes) {
+  (void)is_decode;
+  DSA_TRY(check_common(P, R));
+  const int64_t ld = scores_ld(R);
+  const int64_t row = ld * 4 + round_up((int64_t)P->top_k * 4, 16);
+  if (min_bytes) *min_bytes = (size_t)row;
+  if (rec_bytes) {
+    // enough rows per pass to fill the GPU many times over, bounded at 1 GiB
+    int64_t rows = std::max<int64_t>(1, std::min<int64_t>(R->total_q, (1ll << 30) / row));
+    *rec_bytes = (size_t)(rows * row);
+  }
+  return DSA_OK;
+}
+
+dsa_status dsa_prefill(const dsa_params* P, const dsa_ragged* R, const void* q_idx,
+                       const void* k_idx, const float* w, const void* q, const void* k_cache,
+                       const void* v_cache, const void* gate, void* out, int32_t* idx_out,
+                       int32_t* err_count, void* workspace, size_t ws_bytes, void* stream) {
+  return run_layer(P, R, q_idx, k_idx, w, q, k_cache, v_cache, gate, out, idx_out, err_count,
+                   workspace, ws_bytes, stream, false);
+}
+
+dsa_status dsa_decode(const dsa_params* P, const dsa_ragged* R, const void* q_idx,
+                      const void* k_idx, const float* w, const void* q, const void* k_cache,
+                      const void* v_cache, const void* gate, void* out, int32_t* idx_out,
+                      int32_t* err_count, void* workspace, size_t ws_bytes, void* stream) {
+  return run_layer(P, R, q_idx, k_idx, w, q, k_cache, v_cache, gate, out, idx_out, err_count,
+                   workspace, ws_bytes, stream, true);
+}
+
+dsa_status dsa_device_status(void* stream, int32_t* status, int clear) {
+  if (!status) return DSA_ERR_INVALID_ARG;
+  DeviceState* dev = nullptr;
+  DSA_TRY(device_setup(&dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, dev->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  *status = v;
+  if (clear && v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(dev->status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+      return DSA_ERR_CUDA;
+  }
+  return DSA_OK;
+}
+
+int64_t dsa_launch_count(void) { return t_launches; }
+
+dsa_status dsa_stage_timing(int enable) {
+  t_timing = enable != 0;
+  return DSA_OK;
+}
+
+dsa_status dsa_stage_times(double* ms, int64_t* launches, int reset) {
+  for (auto& rec : t_pending) {
+    if (cudaEventSynchronize(rec.stop) != cudaSuccess) return DSA_ERR_CUDA;
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, rec.start, rec.stop) != cudaSuccess) return DSA_ERR_CUDA;
+    t_stage_ms[rec.stage] += t;
+    t_free_events.push_back(rec.start);
+    t_free_events.push_back(rec.stop);
+  }
+  t_pending.clear();
+  for (int s = 0; s < 3; ++s) {
+    if (ms) ms[s] = t_stage_ms[s];
+    if (launches) launches[s] = t_stage_launches[s];
+    if (reset) {
+      t_stage_ms[s] = 0;
+      t_stage_launches[s] = 0;
+    }
+  }
+  return DSA_OK;
+}
+
+}  // extern "C"

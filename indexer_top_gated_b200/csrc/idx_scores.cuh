@@ -1,0 +1,310 @@
+// idx_scores.cuh - step 1 of the layer, the indexer, on tcgen05 tensor cores.
+//
+//   s[t, j] = sum_h w_h * max(0, c * q_idx[t,h,:] . k_idx[j,h,:]),   j = 0..p(t)
+//
+// Design (sm_100a):
+//  - One CTA owns a tile of BQ consecutive packed query rows (BQ = 64 for prefill,
+//    16 when sequences have one query each) and a range of 128-position key tiles.
+//  - The key tile is the MMA's M side (128 TMEM lanes = 128 key positions) and the
+//    query tile its N side, so in the epilogue each warp holds 32 consecutive key
+//    positions of one query row: every score store is a coalesced 128-byte line.
+//  - Warp 0 issues TMA loads (128-byte swizzled, one box per indexer head) into a
+//    3-stage ring; warp 1 issues tcgen05.mma (one per head and 16-wide K step) into one
+//    of two TMEM accumulator buffers; warps 2-5 drain TMEM (tcgen05.ld), apply ReLU,
+//    the head weights and the head sum, mask causally and store fp32 scores.
+//  - Tiles may straddle sequences of a ragged batch: the CTA runs one pass per
+//    sequence it touches and masks the other rows.  Tiles are scheduled largest
+//    first (the last rows of a sequence see the most keys).
+//  - Every wait is bounded; on a timeout the CTA records it, waits (bounded) for its
+//    own copies and MMAs in flight, frees TMEM and returns.
+#pragma once
+
+#include "common.cuh"
+
+namespace dsa {
+
+struct IdxArgs {
+  const int32_t* q_offsets;
+  const int32_t* kv_offsets;
+  int batch;
+  int n_heads;         // H_i (<= 4)
+  int64_t q_begin;     // first packed query row of this launch
+  int64_t q_count;     // rows in this launch
+  int n_tiles;         // ceil(q_count / BQ)
+  int kt_per_split;    // key tiles per blockIdx.y
+  const float* w;
+  int w_row_stride;
+  float scale;         // idx_scale_q * idx_scale_k
+  float* scores;
+  int64_t ld;
+  int* status;
+};
+
+constexpr int kIdxStages = 3;
+constexpr int kIdxKeyTile = 128;
+constexpr int kIdxThreads = 192;
+
+template <bool FP8>
+struct IdxGeom {
+  static constexpr int kRowBytes = FP8 ? 64 : 128;   // D_i = 64 elements
+  static constexpr int kKStep = FP8 ? 32 : 16;       // MMA K per instruction
+  static constexpr int kKSteps = 64 / kKStep;
+  static constexpr uint32_t kLayout = FP8 ? 4u : 2u; // 64B / 128B swizzle
+  static constexpr uint32_t kSbo = 8 * kRowBytes;    // 8-row group stride
+};
+
+__host__ __device__ inline int idx_tmem_cols(int n_heads, int bq) {
+  int need = 2 * n_heads * bq;
+  int c = 32;
+  while (c < need) c <<= 1;
+  return c;
+}
+
+// Dynamic shared memory of one CTA.  A CTA whose TMEM allocation exceeds a quarter of
+// the 512 columns asks for enough shared memory that CTAs sharing an SM can never
+// oversubscribe TMEM (an allocation that cannot be met would block).
+__host__ inline size_t idx_smem_bytes(int n_heads, int bq, bool fp8) {
+  size_t row = fp8 ? 64 : 128;
+  size_t q = (size_t)n_heads * bq * row;
+  size_t k = (size_t)kIdxStages * n_heads * kIdxKeyTile * row;
+  size_t bytes = 1024 /*align slack*/ + q + k + 256 /*barriers*/;
+  const int cols = idx_tmem_cols(n_heads, bq);
+  if (cols > 256 && bytes < 120 * 1024) bytes = 120 * 1024;       // 1 CTA per SM
+  else if (cols > 128 && bytes < 80 * 1024) bytes = 80 * 1024;    // <= 2 CTAs per SM
+  else if (cols > 64 && bytes < 58 * 1024) bytes = 58 * 1024;     // <= 3 CTAs per SM
+  return bytes;
+}
+
+template <int BQ, bool FP8>
+__global__ void __launch_bounds__(kIdxThreads, 1)
+    idx_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                      const __grid_constant__ CUtensorMap tmap_k, IdxArgs a) {
+  using Geo = IdxGeom<FP8>;
+  constexpr int ST = kIdxStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int H = a.n_heads;
+  const uint32_t q_head_bytes = BQ * Geo::kRowBytes;
+  const uint32_t k_head_bytes = kIdxKeyTile * Geo::kRowBytes;
+  uint8_t* sQ = smem;
+  uint8_t* sK = smem + H * q_head_bytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sK + (size_t)ST * H * k_head_bytes);
+  uint64_t* full = bars;            // [ST]
+  uint64_t* empty = bars + ST;      // [ST]
+  uint64_t* tfull = bars + 2 * ST;  // [2]
+  uint64_t* tempty = tfull + 2;     // [2]
+  uint64_t* qfull = tempty + 2;     // [1]
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_bfirst, s_blast;
+  __shared__ volatile int s_abort;
+  __shared__ int s_consumed;  // jobs whose smem stage the MMA warp has released
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = lane_id();
+  const int tile = a.n_tiles - 1 - (int)blockIdx.x;  // largest first
+  const int64_t r0 = a.q_begin + (int64_t)tile * BQ;
+  const int64_t q_end = a.q_begin + a.q_count;
+  const int64_t r_last = (r0 + BQ < q_end ? r0 + BQ : q_end) - 1;
+  const int kt_lo = (int)blockIdx.y * a.kt_per_split;
+
+  if (threadIdx.x == 0) {
+    s_bfirst = seq_of_row(a.q_offsets, a.batch, r0);
+    s_blast = seq_of_row(a.q_offsets, a.batch, r_last);
+    s_abort = 0;
+    s_consumed = 0;
+  }
+  __syncthreads();
+  const int b_first = s_bfirst, b_last = s_blast;
+
+  // Jobs of this CTA: for each sequence b in the tile, key tiles [kt_lo, kt_hi(b)).
+  auto seq_range = [&](int b, int64_t& rs, int64_t& re, int& kt_hi, int64_t& pbase) -> bool {
+    int64_t qo = __ldg(a.q_offsets + b), qn = __ldg(a.q_offsets + b + 1);
+    int64_t ko = __ldg(a.kv_offsets + b), kn = __ldg(a.kv_offsets + b + 1);
+    rs = r0 > qo ? r0 : qo;
+    re = (r_last + 1) < qn ? (r_last + 1) : qn;
+    if (rs >= re) return false;
+    pbase = (kn - ko) - (qn - qo) - qo;  // p(r) = pbase + r
+    int64_t pmax = pbase + re - 1;
+    if (pmax < 0) return false;
+    int n_kt = (int)(pmax / kIdxKeyTile) + 1;
+    kt_hi = n_kt < kt_lo + a.kt_per_split ? n_kt : kt_lo + a.kt_per_split;
+    return kt_lo < kt_hi;
+  };
+
+  int n_jobs = 0;
+  for (int b = b_first; b <= b_last; ++b) {
+    int64_t rs, re, pb;
+    int kh;
+    if (seq_range(b, rs, re, kh, pb)) n_jobs += kh - kt_lo;
+  }
+  if (n_jobs == 0) return;  // uniform across the CTA
+
+  const int ncols = idx_tmem_cols(H, BQ);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&tfull[i]), 1);
+      mbar_init(smem_u32(&tempty[i]), 4);
+    }
+    mbar_init(smem_u32(qfull), 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&s_tmem), (uint32_t)ncols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmap_q);
+      prefetch_tensormap(&tmap_k);
+      mbar_arrive_expect_tx(smem_u32(qfull), H * q_head_bytes);
+      for (int h = 0; h < H; ++h)
+        tma_load_2d(smem_u32(sQ + h * q_head_bytes), &tmap_q, smem_u32(qfull), h * 64, (int)r0);
+      int i = 0;
+      bool ok = true;
+      for (int b = b_first; b <= b_last && ok; ++b) {
+        int64_t rs, re, pb;
+        int kh;
+        if (!seq_range(b, rs, re, kh, pb)) continue;
+        const int64_t kbase = __ldg(a.kv_offsets + b);
+        for (int kt = kt_lo; kt < kh; ++kt, ++i) {
+          const int s = i % ST;
+          if (!mbar_wait_bounded(smem_u32(&empty[s]), ((i / ST) & 1) ^ 1, a.status, &s_abort)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(smem_u32(&full[s]), H * k_head_bytes);
+          for (int h = 0; h < H; ++h)
+            tma_load_2d(smem_u32(sK + ((size_t)s * H + h) * k_head_bytes), &tmap_k,
+                        smem_u32(&full[s]), h * 64, (int)(kbase + (int64_t)kt * kIdxKeyTile));
+        }
+      }
+      if (!ok) {
+        // drain: every issued load lands before the CTA exits
+        mbar_wait_bounded(smem_u32(qfull), 0, nullptr, nullptr);
+        for (int j = s_consumed; j < i; ++j)
+          mbar_wait_bounded(smem_u32(&full[j % ST]), (j / ST) & 1, nullptr, nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t idesc = umma_idesc(128, BQ, FP8 ? 0u : 1u);
+    int i = 0;
+    int issued = 0;
+    bool ok = mbar_wait_bounded(smem_u32(qfull), 0, a.status, &s_abort);
+    for (int b = b_first; b <= b_last && ok; ++b) {
+      int64_t rs, re, pb;
+      int kh;
+      if (!seq_range(b, rs, re, kh, pb)) continue;
+      for (int kt = kt_lo; kt < kh; ++kt, ++i) {
+        const int s = i % ST, buf = i & 1;
+        if (!mbar_wait_bounded(smem_u32(&full[s]), (i / ST) & 1, a.status, &s_abort) ||
+            !mbar_wait_bounded(smem_u32(&tempty[buf]), ((i >> 1) & 1) ^ 1, a.status, &s_abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          for (int h = 0; h < H; ++h) {
+            const uint32_t a_base = smem_u32(sK + ((size_t)s * H + h) * k_head_bytes);
+            const uint32_t b_base = smem_u32(sQ + h * q_head_bytes);
+            const uint32_t d = tmem + (uint32_t)(buf * H * BQ + h * BQ);
+#pragma unroll
+            for (int kk = 0; kk < Geo::kKSteps; ++kk) {
+              const uint64_t ad = umma_smem_desc(a_base + kk * 32, Geo::kSbo, Geo::kLayout);
+              const uint64_t bd = umma_smem_desc(b_base + kk * 32, Geo::kSbo, Geo::kLayout);
+              if (FP8) umma_fp8(d, ad, bd, idesc, kk > 0);
+              else umma_bf16(d, ad, bd, idesc, kk > 0);
+            }
+          }
+          umma_commit(smem_u32(&empty[s]));
+          umma_commit(smem_u32(&tfull[buf]));
+        }
+        __syncwarp();
+        issued = i + 1;
+        if (lane == 0) s_consumed = i + 1;
+      }
+    }
+    if (!ok && issued > 0 && lane == 0) {
+      // the last commit completes after every MMA issued before it
+      const int j = issued - 1;
+      mbar_wait_bounded(smem_u32(&tfull[j & 1]), (j >> 1) & 1, nullptr, nullptr);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2-5)
+    const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    float wsh[4] = {0.f, 0.f, 0.f, 0.f};
+    if (a.w_row_stride == 0)
+      for (int h = 0; h < H; ++h) wsh[h] = __ldg(a.w + h);
+    int i = 0;
+    bool ok = true;
+    for (int b = b_first; b <= b_last && ok; ++b) {
+      int64_t rs, re, pbase;
+      int kh;
+      if (!seq_range(b, rs, re, kh, pbase)) continue;
+      for (int kt = kt_lo; kt < kh; ++kt, ++i) {
+        const int buf = i & 1;
+        if (!mbar_wait_bounded(smem_u32(&tfull[buf]), (i >> 1) & 1, a.status, &s_abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int64_t j = (int64_t)kt * kIdxKeyTile + quad * 32 + lane;  // key position
+        // columns c of this tile that belong to sequence b: rows rs..re-1
+        const int c_lo = (int)(rs - r0), c_hi = (int)(re - r0);
+        for (int c0 = (c_lo / 16) * 16; c0 < c_hi; c0 += 16) {
+          // skip chunks whose rows all precede this key tile (causal)
+          const int64_t p_chunk_max = pbase + r0 + (c0 + 15 < c_hi - 1 ? c0 + 15 : c_hi - 1);
+          if (p_chunk_max < (int64_t)kt * kIdxKeyTile) continue;
+          float acc[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) acc[c] = 0.f;
+          for (int h = 0; h < H; ++h) {
+            float v[16];
+            tmem_ld16(tmem + lane_base + (uint32_t)(buf * H * BQ + h * BQ + c0), v);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              float wv = wsh[h];
+              if (a.w_row_stride != 0) {
+                int64_t r = r0 + c0 + c;
+                if (r > r_last) r = r_last;
+                wv = __ldg(a.w + r * a.w_row_stride + h);
+              }
+              acc[c] = fmaf(wv, fmaxf(v[c] * a.scale, 0.f), acc[c]);
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int cc = c0 + c;
+            const int64_t r = r0 + cc;
+            if (cc >= c_lo && cc < c_hi && j <= pbase + r && j < a.ld)
+              a.scores[(r - a.q_begin) * a.ld + j] = acc[c];
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&tempty[buf]));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, (uint32_t)ncols);
+  }
+}
+
+}  // namespace dsa

@@ -1,0 +1,123 @@
+"""CPU-side checks of the C-ABI library: it builds, loads, exports every declared entry
+point, and rejects bad arguments on the host before any CUDA call is made."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dsa_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for required in ("dsa_index_scores", "dsa_topk", "dsa_sparse_attn_gated", "dsa_prefill",
+                     "dsa_decode", "dsa_workspace_size", "dsa_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    import indexer_top_gated_b200 as dsa
+    lib = ctypes.CDLL(dsa.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", dsa.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    exported = set(re.findall(r"\bT (dsa_\w+)", out))
+    assert set(_declared()) <= exported
+    assert set(dsa.EXPORTS) == set(_declared())
+
+
+def test_status_strings_and_version():
+    import indexer_top_gated_b200 as dsa
+    assert dsa.status_string(0) == "ok"
+    assert "workspace" in dsa.status_string(dsa.DSA_ERR_WORKSPACE)
+    assert dsa.lib.dsa_version() >= 100
+
+
+class _FakeTensor:
+    """Stands in for a device tensor: only its address is read on the host path."""
+
+    def __init__(self, addr, nbytes=1 << 20):
+        self.addr, self.nbytes = addr, nbytes
+
+    def data_ptr(self):
+        return self.addr
+
+    def numel(self):
+        return self.nbytes
+
+    def element_size(self):
+        return 1
+
+
+def _rg(dsa, batch=1, max_q=8, max_kv=8):
+    return dsa.Ragged(batch, 0x1000, 0x2000, max_q, max_kv, max_q * batch, max_kv * batch)
+
+
+def test_host_validation_rejects_bad_arguments():
+    import indexer_top_gated_b200 as dsa
+    L = dsa.lib
+    good = dsa.LayerShape(top_k=4)
+    rg = _rg(dsa)
+    P = good.params()
+    null = None
+    A = 0x10000  # 16-byte aligned fake addresses; never dereferenced on these paths
+    # bad K
+    bad = dsa.LayerShape(top_k=0).params()
+    assert L.dsa_topk(ctypes.byref(bad), ctypes.byref(rg), A, 8, 0, 1, A, 4, null, null) == \
+        dsa.DSA_ERR_UNSUPPORTED
+    # scores leading dimension not a multiple of 4 / too small
+    assert L.dsa_topk(ctypes.byref(P), ctypes.byref(rg), A, 6, 0, 1, A, 4, null, null) == \
+        dsa.DSA_ERR_INVALID_ARG
+    assert L.dsa_topk(ctypes.byref(P), ctypes.byref(rg), A, 4, 0, 1, A, 4, null, null) == \
+        dsa.DSA_ERR_INVALID_ARG
+    # row range outside the batch
+    assert L.dsa_topk(ctypes.byref(P), ctypes.byref(rg), A, 8, 4, 5, A, 4, null, null) == \
+        dsa.DSA_ERR_INVALID_ARG
+    # idx leading dimension below K
+    assert L.dsa_topk(ctypes.byref(P), ctypes.byref(rg), A, 8, 0, 1, A, 3, null, null) == \
+        dsa.DSA_ERR_INVALID_ARG
+    # unsupported indexer dim / head dim / GQA layout
+    for shape in (dsa.LayerShape(idx_dim=32), dsa.LayerShape(n_idx_heads=5)):
+        p = shape.params()
+        assert L.dsa_index_scores(ctypes.byref(p), ctypes.byref(rg), A, A, A, 0, 1, A, 8, null) \
+            == dsa.DSA_ERR_UNSUPPORTED
+    for shape, code in ((dsa.LayerShape(head_dim=64), dsa.DSA_ERR_UNSUPPORTED),
+                        (dsa.LayerShape(n_q_heads=30, n_kv_heads=4), dsa.DSA_ERR_INVALID_ARG),
+                        (dsa.LayerShape(n_q_heads=64, n_kv_heads=2), dsa.DSA_ERR_UNSUPPORTED),
+                        (dsa.LayerShape(n_q_heads=12, n_kv_heads=3), dsa.DSA_ERR_UNSUPPORTED)):
+        p = shape.params()
+        assert L.dsa_sparse_attn_gated(ctypes.byref(p), ctypes.byref(rg), A, A, A, A, 2048, 0, 1,
+                                       null, A, null, null, null) == code
+    # misaligned tensors
+    p = dsa.LayerShape(top_k=4).params()
+    assert L.dsa_sparse_attn_gated(ctypes.byref(p), ctypes.byref(rg), A + 2, A, A, A, 4, 0, 1,
+                                   null, A, null, null, null) == dsa.DSA_ERR_INVALID_ARG
+    # workspace missing / misaligned / too small
+    for ws, nbytes in ((None, 1 << 20), (A + 16, 1 << 20), (A, 8)):
+        rc = L.dsa_prefill(ctypes.byref(p), ctypes.byref(rg), A, A, A, A, A, A, null, A, null,
+                           null, ws, nbytes, null)
+        assert rc == dsa.DSA_ERR_WORKSPACE, (ws, nbytes, rc)
+    # decode needs one query per sequence
+    rg2 = _rg(dsa, batch=2, max_q=3)
+    assert L.dsa_decode(ctypes.byref(p), ctypes.byref(rg2), A, A, A, A, A, A, null, A, null, null,
+                        A, 1 << 20, null) == dsa.DSA_ERR_INVALID_ARG
+    # null ragged / params
+    assert L.dsa_topk(None, ctypes.byref(rg), A, 8, 0, 1, A, 4, null, null) == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_workspace_size_is_host_only():
+    import indexer_top_gated_b200 as dsa
+    shape = dsa.LayerShape(top_k=2048)
+    rg = dsa.Ragged(1, 0x1000, 0x2000, 32768, 32768, 32768, 32768)
+    mn, rec = dsa.dsa_workspace_size(shape, rg)
+    assert mn == 32768 * 4 + 2048 * 4
+    assert mn <= rec <= (1 << 30) + mn
