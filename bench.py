@@ -86,6 +86,17 @@ def algorithmic(w):
     }
 
 
+def aggregate_max(ms_local: float, tokens_per_rank: int, world: int, device="cuda"):
+    """Whole-job throughput: tokens of all ranks over the slowest rank's time (max over ranks)."""
+    import torch
+    t = torch.tensor([ms_local], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    return ms_max, tokens_per_rank * world / (ms_max / 1e3)
+
+
 def source_sha(paths):
     h = hashlib.sha256()
     for p in paths:
@@ -231,12 +242,7 @@ def run_ours(args, rank, world, local_rank):
     assert status == 0, f"device status {status}"
     assert int(err.item()) == 0
 
-    t = torch.tensor([ms_total], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
-    tokens = w.total_q * world * args.steps
-    value = tokens / (ms_max / 1e3)
+    ms_max, value = aggregate_max(ms_total, w.total_q * args.steps, world)
 
     # ---- end to end through the C ABI with host buffers
     e2e = None
@@ -264,12 +270,10 @@ def run_ours(args, rank, world, local_rank):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device="cuda")
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": w.total_q * world * n_e2e / (float(te.item()) / 1e3), "unit": "tokens/s",
+        te_ms, te_val = aggregate_max(e0.elapsed_time(e1), w.total_q * n_e2e, world)
+        e2e = {"value": te_val, "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "steps": n_e2e, "ms_per_step": float(te.item()) / n_e2e}
+               "steps": n_e2e, "ms_per_step": te_ms / n_e2e}
 
     result = {
         "w": w, "value": value, "ms_total": ms_max, "launches": launches,
