@@ -34,8 +34,9 @@
  *
  * Conventions for every entry point
  *  - Ownership: the caller owns every buffer and the stream.  The library never
- *    allocates device memory; scratch comes from a caller-provided workspace.  The
- *    library keeps no per-call state and may be called from several host threads.
+ *    allocates device memory; scratch comes from a caller-provided workspace (or, for
+ *    dsa_decode_noalloc only, a fixed array inside the library).  The library keeps no
+ *    per-call state and may be called from several host threads.
  *  - Synchrony: every compute call is asynchronous on `stream` (a cudaStream_t; NULL
  *    is the legacy default stream).  Argument errors are returned before anything is
  *    launched; a failed launch returns DSA_ERR_CUDA.  No exception crosses the ABI.
@@ -194,6 +195,32 @@ dsa_status dsa_decode(const dsa_params* params, const dsa_ragged* ragged, const 
                       const void* k_idx, const float* w, const void* q, const void* k_cache,
                       const void* v_cache, const void* gate, void* out, int32_t* idx_out,
                       int32_t* err_count, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * dsa_decode without a workspace argument, for callers that cannot allocate device
+ * memory: code embedded in a host framework whose allocator owns the whole device
+ * (a side allocation would break its accounting or pools), decode loops that must not
+ * allocate after warm-up because an allocation can synchronise the device, and plugin
+ * interfaces that hand over tensors but no allocator.  The pages have no counterpart;
+ * this is a deployment convenience.
+ *   Arguments and outputs are those of dsa_decode minus workspace / ws_bytes.
+ *   Scratch: a fixed 32 MiB array inside the library on each device (reserved on every
+ *   GPU that loads the library until the process exits).  The layer runs in as many
+ *   passes as that needs; a single query row must fit, i.e. 4 * roundup(max_kv_len, 32)
+ *   (+ 4 * K when idx_out is NULL) <= 32 MiB, otherwise DSA_ERR_WORKSPACE is returned
+ *   before anything is launched (max_kv_len up to about 8.3 million at K = 2048).
+ *   This entry point calls no cudaMalloc, cudaFree or other allocating routine.
+ *   The first call on a device looks up the scratch's device address
+ *   (cudaGetSymbolAddress), so make that first call before any stream capture.
+ *   All calls on a device share the one scratch array: calls that can overlap on the
+ *   GPU (different streams, or different host threads) race and must be serialised by
+ *   the caller.  No part of the scratch needs to be zeroed between calls.
+ */
+dsa_status dsa_decode_noalloc(const dsa_params* params, const dsa_ragged* ragged,
+                              const void* q_idx, const void* k_idx, const float* w,
+                              const void* q, const void* k_cache, const void* v_cache,
+                              const void* gate, void* out, int32_t* idx_out, int32_t* err_count,
+                              void* stream);
 
 /*
  * Device status word of the current device: synchronises `stream`, stores the status

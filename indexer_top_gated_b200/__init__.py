@@ -53,6 +53,7 @@ EXPORTS = [
     "dsa_status_string", "dsa_version", "dsa_index_scores", "dsa_topk",
     "dsa_sparse_attn_gated", "dsa_workspace_size", "dsa_prefill", "dsa_decode",
     "dsa_device_status", "dsa_launch_count", "dsa_stage_timing", "dsa_stage_times",
+    "dsa_decode_noalloc",
 ]
 
 
@@ -71,13 +72,15 @@ def _load():
     L.dsa_workspace_size.argtypes = [PP, RP, ctypes.c_int, ctypes.POINTER(sz), ctypes.POINTER(sz)]
     L.dsa_prefill.argtypes = [PP, RP, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.dsa_decode.argtypes = L.dsa_prefill.argtypes
+    L.dsa_decode_noalloc.argtypes = [PP, RP, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     L.dsa_device_status.argtypes = [vp, ctypes.POINTER(i32), ctypes.c_int]
     L.dsa_launch_count.argtypes = []
     L.dsa_launch_count.restype = i64
     L.dsa_stage_timing.argtypes = [ctypes.c_int]
     L.dsa_stage_times.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64), ctypes.c_int]
     for name in ("dsa_index_scores", "dsa_topk", "dsa_sparse_attn_gated", "dsa_workspace_size",
-                 "dsa_prefill", "dsa_decode", "dsa_device_status", "dsa_stage_timing",
+                 "dsa_prefill", "dsa_decode", "dsa_decode_noalloc", "dsa_device_status",
+                 "dsa_stage_timing",
                  "dsa_stage_times"):
         getattr(L, name).restype = ctypes.c_int
     return L
@@ -187,6 +190,16 @@ def dsa_decode(shape: LayerShape, rg: Ragged, q_idx, k_idx, w, q, k_cache, v_cac
                idx_out=None, err_count=None, workspace=None, ws_bytes=None, stream=None):
     _layer(lib.dsa_decode, "dsa_decode", shape, rg, q_idx, k_idx, w, q, k_cache, v_cache, gate,
            out, idx_out, err_count, workspace, ws_bytes, stream)
+
+
+def dsa_decode_noalloc(shape: LayerShape, rg: Ragged, q_idx, k_idx, w, q, k_cache, v_cache, gate,
+                       out, idx_out=None, err_count=None, stream=None):
+    """dsa_decode whose scratch is the library's fixed per-device array (no allocation)."""
+    p = shape.params()
+    _check(lib.dsa_decode_noalloc(ctypes.byref(p), ctypes.byref(rg), _ptr(q_idx), _ptr(k_idx),
+                                  _ptr(w), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(gate),
+                                  _ptr(out), _ptr(idx_out), _ptr(err_count), _stream(stream)),
+           "dsa_decode_noalloc")
 
 
 def dsa_device_status(clear: bool = True, stream=None) -> int:

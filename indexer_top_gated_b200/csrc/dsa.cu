@@ -448,6 +448,52 @@ dsa_status dsa_decode(const dsa_params* P, const dsa_ragged* R, const void* q_id
                    workspace, ws_bytes, stream, true);
 }
 
+// ---------------------------------------------------------------- allocation-free decode
+//
+// Scratch for dsa_decode_noalloc: one fixed array in the library's own device memory,
+// so callers that cannot allocate never have to.  It is reserved on every GPU that
+// loads the library and kept until the process exits.  Host code must not pass the
+// symbol itself to a kernel (on the host it names a stand-in, not device memory): the
+// first call on each device looks up its device address with cudaGetSymbolAddress.
+namespace dsa {
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB per device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+dsa_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr)
+      return DSA_ERR_CUDA;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return DSA_OK;
+}
+}  // namespace
+}  // namespace dsa
+
+dsa_status dsa_decode_noalloc(const dsa_params* P, const dsa_ragged* R, const void* q_idx,
+                              const void* k_idx, const float* w, const void* q,
+                              const void* k_cache, const void* v_cache, const void* gate,
+                              void* out, int32_t* idx_out, int32_t* err_count, void* stream) {
+  DSA_TRY(check_common(P, R));
+  // one query row of scores (and its index row) must fit the fixed scratch
+  const int64_t row = scores_ld(R) * 4 + (idx_out ? 0 : round_up((int64_t)P->top_k * 4, 16));
+  if (row > (int64_t)kNoAllocScratchBytes) return DSA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  DSA_TRY(noalloc_scratch(&scratch));
+  // Nothing in the scratch has to start at zero: each pass writes every score and index
+  // entry it later reads.
+  return run_layer(P, R, q_idx, k_idx, w, q, k_cache, v_cache, gate, out, idx_out, err_count,
+                   scratch, kNoAllocScratchBytes, stream, true);
+}
+
 dsa_status dsa_device_status(void* stream, int32_t* status, int clear) {
   if (!status) return DSA_ERR_INVALID_ARG;
   DeviceState* dev = nullptr;
