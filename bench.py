@@ -48,7 +48,14 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target wall time of the CPU-baseline sample")
-    return ap.parse_args()
+    ap.add_argument("--ws-rows", type=int, default=0,
+                    help="cap the workspace at this many query rows per pass (profiling)")
+    ap.add_argument("--lean", action="store_true",
+                    help="only the timed region: no e2e, decode or CPU-baseline legs")
+    a = ap.parse_args()
+    if a.lean:
+        a.no_e2e = a.no_decode = a.no_cpu_baseline = True
+    return a
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -202,7 +209,9 @@ def run_ours(args, rank, world, local_rank):
     rg = dsa.ragged(inputs["q_offsets"], inputs["kv_offsets"], w.q_lens, w.kv_lens)
     decode = max(w.q_lens) == 1
     layer = dsa.dsa_decode if decode else dsa.dsa_prefill
-    _, ws_bytes = dsa.dsa_workspace_size(shape, rg, decode)
+    ws_min, ws_bytes = dsa.dsa_workspace_size(shape, rg, decode)
+    if args.ws_rows > 0:
+        ws_bytes = min(ws_bytes, ws_min * args.ws_rows)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
     out = torch.empty((w.total_q, w.n_q_heads, w.head_dim), dtype=torch.bfloat16, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")

@@ -105,7 +105,7 @@ dsa_status device_setup(DeviceState** out) {
     e = e ? e : allow_smem(idx_scores_kernel<16, false>, idx_max);
     e = e ? e : allow_smem(idx_scores_kernel<64, true>, idx_max);
     e = e ? e : allow_smem(idx_scores_kernel<16, true>, idx_max);
-    e = e ? e : allow_smem(topk_kernel, kTopkStageCap * sizeof(uint32_t));
+    e = e ? e : allow_smem(topk_kernel, topk_smem_bytes(kTopkStageCap));
     e = e ? e : allow_smem(sparse_attn_kernel<1, 1>, attn_smem_bytes());
     e = e ? e : allow_smem(sparse_attn_kernel<2, 1>, attn_smem_bytes());
     e = e ? e : allow_smem(sparse_attn_kernel<4, 1>, attn_smem_bytes());
@@ -248,8 +248,7 @@ dsa_status launch_topk(const dsa_params* P, const dsa_ragged* R, const float* sc
   a.idx = idx;
   a.ld_idx = ld_idx;
   a.cnt = cnt;
-  const size_t smem =
-      (size_t)std::min<int64_t>(kTopkStageCap, (int64_t)R->max_kv_len + 4) * sizeof(uint32_t);
+  const size_t smem = topk_smem_bytes(R->max_kv_len);
   StageScope scope(1, stream);
   topk_kernel<<<(unsigned)q_count, kTopkThreads, smem, stream>>>(a);
   ++t_launches;

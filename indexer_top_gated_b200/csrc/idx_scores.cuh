@@ -267,12 +267,19 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           // skip chunks whose rows all precede this key tile (causal)
           const int64_t p_chunk_max = pbase + r0 + (c0 + 15 < c_hi - 1 ? c0 + 15 : c_hi - 1);
           if (p_chunk_max < (int64_t)kt * kIdxKeyTile) continue;
+          // all heads' TMEM loads in flight together, one wait
+          uint32_t v[4][16];
+#pragma unroll
+          for (int h = 0; h < 4; ++h)
+            if (h < H) tmem_ld16_async(tmem + lane_base + (uint32_t)(buf * H * BQ + h * BQ + c0), v[h]);
+          tmem_wait_ld();
           float acc[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) acc[c] = 0.f;
-          for (int h = 0; h < H; ++h) {
-            float v[16];
-            tmem_ld16(tmem + lane_base + (uint32_t)(buf * H * BQ + h * BQ + c0), v);
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            if (h >= H) break;
+            reg_fence(v[h]);
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
               float wv = wsh[h];
@@ -281,7 +288,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
                 if (r > r_last) r = r_last;
                 wv = __ldg(a.w + r * a.w_row_stride + h);
               }
-              acc[c] = fmaf(wv, fmaxf(v[c] * a.scale, 0.f), acc[c]);
+              acc[c] = fmaf(wv, fmaxf(__uint_as_float(v[h][c]) * a.scale, 0.f), acc[c]);
             }
           }
 #pragma unroll

@@ -109,25 +109,38 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(AttnArgs a
   if (tid == 0 && s_err && a.err_count && blockIdx.y == 0) atomicAdd(a.err_count, s_err);
   const int n_chunks = (s_last + CH) / CH;  // 0 when nothing is selected
 
-  // ---- gather of one chunk of selected positions into stage st
+  // ---- gather of one chunk of selected positions into stage st.  Each warp copies whole
+  // position rows: one (broadcast) index load per position, then every cp.async of the
+  // warp covers a contiguous 512-byte run of the row (K and V rows alike).
   auto load_chunk = [&](int c, int st) {
+    constexpr int CPR = HKV_CTA * 16;             // 16-byte pieces per position row
+    constexpr int LPP = CPR < 32 ? CPR : 32;      // lanes per position
+    constexpr int PPI = 32 / LPP;                 // positions per warp iteration
+    constexpr int PIECES = CPR / LPP;             // pieces per lane per position row
+    constexpr int PPW = CH / 8;                   // positions per warp per chunk
     uint8_t* base = smem + (size_t)st * Geo::kStageBytes;
-#pragma unroll 4
-    for (int it = 0; it < Geo::kPieces / kAttnThreads; ++it) {
-      const int flat = tid + kAttnThreads * it;
-      const int kv = flat / (Geo::kPieces / 2);
-      const int rem = flat % (Geo::kPieces / 2);
-      const int pos = rem / (HKV_CTA * 16);
-      const int ch = rem % (HKV_CTA * 16);  // (head, 8-dim chunk) within the row
+    const int sub_lane = lane % LPP;
+#pragma unroll
+    for (int it = 0; it < PPW / PPI; ++it) {
+      const int pos = warp * PPW + it * PPI + lane / LPP;
       const int e = c * CH + pos;
       const int j = e < K ? __ldg(irow + e) : -1;
       const bool valid = j >= 0 && (int64_t)j <= p;
-      const __nv_bfloat16* src = (kv ? a.v : a.k) +
-                                 ((kbase + (valid ? j : 0)) * a.Hkv + g0) * kHeadDim + ch * 8;
-      const uint32_t dst = smem_u32(base + kv * Geo::kHalfBytes + pos * ROWB +
-                                    ((ch ^ (pos & 7)) << 4));
-      cp_async_16(dst, valid ? (const void*)src : (const void*)a.k, valid ? 16u : 0u);
-      if (kv == 0 && ch == 0) s_valid[st][pos] = valid ? 1 : 0;
+      const int64_t row_elem = ((kbase + (valid ? j : 0)) * a.Hkv + g0) * kHeadDim;
+      const __nv_bfloat16* ksrc = a.k + row_elem;
+      const __nv_bfloat16* vsrc = a.v + row_elem;
+      uint8_t* kdst = base + pos * ROWB;
+      uint8_t* vdst = kdst + Geo::kHalfBytes;
+#pragma unroll
+      for (int q = 0; q < PIECES; ++q) {
+        const int ch = sub_lane + q * LPP;
+        const uint32_t off = (uint32_t)((ch ^ (pos & 7)) << 4);
+        cp_async_16(smem_u32(kdst + off), valid ? (const void*)(ksrc + ch * 8) : (const void*)a.k,
+                    valid ? 16u : 0u);
+        cp_async_16(smem_u32(vdst + off), valid ? (const void*)(vsrc + ch * 8) : (const void*)a.k,
+                    valid ? 16u : 0u);
+      }
+      if (sub_lane == 0) s_valid[st][pos] = valid ? 1 : 0;
     }
   };
 

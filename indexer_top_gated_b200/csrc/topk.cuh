@@ -2,16 +2,20 @@
 //
 // For a score row s[0..n) (n = p+1 causal candidates) and K < n:
 //  - every fp32 score becomes an order-preserving 32-bit key (-0.0 folded onto +0.0);
-//  - up to four MSB-first 8-bit digit passes build a 256-bin shared-memory histogram of
-//    the keys that still match the chosen prefix (warp-aggregated atomics: lanes with
-//    the same digit add once), and pick the bin holding the K-th largest key;
-//  - one ordered pass over positions then keeps every key above the threshold plus the
-//    first (K - count above) keys equal to it: a block-wide exclusive scan of packed
-//    (definite, tie) counts gives each kept position its output slot, so the output is
-//    in ascending position order and ties go to the lower position.
-// Rows of up to kTopkStageCap scores are staged in shared memory on the first pass, so
-// the row is read from global memory once; longer rows are re-read (from L2).
-// No sort, no global scratch.
+//  - pass A: a 4096-bin shared-memory histogram of the top 12 key bits over the whole row
+//    (the row is staged in shared memory on the way when it fits) picks the bin that
+//    holds the K-th largest key;
+//  - the keys of that bin (at most kTopkCandCap of them) are compacted into a candidate
+//    list, and two 1024-bin passes over the candidates alone settle the remaining 20 bits,
+//    giving the exact threshold key tau and how many keys equal to tau are still needed;
+//    a bin that is kept whole ends the search early;
+//  - one ordered pass over positions keeps every key above tau plus the first needed keys
+//    equal to it: a block-wide exclusive scan of packed (definite, tie) counts gives each
+//    kept position its output slot, so the output is in ascending position order and
+//    ties go to the lower position.
+// Full-row passes: 3 (histogram, candidate compaction, output).  A threshold bin larger
+// than the candidate list falls back to filtered passes over the whole row.  No sort and
+// no global scratch.
 #pragma once
 
 #include "common.cuh"
@@ -20,6 +24,13 @@ namespace dsa {
 
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkStageCap = 32768;  // scores staged in shared memory (128 KiB)
+constexpr int kTopkCandCap = 16384;   // candidate keys of the threshold bin (64 KiB)
+constexpr int kTopkHistBins = 4096;
+
+__host__ inline size_t topk_smem_bytes(int64_t max_kv_len) {
+  const int64_t stage = max_kv_len + 4 < kTopkStageCap ? max_kv_len + 4 : kTopkStageCap;
+  return (size_t)(kTopkHistBins + kTopkCandCap + stage) * sizeof(uint32_t);
+}
 
 struct TopkArgs {
   const int32_t* q_offsets;
@@ -39,15 +50,6 @@ DSA_DEV uint32_t topk_key(float f) {
   uint32_t u = __float_as_uint(f);
   if (u == 0x80000000u) u = 0u;  // -0.0 == +0.0
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-// Add 1 to hist[bin] for every active lane; lanes sharing a bin add once together.
-DSA_DEV void hist_add(uint32_t* hist, uint32_t bin, bool active) {
-  const unsigned m = __ballot_sync(0xFFFFFFFFu, active);
-  if (active) {
-    const unsigned peers = __match_any_sync(m, bin);
-    if ((int)(__ffs(peers) - 1) == lane_id()) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
-  }
 }
 
 // Block-wide exclusive scan of one 32-bit value per thread (1024 threads).
@@ -79,13 +81,47 @@ DSA_DEV uint32_t block_excl_scan(uint32_t v, uint32_t* warp_tot, uint32_t& total
   return res;
 }
 
-__global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkArgs a) {
-  extern __shared__ uint32_t s_keys[];  // [kTopkStageCap] when the row is staged
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t warp_tot[33];
-  __shared__ uint32_t s_sel[3];  // chosen digit, remaining, early-exit flag
-
+// Pick, over hist[0 .. 1024*BPT) scanned from the top bin down, the bin in which the
+// count of larger keys first reaches `remaining`.  s_sel = {bin, still needed from that
+// bin, bin kept whole}.  All threads return after s_sel is visible.
+template <int BPT>
+DSA_DEV void select_bin(const uint32_t* hist, uint32_t remaining, uint32_t* warp_tot,
+                        uint32_t* s_sel) {
+  const int top = kTopkThreads * BPT - 1;
   const int tid = threadIdx.x;
+  uint32_t c[BPT], sum = 0;
+#pragma unroll
+  for (int q = 0; q < BPT; ++q) {
+    c[q] = hist[top - tid * BPT - q];
+    sum += c[q];
+  }
+  uint32_t total;
+  const uint32_t excl = block_excl_scan(sum, warp_tot, total);
+  if (excl < remaining && remaining <= excl + sum) {
+    uint32_t above = excl;
+#pragma unroll
+    for (int q = 0; q < BPT; ++q) {
+      if (above < remaining && remaining <= above + c[q]) {
+        s_sel[0] = (uint32_t)(top - tid * BPT - q);
+        s_sel[1] = remaining - above;
+        s_sel[2] = (remaining - above == c[q]) ? 1u : 0u;
+      }
+      above += c[q];
+    }
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkArgs a) {
+  extern __shared__ uint32_t dyn[];
+  uint32_t* hist = dyn;                         // [kTopkHistBins]
+  uint32_t* cand = dyn + kTopkHistBins;         // [kTopkCandCap]
+  uint32_t* s_keys = cand + kTopkCandCap;       // [kTopkStageCap] when the row is staged
+  __shared__ uint32_t warp_tot[33];
+  __shared__ uint32_t s_sel[3];
+  __shared__ uint32_t s_ncand;
+
+  const int tid = threadIdx.x, lane = lane_id();
   const int64_t i = a.q_count - 1 - (int64_t)blockIdx.x;  // rows late in a sequence first
   const int64_t r = a.q_begin + i;
   const int b = seq_of_row(a.q_offsets, a.batch, r);
@@ -104,79 +140,97 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkArgs a) {
 
   const float* row = a.scores + i * a.ld;
   const bool staged = n <= kTopkStageCap;
-  uint32_t prefix = 0, mask = 0, remaining = (uint32_t)K;
-  bool ge_mode = false;  // true: keep every key >= prefix, no ties to split
+  // four consecutive keys starting at j0 (0 past the end)
+  auto load4 = [&](int64_t j0, uint32_t (&k4)[4], bool from_global) {
+    if (!from_global) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) k4[q] = j0 + q < n ? s_keys[j0 + q] : 0u;
+    } else if (j0 + 3 < n) {
+      const float4 f = __ldg(reinterpret_cast<const float4*>(row + j0));
+      k4[0] = topk_key(f.x);
+      k4[1] = topk_key(f.y);
+      k4[2] = topk_key(f.z);
+      k4[3] = topk_key(f.w);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) k4[q] = j0 + q < n ? topk_key(__ldg(row + j0 + q)) : 0u;
+    }
+  };
 
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    for (int t = tid; t < 256; t += kTopkThreads) hist[t] = 0;
-    __syncthreads();
-    for (int64_t base = 0; base < n; base += 4 * kTopkThreads) {
-      const int64_t j0 = base + 4 * tid;
-      uint32_t k4[4];
-      if (pass == 0 || !staged) {
-        if (j0 + 3 < n) {
-          const float4 f = __ldg(reinterpret_cast<const float4*>(row + j0));
-          k4[0] = topk_key(f.x); k4[1] = topk_key(f.y);
-          k4[2] = topk_key(f.z); k4[3] = topk_key(f.w);
-        } else {
+  // ---- pass A: histogram of the top 12 bits (and staging)
+  for (int t = tid; t < kTopkHistBins; t += kTopkThreads) hist[t] = 0;
+  if (tid == 0) s_ncand = 0;
+  __syncthreads();
+  for (int64_t base = 0; base < n; base += 4 * kTopkThreads) {
+    const int64_t j0 = base + 4 * tid;
+    uint32_t k4[4];
+    load4(j0, k4, true);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) k4[q] = j0 + q < n ? topk_key(__ldg(row + j0 + q)) : 0u;
+    for (int q = 0; q < 4; ++q) {
+      if (j0 + q < n) {
+        if (staged) s_keys[j0 + q] = k4[q];
+        atomicAdd(&hist[k4[q] >> 20], 1u);
+      }
+    }
+  }
+  __syncthreads();
+  select_bin<4>(hist, (uint32_t)K, warp_tot, s_sel);
+  const uint32_t b12 = s_sel[0];
+  uint32_t remaining = s_sel[1];
+  uint32_t prefix = b12 << 20;
+  bool ge_mode = s_sel[2] != 0;  // true: keep every key >= prefix, no ties to split
+
+  if (!ge_mode) {
+    const uint32_t n_bin = hist[b12];
+    const bool use_cand = n_bin <= (uint32_t)kTopkCandCap;
+    __syncthreads();  // every thread has read hist[b12] before it is cleared below
+    if (use_cand) {
+      // candidates: low 20 bits of the keys in the threshold bin (order is irrelevant)
+      for (int64_t base = 0; base < n; base += 4 * kTopkThreads) {
+        const int64_t j0 = base + 4 * tid;
+        uint32_t k4[4];
+        load4(j0, k4, !staged);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const bool m = (j0 + q < n) && ((k4[q] >> 20) == b12);
+          const unsigned bal = __ballot_sync(0xFFFFFFFFu, m);
+          if (bal) {
+            uint32_t slot = 0;
+            if (lane == 0) slot = atomicAdd(&s_ncand, (uint32_t)__popc(bal));
+            slot = __shfl_sync(0xFFFFFFFFu, slot, 0);
+            if (m) cand[slot + __popc(bal & ((1u << lane) - 1u))] = k4[q] & 0xFFFFFu;
+          }
         }
-        if (pass == 0 && staged) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if (j0 + q < n) s_keys[j0 + q] = k4[q];
+      }
+    }
+    // two 10-bit digits below the 12-bit prefix
+    for (int level = 0; level < 2 && !ge_mode; ++level) {
+      const int shift = level == 0 ? 10 : 0;
+      for (int t = tid; t < 1024; t += kTopkThreads) hist[t] = 0;
+      __syncthreads();
+      if (use_cand) {
+        for (uint32_t c = tid; c < n_bin; c += kTopkThreads) {
+          const uint32_t low = cand[c];
+          if (level == 0 || (low >> 10) == ((prefix >> 10) & 1023u))
+            atomicAdd(&hist[(low >> shift) & 1023u], 1u);
         }
       } else {
+        const uint32_t want_mask = level == 0 ? 0xFFF00000u : 0xFFFFFC00u;
+        for (int64_t base = 0; base < n; base += 4 * kTopkThreads) {
+          const int64_t j0 = base + 4 * tid;
+          uint32_t k4[4];
+          load4(j0, k4, !staged);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) k4[q] = j0 + q < n ? s_keys[j0 + q] : 0u;
-      }
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const bool act = (j0 + q < n) && ((k4[q] & mask) == prefix);
-        hist_add(hist, (k4[q] >> shift) & 255u, act);
-      }
-    }
-    __syncthreads();
-    if (tid < 32) {
-      // lane l owns bins 255-8l .. 248-8l (descending); find the bin where the count of
-      // larger keys first reaches `remaining`
-      uint32_t c[8], sum = 0;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        c[q] = hist[255 - 8 * tid - q];
-        sum += c[q];
-      }
-      uint32_t incl = sum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-        if (tid >= o) incl += y;
-      }
-      const uint32_t excl = incl - sum;
-      const bool mine = excl < remaining && remaining <= incl;
-      if (mine) {
-        uint32_t above = excl;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          if (above < remaining && remaining <= above + c[q]) {
-            s_sel[0] = 255u - 8u * tid - q;
-            s_sel[1] = remaining - above;
-            s_sel[2] = (remaining - above == c[q]) ? 1u : 0u;
-          }
-          above += c[q];
+          for (int q = 0; q < 4; ++q)
+            if (j0 + q < n && (k4[q] & want_mask) == prefix)
+              atomicAdd(&hist[(k4[q] >> shift) & 1023u], 1u);
         }
       }
-    }
-    __syncthreads();
-    const uint32_t digit = s_sel[0];
-    remaining = s_sel[1];
-    prefix |= digit << shift;
-    mask |= 255u << shift;
-    if (s_sel[2]) {  // the whole bin is kept: threshold is "key >= prefix"
-      ge_mode = true;
-      break;
+      __syncthreads();
+      select_bin<1>(hist, remaining, warp_tot, s_sel);
+      prefix |= s_sel[0] << shift;
+      remaining = s_sel[1];
+      ge_mode = s_sel[2] != 0;
     }
   }
 
