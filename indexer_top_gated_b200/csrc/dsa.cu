@@ -307,6 +307,32 @@ int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 // Workspace per pass row: scores row (ld floats) plus an index row when idx_out is absent.
 int64_t scores_ld(const dsa_ragged* R) { return round_up(std::max(R->max_kv_len, 1), 32); }
 
+// Rows of one indexer / Top-K sub-pass: bounded by kScorePassBytes of scores (more rows per
+// launch amortise CTA set-up; fewer keep the scores closer to L2); attention passes take as
+// many rows as the rest of the workspace holds.
+constexpr int64_t kScorePassBytes = int64_t(512) << 20;
+
+struct PassPlan {
+  int64_t rows_s;  // query rows per indexer / Top-K sub-pass
+  int64_t rows_a;  // query rows per attention pass
+};
+
+// srow / irow: workspace bytes of one score row / one index row (irow = 0 when the
+// caller provides the index output).  Returns false if not even one row of each fits.
+bool plan_passes(int64_t total_q, int64_t srow, int64_t irow, int64_t ws, int num_sms,
+                 PassPlan* plan) {
+  if (ws < srow + irow) return false;
+  int64_t rows_s = std::max<int64_t>(kScorePassBytes / srow, std::min<int64_t>(total_q, num_sms));
+  rows_s = std::max<int64_t>(1, std::min(rows_s, total_q));
+  // a score pass never takes more than an attention pass of the same size leaves room for
+  rows_s = std::max<int64_t>(1, std::min(rows_s, ws / (srow + irow)));
+  int64_t rows_a = irow ? (ws - rows_s * srow) / irow : total_q;
+  rows_a = std::max<int64_t>(rows_s, std::min(rows_a, total_q));
+  plan->rows_s = rows_s;
+  plan->rows_a = std::min(rows_a, total_q);
+  return true;
+}
+
 dsa_status run_layer(const dsa_params* P, const dsa_ragged* R, const void* q_idx,
                      const void* k_idx, const float* w, const void* q, const void* k,
                      const void* v, const void* gate, void* out, int32_t* idx_out,
@@ -324,22 +350,28 @@ dsa_status run_layer(const dsa_params* P, const dsa_ragged* R, const void* q_idx
   if (R->total_q == 0) return DSA_OK;
   const int64_t ld = scores_ld(R);
   const int64_t K = P->top_k;
-  const int64_t row_bytes = ld * 4 + (idx_out ? 0 : round_up(K * 4, 16));
-  const int64_t rows = std::min<int64_t>(R->total_q, (int64_t)ws_bytes / row_bytes);
-  if (rows < 1) return DSA_ERR_WORKSPACE;
+  const int64_t irow = idx_out ? 0 : round_up(K * 4, 16);
+  if ((int64_t)ws_bytes < ld * 4 + irow) return DSA_ERR_WORKSPACE;
   DeviceState* dev = nullptr;
   DSA_TRY(device_setup(&dev));
+  PassPlan plan;
+  if (!plan_passes(R->total_q, ld * 4, irow, (int64_t)ws_bytes, dev->num_sms, &plan))
+    return DSA_ERR_WORKSPACE;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
   float* scores = static_cast<float*>(ws);
-  int32_t* idx_ws =
-      idx_out ? nullptr : reinterpret_cast<int32_t*>(static_cast<char*>(ws) + rows * ld * 4);
+  int32_t* idx_ws = idx_out ? nullptr
+                            : reinterpret_cast<int32_t*>(static_cast<char*>(ws) +
+                                                         plan.rows_s * ld * 4);
   const int bq = (decode || R->max_q_len <= 16) ? 16 : 64;
-  for (int64_t r0 = 0; r0 < R->total_q; r0 += rows) {
-    const int64_t cnt = std::min<int64_t>(rows, R->total_q - r0);
-    int32_t* idx = idx_out ? idx_out + r0 * K : idx_ws;
-    DSA_TRY(launch_index_scores(*dev, P, R, q_idx, k_idx, w, r0, cnt, scores, ld, bq, stream));
-    DSA_TRY(launch_topk(P, R, scores, ld, r0, cnt, idx, K, nullptr, stream));
-    DSA_TRY(launch_attn(P, R, q, k, v, idx, K, r0, cnt, gate, out, nullptr, err_count, stream));
+  for (int64_t a0 = 0; a0 < R->total_q; a0 += plan.rows_a) {
+    const int64_t cnt_a = std::min<int64_t>(plan.rows_a, R->total_q - a0);
+    int32_t* idx = idx_out ? idx_out + a0 * K : idx_ws;
+    for (int64_t s0 = a0; s0 < a0 + cnt_a; s0 += plan.rows_s) {
+      const int64_t cnt_s = std::min<int64_t>(plan.rows_s, a0 + cnt_a - s0);
+      DSA_TRY(launch_index_scores(*dev, P, R, q_idx, k_idx, w, s0, cnt_s, scores, ld, bq, stream));
+      DSA_TRY(launch_topk(P, R, scores, ld, s0, cnt_s, idx + (s0 - a0) * K, K, nullptr, stream));
+    }
+    DSA_TRY(launch_attn(P, R, q, k, v, idx, K, a0, cnt_a, gate, out, nullptr, err_count, stream));
   }
   return DSA_OK;
 }
@@ -420,13 +452,17 @@ dsa_status dsa_workspace_size(const dsa_params* P, const dsa_ragged* R, int is_d
                               size_t* min_bytes, size_t* rec_bytes) {
   (void)is_decode;
   DSA_TRY(check_common(P, R));
-  const int64_t ld = scores_ld(R);
-  const int64_t row = ld * 4 + round_up((int64_t)P->top_k * 4, 16);
-  if (min_bytes) *min_bytes = (size_t)row;
+  const int64_t srow = scores_ld(R) * 4;
+  const int64_t irow = round_up((int64_t)P->top_k * 4, 16);
+  if (min_bytes) *min_bytes = (size_t)(srow + irow);
   if (rec_bytes) {
-    // enough rows per pass to fill the GPU many times over, bounded at 1 GiB
-    int64_t rows = std::max<int64_t>(1, std::min<int64_t>(R->total_q, (1ll << 30) / row));
-    *rec_bytes = (size_t)(rows * row);
+    // a score sub-pass of up to kScorePassBytes (at least one row per SM) plus index rows
+    // for attention passes of up to 16384 query rows
+    const int64_t tq = std::max<int64_t>(1, R->total_q);
+    int64_t rows_s = std::max<int64_t>(kScorePassBytes / srow, std::min<int64_t>(tq, 148));
+    rows_s = std::max<int64_t>(1, std::min(rows_s, tq));
+    const int64_t rows_a = std::max(rows_s, std::min<int64_t>(tq, 16384));
+    *rec_bytes = (size_t)(rows_s * srow + rows_a * irow);
   }
   return DSA_OK;
 }

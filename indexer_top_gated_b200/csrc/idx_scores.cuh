@@ -10,8 +10,9 @@
 //    positions of one query row: every score store is a coalesced 128-byte line.
 //  - Warp 0 issues TMA loads (128-byte swizzled, one box per indexer head) into a
 //    3-stage ring; warp 1 issues tcgen05.mma (one per head and 16-wide K step) into one
-//    of two TMEM accumulator buffers; warps 2-5 drain TMEM (tcgen05.ld), apply ReLU,
-//    the head weights and the head sum, mask causally and store fp32 scores.
+//    of two TMEM accumulator buffers; warps 2-9 drain TMEM (tcgen05.ld; two warps per
+//    lane quadrant, alternate 16-column chunks), apply ReLU, the head weights and the
+//    head sum, mask causally and store fp32 scores.
 //  - Tiles may straddle sequences of a ragged batch: the CTA runs one pass per
 //    sequence it touches and masks the other rows.  Tiles are scheduled largest
 //    first (the last rows of a sequence see the most keys).
@@ -42,7 +43,8 @@ struct IdxArgs {
 
 constexpr int kIdxStages = 3;
 constexpr int kIdxKeyTile = 128;
-constexpr int kIdxThreads = 192;
+constexpr int kIdxEpiWarps = 8;  // two warps per TMEM lane quadrant
+constexpr int kIdxThreads = 64 + 32 * kIdxEpiWarps;
 
 template <bool FP8>
 struct IdxGeom {
@@ -148,7 +150,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&tfull[i]), 1);
-      mbar_init(smem_u32(&tempty[i]), 4);
+      mbar_init(smem_u32(&tempty[i]), kIdxEpiWarps);
     }
     mbar_init(smem_u32(qfull), 1);
     fence_mbar_init();
@@ -241,12 +243,15 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       mbar_wait_bounded(smem_u32(&tfull[j & 1]), (j >> 1) & 1, nullptr, nullptr);
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2-5)
+    // ------------------------------------------------------------ epilogue (warps 2-9)
     const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
+    const int half = (warp - 2) >> 2;  // the two warps of a quadrant take alternate chunks
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    // shared head weights with the (positive) dequantisation scale folded in:
+    // w * max(0, c * x) = (w * c) * max(0, x) for c > 0
     float wsh[4] = {0.f, 0.f, 0.f, 0.f};
     if (a.w_row_stride == 0)
-      for (int h = 0; h < H; ++h) wsh[h] = __ldg(a.w + h);
+      for (int h = 0; h < H; ++h) wsh[h] = __ldg(a.w + h) * a.scale;
     int i = 0;
     bool ok = true;
     for (int b = b_first; b <= b_last && ok; ++b) {
@@ -263,7 +268,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         const int64_t j = (int64_t)kt * kIdxKeyTile + quad * 32 + lane;  // key position
         // columns c of this tile that belong to sequence b: rows rs..re-1
         const int c_lo = (int)(rs - r0), c_hi = (int)(re - r0);
-        for (int c0 = (c_lo / 16) * 16; c0 < c_hi; c0 += 16) {
+        for (int c0 = (c_lo / 16) * 16 + 16 * half; c0 < c_hi; c0 += 32) {
           // skip chunks whose rows all precede this key tile (causal)
           const int64_t p_chunk_max = pbase + r0 + (c0 + 15 < c_hi - 1 ? c0 + 15 : c_hi - 1);
           if (p_chunk_max < (int64_t)kt * kIdxKeyTile) continue;
@@ -280,23 +285,40 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           for (int h = 0; h < 4; ++h) {
             if (h >= H) break;
             reg_fence(v[h]);
+            if (a.w_row_stride == 0) {
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              float wv = wsh[h];
-              if (a.w_row_stride != 0) {
+              for (int c = 0; c < 16; ++c)
+                acc[c] = fmaf(wsh[h], fmaxf(__uint_as_float(v[h][c]), 0.f), acc[c]);
+            } else {
+#pragma unroll
+              for (int c = 0; c < 16; ++c) {
                 int64_t r = r0 + c0 + c;
                 if (r > r_last) r = r_last;
-                wv = __ldg(a.w + r * a.w_row_stride + h);
+                const float wv = __ldg(a.w + r * a.w_row_stride + h);
+                acc[c] = fmaf(wv, fmaxf(__uint_as_float(v[h][c]) * a.scale, 0.f), acc[c]);
               }
-              acc[c] = fmaf(wv, fmaxf(__uint_as_float(v[h][c]) * a.scale, 0.f), acc[c]);
             }
           }
+          // rows r0+c0 .. r0+c0+15; key j.  Interior chunk: every row belongs to this
+          // sequence and sees the whole key tile, so no per-element predicate is needed.
+          float* dst = a.scores + (r0 + c0 - a.q_begin) * a.ld + j;
+          const bool interior = c0 >= c_lo && c0 + 16 <= c_hi &&
+                                (int64_t)kt * kIdxKeyTile + (kIdxKeyTile - 1) <= pbase + r0 + c0 &&
+                                (int64_t)kt * kIdxKeyTile + kIdxKeyTile <= a.ld;
+          if (interior) {
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const int cc = c0 + c;
-            const int64_t r = r0 + cc;
-            if (cc >= c_lo && cc < c_hi && j <= pbase + r && j < a.ld)
-              a.scores[(r - a.q_begin) * a.ld + j] = acc[c];
+            for (int c = 0; c < 16; ++c) {
+              *dst = acc[c];
+              dst += a.ld;
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const int cc = c0 + c;
+              const int64_t r = r0 + cc;
+              if (cc >= c_lo && cc < c_hi && j <= pbase + r && j < a.ld) *dst = acc[c];
+              dst += a.ld;
+            }
           }
         }
         tc_fence_before();
