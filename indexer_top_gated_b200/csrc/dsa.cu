@@ -255,7 +255,8 @@ dsa_status launch_topk(const dsa_params* P, const dsa_ragged* R, const float* sc
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
-dsa_status launch_attn(const dsa_params* P, const dsa_ragged* R, const void* q, const void* k,
+dsa_status launch_attn(const DeviceState& dev, const dsa_params* P, const dsa_ragged* R,
+                       const void* q, const void* k,
                        const void* v, const int32_t* idx, int64_t ld_idx, int64_t q_begin,
                        int64_t q_count, const void* gate, void* out, float* lse,
                        int32_t* err_count, cudaStream_t stream) {
@@ -276,6 +277,7 @@ dsa_status launch_attn(const dsa_params* P, const dsa_ragged* R, const void* q, 
   a.out = static_cast<__nv_bfloat16*>(out);
   a.lse = lse;
   a.err_count = err_count;
+  a.status = dev.status;
   a.Hq = P->n_q_heads;
   a.Hkv = P->n_kv_heads;
   a.G = P->n_q_heads / P->n_kv_heads;
@@ -371,7 +373,8 @@ dsa_status run_layer(const dsa_params* P, const dsa_ragged* R, const void* q_idx
       DSA_TRY(launch_index_scores(*dev, P, R, q_idx, k_idx, w, s0, cnt_s, scores, ld, bq, stream));
       DSA_TRY(launch_topk(P, R, scores, ld, s0, cnt_s, idx + (s0 - a0) * K, K, nullptr, stream));
     }
-    DSA_TRY(launch_attn(P, R, q, k, v, idx, K, a0, cnt_a, gate, out, nullptr, err_count, stream));
+    DSA_TRY(launch_attn(*dev, P, R, q, k, v, idx, K, a0, cnt_a, gate, out, nullptr, err_count,
+                        stream));
   }
   return DSA_OK;
 }
@@ -444,8 +447,8 @@ dsa_status dsa_sparse_attn_gated(const dsa_params* P, const dsa_ragged* R, const
   if (q_count > INT32_MAX) return DSA_ERR_UNSUPPORTED;
   DeviceState* dev = nullptr;
   DSA_TRY(device_setup(&dev));
-  return launch_attn(P, R, q, k_cache, v_cache, idx, ld_idx, q_begin, q_count, gate, out, lse,
-                     err_count, static_cast<cudaStream_t>(stream));
+  return launch_attn(*dev, P, R, q, k_cache, v_cache, idx, ld_idx, q_begin, q_count, gate, out,
+                     lse, err_count, static_cast<cudaStream_t>(stream));
 }
 
 dsa_status dsa_workspace_size(const dsa_params* P, const dsa_ragged* R, int is_decode,

@@ -1,31 +1,34 @@
 // sparse_attn.cuh - steps 3-4 of the layer: exact softmax attention over the selected
 // cache rows, with the sigmoid output gate fused into the epilogue.
 //
-// One CTA per (query row, block of up to 8 KV heads).  Per chunk of selected positions:
-//  - gather: all KV heads of a selected position are one contiguous run in the cache
-//    ([pos][Hkv][d]), so the CTA copies K and V rows with 16-byte cp.async into a
-//    3-stage ring in shared memory (XOR-swizzled 16-byte chunks, conflict-free for
-//    ldmatrix).  Padding / out-of-range entries are zero-filled and masked.
-//  - each warp owns one KV head and 16 positions of the chunk; the query heads of the
-//    GQA group share that gather.  Logits are computed transposed, S^T = K_sel Q^T
-//    (mma.sync m16n8k16, keys on M, the group's 8 query heads on N), so a group of 8
-//    heads needs no padding.
+// One CTA per (query row, block of up to 8 KV heads), 8 warps.  Each warp owns one KV
+// head and 16 positions of every chunk of selected positions, and gathers exactly the
+// bytes it consumes, so warps never synchronise with each other inside the main loop:
+//  - gather: the warp's 16 positions x (K and V slices of its head, 256 B each) arrive
+//    through 16-byte cp.async (32 lanes = 512 contiguous bytes per instruction) into the
+//    warp's own 3-stage ring (XOR-swizzled 16-byte chunks, conflict-free for ldmatrix).
+//    Index entries are read once per position and shared across the warp by shuffles;
+//    padding / out-of-range entries are zero-filled and masked (a ballot mask).
+//  - logits are computed transposed, S^T = K_sel Q^T (mma.sync m16n8k16, keys on M, the
+//    group's 8 query heads on N, two independent accumulation chains), so a group of 8
+//    heads needs no padding and the query heads of a GQA group share the gather.
 //  - online softmax in registers (log2 domain); P^T becomes the B operand of
 //    O^T += V_sel^T P^T through movmatrix (8x8 transposes in registers) and V^T comes
-//    from ldmatrix.trans.  P enters as two bf16 terms (P_hi + P_lo), so rounding P
-//    costs ~2^-17 relative instead of 2^-9: the error no longer scales with
-//    sum_j p_j |v_j| (which dominates outputs that nearly cancel).
+//    from ldmatrix.trans.  P enters as two bf16 terms (P_hi + P_lo), so rounding P costs
+//    ~2^-17 relative instead of 2^-9: the error no longer scales with sum_j p_j |v_j|
+//    (which dominates outputs that nearly cancel).
 //  - warps of the same KV head merge (m, l, O) through shared memory; the epilogue
 //    divides by l, multiplies by sigmoid(gate) and stores bf16 (and the LSE).
-// The work per row is bound by the gather bytes (K * Hkv * d * 2 * 2 per query), so
-// the tensor-core path here only has to keep up with memory.
+// The work per row is bound by the gather bytes (K * Hkv * d * 2 * 2 per query), so the
+// tensor-core path here only has to keep up with memory.
 #pragma once
 
 #include "common.cuh"
 
 namespace dsa {
 
-constexpr int kAttnThreads = 256;
+constexpr int kAttnWarps = 8;
+constexpr int kAttnThreads = 32 * kAttnWarps;
 constexpr int kAttnStages = 3;
 constexpr int kHeadDim = 128;
 
@@ -45,33 +48,30 @@ struct AttnArgs {
   __nv_bfloat16* out;
   float* lse;
   int32_t* err_count;
+  int* status;
   int Hq, Hkv, G;
   float scale_log2;  // softmax scale * log2(e)
 };
 
 template <int HKV_CTA>
 struct AttnGeom {
-  static constexpr int kWPG = 8 / HKV_CTA;            // warps per KV head
-  static constexpr int kChunk = 16 * kWPG;            // positions per stage
-  static constexpr int kRowBytes = HKV_CTA * kHeadDim * 2;
-  static constexpr int kHalfBytes = kChunk * kRowBytes;  // K (or V) part of a stage
-  static constexpr int kStageBytes = 2 * kHalfBytes;     // 64 KiB
-  static constexpr int kPieces = kStageBytes / 16;       // 16-byte copies per stage
+  static constexpr int kWPG = kAttnWarps / HKV_CTA;  // warps per KV head
+  static constexpr int kChunk = 16 * kWPG;           // positions per chunk (all warps)
+  static constexpr int kWarpHalf = 16 * kHeadDim * 2;  // one warp's K (or V) slice: 4 KiB
+  static constexpr int kWarpStage = 2 * kWarpHalf;     // K + V: 8 KiB
 };
 
 __host__ inline size_t attn_smem_bytes() {
-  return (size_t)kAttnStages * AttnGeom<1>::kStageBytes + 128 /*align*/;
+  return (size_t)kAttnWarps * kAttnStages * AttnGeom<1>::kWarpStage + 128 /*align*/;
 }
 
 template <int HKV_CTA, int NT>
 __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(AttnArgs a) {
   using Geo = AttnGeom<HKV_CTA>;
   constexpr int CH = Geo::kChunk;
-  constexpr int ROWB = Geo::kRowBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  __shared__ uint8_t s_valid[kAttnStages][CH];
   __shared__ int s_last;
   __shared__ int s_err;
 
@@ -109,45 +109,40 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(AttnArgs a
   if (tid == 0 && s_err && a.err_count && blockIdx.y == 0) atomicAdd(a.err_count, s_err);
   const int n_chunks = (s_last + CH) / CH;  // 0 when nothing is selected
 
-  // ---- gather of one chunk of selected positions into stage st.  Each warp copies whole
-  // position rows: one (broadcast) index load per position, then every cp.async of the
-  // warp covers a contiguous 512-byte run of the row (K and V rows alike).
-  auto load_chunk = [&](int c, int st) {
-    constexpr int CPR = HKV_CTA * 16;             // 16-byte pieces per position row
-    constexpr int LPP = CPR < 32 ? CPR : 32;      // lanes per position
-    constexpr int PPI = 32 / LPP;                 // positions per warp iteration
-    constexpr int PIECES = CPR / LPP;             // pieces per lane per position row
-    constexpr int PPW = CH / 8;                   // positions per warp per chunk
-    uint8_t* base = smem + (size_t)st * Geo::kStageBytes;
-    const int sub_lane = lane % LPP;
-#pragma unroll
-    for (int it = 0; it < PPW / PPI; ++it) {
-      const int pos = warp * PPW + it * PPI + lane / LPP;
-      const int e = c * CH + pos;
-      const int j = e < K ? __ldg(irow + e) : -1;
-      const bool valid = j >= 0 && (int64_t)j <= p;
-      const int64_t row_elem = ((kbase + (valid ? j : 0)) * a.Hkv + g0) * kHeadDim;
-      const __nv_bfloat16* ksrc = a.k + row_elem;
-      const __nv_bfloat16* vsrc = a.v + row_elem;
-      uint8_t* kdst = base + pos * ROWB;
-      uint8_t* vdst = kdst + Geo::kHalfBytes;
-#pragma unroll
-      for (int q = 0; q < PIECES; ++q) {
-        const int ch = sub_lane + q * LPP;
-        const uint32_t off = (uint32_t)((ch ^ (pos & 7)) << 4);
-        cp_async_16(smem_u32(kdst + off), valid ? (const void*)(ksrc + ch * 8) : (const void*)a.k,
-                    valid ? 16u : 0u);
-        cp_async_16(smem_u32(vdst + off), valid ? (const void*)(vsrc + ch * 8) : (const void*)a.k,
-                    valid ? 16u : 0u);
-      }
-      if (sub_lane == 0) s_valid[st][pos] = valid ? 1 : 0;
-    }
-  };
-
-  // ---- per-warp state: one KV head (g) and 16 positions (sub) of every chunk
+  // ---- per-warp state: one KV head (g) and positions sub*16 .. sub*16+15 of every chunk
   const int g = warp / Geo::kWPG;
   const int sub = warp % Geo::kWPG;
   const int hg = g0 + g;  // KV head
+  uint8_t* wsm = smem + (size_t)warp * kAttnStages * Geo::kWarpStage;  // this warp's ring
+  const __nv_bfloat16* kh = a.k + (int64_t)hg * kHeadDim;
+  const __nv_bfloat16* vh = a.v + (int64_t)hg * kHeadDim;
+  const int64_t row_stride = (int64_t)a.Hkv * kHeadDim;
+
+  // gather chunk c into ring slot st; returns the validity mask of its 16 positions
+  auto load_chunk = [&](int c, int st) -> uint32_t {
+    const int e = c * CH + sub * 16 + (lane & 15);
+    const int j = e < K ? __ldg(irow + e) : -1;
+    const bool valid = j >= 0 && (int64_t)j <= p;
+    const int row = (int)(valid ? j : 0);
+    const uint32_t vmask = __ballot_sync(0xFFFFFFFFu, valid) & 0xFFFFu;
+    uint8_t* kdst = wsm + st * Geo::kWarpStage;
+    uint8_t* vdst = kdst + Geo::kWarpHalf;
+    const int ch = lane & 15;  // 16-byte chunk within the 256-byte head slice
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int t = 2 * k + (lane >> 4);  // position within the warp's 16
+      const int rt = __shfl_sync(0xFFFFFFFFu, row, t);
+      const bool vt = (vmask >> t) & 1u;
+      const int64_t off = (kbase + rt) * row_stride + ch * 8;
+      const uint32_t so = (uint32_t)(t * 256 + ((ch ^ (t & 7)) << 4));
+      cp_async_16(smem_u32(kdst + so), vt ? (const void*)(kh + off) : (const void*)a.k,
+                  vt ? 16u : 0u);
+      cp_async_16(smem_u32(vdst + so), vt ? (const void*)(vh + off) : (const void*)a.k,
+                  vt ? 16u : 0u);
+    }
+    return vmask;
+  };
+
   uint32_t bq[NT][8][2];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
@@ -173,49 +168,60 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(AttnArgs a
     l_run[nt][0] = l_run[nt][1] = 0.f;
   }
 
+  // ldmatrix row of this lane within the warp's 16 positions (K: A rows; V: A^T rows)
+  const int kt = (lane & 7) + ((lane >> 3) & 1) * 8;
+  const int vt = (lane & 7) + (lane >> 4) * 8;
+  const int kch = lane >> 4, vch = (lane >> 3) & 1;
+
+  uint64_t vmasks = 0;  // 16-bit validity mask of each ring slot
 #pragma unroll
   for (int s = 0; s < kAttnStages - 1; ++s) {
-    if (s < n_chunks) load_chunk(s, s);
+    if (s < n_chunks) vmasks |= (uint64_t)load_chunk(s, s) << (16 * s);
     cp_async_commit();
   }
 
   for (int c = 0; c < n_chunks; ++c) {
     cp_async_wait<kAttnStages - 2>();
-    __syncthreads();
+    __syncwarp();
+    const int st = c % kAttnStages;
+    const uint32_t vm = (uint32_t)(vmasks >> (16 * st)) & 0xFFFFu;
     {
       const int nxt = c + kAttnStages - 1;
-      if (nxt < n_chunks) load_chunk(nxt, nxt % kAttnStages);
+      if (nxt < n_chunks) {
+        const int ns = nxt % kAttnStages;
+        vmasks = (vmasks & ~(0xFFFFull << (16 * ns))) | ((uint64_t)load_chunk(nxt, ns) << (16 * ns));
+      }
       cp_async_commit();
     }
-    const int st = c % kAttnStages;
-    const uint8_t* kst = smem + (size_t)st * Geo::kStageBytes;
-    const uint8_t* vst = kst + Geo::kHalfBytes;
+    const uint32_t kst = smem_u32(wsm + st * Geo::kWarpStage);
+    const uint32_t vst = kst + Geo::kWarpHalf;
 
-    // S^T[16 pos x 8 heads] = K_sel[16 x 128] * Q^T[128 x 8]
-    float s[NT][4];
+    // S^T[16 pos x 8 heads] = K_sel[16 x 128] * Q^T[128 x 8]; two accumulation chains
+    float s[NT][4], s2[NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-    {
-      const int pos = sub * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-      const uint8_t* rowp = kst + pos * ROWB;
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const int ch = g * 16 + ks * 2 + (lane >> 4);
-        uint32_t af[4];
-        ldmatrix_x4(smem_u32(rowp + ((ch ^ (pos & 7)) << 4)), af);
+      for (int q = 0; q < 4; ++q) s[nt][q] = s2[nt][q] = 0.f;
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[nt], af, bq[nt][ks][0], bq[nt][ks][1]);
+    for (int ks = 0; ks < 8; ++ks) {
+      uint32_t af[4];
+      const int chk = ks * 2 + kch;
+      ldmatrix_x4(kst + kt * 256 + ((chk ^ (kt & 7)) << 4), af);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        if (ks & 1) mma_bf16_16816(s2[nt], af, bq[nt][ks][0], bq[nt][ks][1]);
+        else mma_bf16_16816(s[nt], af, bq[nt][ks][0], bq[nt][ks][1]);
       }
     }
-    const bool v_lo = s_valid[st][sub * 16 + (lane >> 2)] != 0;
-    const bool v_hi = s_valid[st][sub * 16 + (lane >> 2) + 8] != 0;
+    const bool v_lo = (vm >> (lane >> 2)) & 1u;
+    const bool v_hi = (vm >> ((lane >> 2) + 8)) & 1u;
     uint32_t pb[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      s[nt][0] = v_lo ? s[nt][0] * a.scale_log2 : -INFINITY;
-      s[nt][1] = v_lo ? s[nt][1] * a.scale_log2 : -INFINITY;
-      s[nt][2] = v_hi ? s[nt][2] * a.scale_log2 : -INFINITY;
-      s[nt][3] = v_hi ? s[nt][3] * a.scale_log2 : -INFINITY;
+      s[nt][0] = v_lo ? (s[nt][0] + s2[nt][0]) * a.scale_log2 : -INFINITY;
+      s[nt][1] = v_lo ? (s[nt][1] + s2[nt][1]) * a.scale_log2 : -INFINITY;
+      s[nt][2] = v_hi ? (s[nt][2] + s2[nt][2]) * a.scale_log2 : -INFINITY;
+      s[nt][3] = v_hi ? (s[nt][3] + s2[nt][3]) * a.scale_log2 : -INFINITY;
       float mx[2] = {fmaxf(s[nt][0], s[nt][2]), fmaxf(s[nt][1], s[nt][3])};
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
@@ -256,30 +262,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(AttnArgs a
       pb[nt][3] = movmatrix_trans(l23);
     }
     // O^T[128 dims x 8 heads] += V_sel^T[128 x 16] * P^T[16 x 8]
-    {
-      const int pos = sub * 16 + (lane & 7) + (lane >> 4) * 8;
-      const uint8_t* rowp = vst + pos * ROWB;
 #pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        const int ch = g * 16 + mt * 2 + ((lane >> 3) & 1);
-        uint32_t vf[4];
-        ldmatrix_x4_trans(smem_u32(rowp + ((ch ^ (pos & 7)) << 4)), vf);
+    for (int mt = 0; mt < 8; ++mt) {
+      uint32_t vf[4];
+      const int chv = mt * 2 + vch;
+      ldmatrix_x4_trans(vst + vt * 256 + ((chv ^ (vt & 7)) << 4), vf);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          mma_bf16_16816(o[nt][mt], vf, pb[nt][0], pb[nt][1]);
-          mma_bf16_16816(o[nt][mt], vf, pb[nt][2], pb[nt][3]);
-        }
+      for (int nt = 0; nt < NT; ++nt) {
+        mma_bf16_16816(o[nt][mt], vf, pb[nt][0], pb[nt][1]);
+        mma_bf16_16816(o[nt][mt], vf, pb[nt][2], pb[nt][3]);
       }
     }
+    __syncwarp();  // the slot is refilled by the next iteration's loads
   }
   cp_async_wait<0>();
-  __syncthreads();
+
+  __syncthreads();  // all warps are done with their rings: the memory is reused below
 
   // ---- merge the warps of each KV head through shared memory
   constexpr int HPW = NT * 8;  // head slots per warp
-  float* red_o = reinterpret_cast<float*>(smem);               // [8 warps][HPW][128]
-  float* red_m = red_o + 8 * HPW * kHeadDim;                    // [8][HPW]
-  float* red_l = red_m + 8 * HPW;                               // [8][HPW]
+  float* red_o = reinterpret_cast<float*>(smem);       // [8 warps][HPW][128]
+  float* red_m = red_o + kAttnWarps * HPW * kHeadDim;  // [8][HPW]
+  float* red_l = red_m + kAttnWarps * HPW;             // [8][HPW]
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
