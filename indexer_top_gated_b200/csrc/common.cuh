@@ -260,6 +260,13 @@ DSA_DEV uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// 2^x with the hardware approximation (ex2.approx.ftz: about 2 ulp; 2^-inf = 0).
+DSA_DEV float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // The two bf16 halves of a packed pair, as fp32 (exact).
 DSA_DEV float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
 DSA_DEV float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }

@@ -115,30 +115,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(AttnArgs a
   const int hg = g0 + g;  // KV head
   uint8_t* wsm = smem + (size_t)warp * kAttnStages * Geo::kWarpStage;  // this warp's ring
   const __nv_bfloat16* kh = a.k + (int64_t)hg * kHeadDim;
-  const __nv_bfloat16* vh = a.v + (int64_t)hg * kHeadDim;
   const int64_t row_stride = (int64_t)a.Hkv * kHeadDim;
 
-  // gather chunk c into ring slot st; returns the validity mask of its 16 positions
+  // gather chunk c into ring slot st; returns the validity mask of its 16 positions.
+  // Lane t < 16 reads the index of position t and forms its row address once; every
+  // cp.async then moves two whole 256-byte head slices (512 contiguous bytes per warp
+  // instruction), the row address arriving by shuffle.
+  const int lt = lane & 15, lhi = lane >> 4;
+  const int64_t v_minus_k = a.v - a.k;  // V row = K row + this many elements
   auto load_chunk = [&](int c, int st) -> uint32_t {
-    const int e = c * CH + sub * 16 + (lane & 15);
+    const int e = c * CH + sub * 16 + lt;
     const int j = e < K ? __ldg(irow + e) : -1;
     const bool valid = j >= 0 && (int64_t)j <= p;
-    const int row = (int)(valid ? j : 0);
     const uint32_t vmask = __ballot_sync(0xFFFFFFFFu, valid) & 0xFFFFu;
-    uint8_t* kdst = wsm + st * Geo::kWarpStage;
-    uint8_t* vdst = kdst + Geo::kWarpHalf;
-    const int ch = lane & 15;  // 16-byte chunk within the 256-byte head slice
+    const unsigned long long rowp =
+        reinterpret_cast<unsigned long long>(kh + (kbase + (valid ? j : 0)) * row_stride);
+    const uint32_t kdst = smem_u32(wsm + st * Geo::kWarpStage);
+    const uint32_t vdst = kdst + Geo::kWarpHalf;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const int t = 2 * k + (lane >> 4);  // position within the warp's 16
-      const int rt = __shfl_sync(0xFFFFFFFFu, row, t);
+      const int t = 2 * k + lhi;  // position handled by this lane in step k
       const bool vt = (vmask >> t) & 1u;
-      const int64_t off = (kbase + rt) * row_stride + ch * 8;
-      const uint32_t so = (uint32_t)(t * 256 + ((ch ^ (t & 7)) << 4));
-      cp_async_16(smem_u32(kdst + so), vt ? (const void*)(kh + off) : (const void*)a.k,
-                  vt ? 16u : 0u);
-      cp_async_16(smem_u32(vdst + so), vt ? (const void*)(vh + off) : (const void*)a.k,
-                  vt ? 16u : 0u);
+      const __nv_bfloat16* ks =
+          reinterpret_cast<const __nv_bfloat16*>(__shfl_sync(0xFFFFFFFFu, rowp, t)) + lt * 8;
+      const uint32_t so = (uint32_t)(t * 256 + ((lt ^ (t & 7)) << 4));
+      cp_async_16(kdst + so, vt ? (const void*)ks : (const void*)a.k, vt ? 16u : 0u);
+      cp_async_16(vdst + so, vt ? (const void*)(ks + v_minus_k) : (const void*)a.k, vt ? 16u : 0u);
     }
     return vmask;
   };
@@ -230,6 +232,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(AttnArgs a
         mx[cc] = fmaxf(mx[cc], __shfl_xor_sync(0xFFFFFFFFu, mx[cc], 16));
       }
       float alpha[2], pr[4];
+      bool grew = false;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         const float m_new = fmaxf(m_run[nt][cc], mx[cc]);
@@ -238,19 +241,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(AttnArgs a
           pr[cc] = 0.f;
           pr[cc + 2] = 0.f;
         } else {
-          alpha[cc] = exp2f(m_run[nt][cc] - m_new);
-          pr[cc] = exp2f(s[nt][cc] - m_new);
-          pr[cc + 2] = exp2f(s[nt][cc + 2] - m_new);
+          alpha[cc] = ex2_approx(m_run[nt][cc] - m_new);
+          pr[cc] = ex2_approx(s[nt][cc] - m_new);
+          pr[cc + 2] = ex2_approx(s[nt][cc + 2] - m_new);
         }
+        grew |= m_new != m_run[nt][cc];
         m_run[nt][cc] = m_new;
         l_run[nt][cc] = l_run[nt][cc] * alpha[cc] + pr[cc] + pr[cc + 2];
       }
+      if (__any_sync(0xFFFFFFFFu, grew)) {  // a running max moved: rescale the partial sums
 #pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        o[nt][mt][0] *= alpha[0];
-        o[nt][mt][1] *= alpha[1];
-        o[nt][mt][2] *= alpha[0];
-        o[nt][mt][3] *= alpha[1];
+        for (int mt = 0; mt < 8; ++mt) {
+          o[nt][mt][0] *= alpha[0];
+          o[nt][mt][1] *= alpha[1];
+          o[nt][mt][2] *= alpha[0];
+          o[nt][mt][3] *= alpha[1];
+        }
       }
       // P = P_hi + P_lo, both bf16: the P.V product keeps ~16 significant bits of P
       const uint32_t h01 = pack_bf16x2(pr[0], pr[1]), h23 = pack_bf16x2(pr[2], pr[3]);
