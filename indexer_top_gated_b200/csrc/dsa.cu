@@ -105,7 +105,7 @@ dsa_status device_setup(DeviceState** out) {
     e = e ? e : allow_smem(idx_scores_kernel<16, false>, idx_max);
     e = e ? e : allow_smem(idx_scores_kernel<64, true>, idx_max);
     e = e ? e : allow_smem(idx_scores_kernel<16, true>, idx_max);
-    e = e ? e : allow_smem(topk_kernel, topk_smem_bytes(kTopkStageCap));
+    e = e ? e : allow_smem(topk_kernel, topk_smem_bytes(0));
     e = e ? e : allow_smem(sparse_attn_kernel<1, 1>, attn_smem_bytes());
     e = e ? e : allow_smem(sparse_attn_kernel<2, 1>, attn_smem_bytes());
     e = e ? e : allow_smem(sparse_attn_kernel<4, 1>, attn_smem_bytes());
