@@ -290,7 +290,7 @@ dsa_status launch_attn(const DeviceState& dev, const dsa_params* P, const dsa_ra
   StageScope scope(2, stream);
 #define DSA_ATTN_CASE(H, N)                                                         \
   if (hkv_cta == H && nt == N)                                                      \
-    sparse_attn_kernel<H, N><<<grid, kAttnThreads, smem, stream>>>(a);
+    sparse_attn_kernel<H, N><<<grid, AttnGeom<H>::kThreads, smem, stream>>>(a);
   DSA_ATTN_CASE(1, 1)
   DSA_ATTN_CASE(2, 1)
   DSA_ATTN_CASE(4, 1)

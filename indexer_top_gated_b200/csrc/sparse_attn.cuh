@@ -27,10 +27,16 @@
 
 namespace dsa {
 
-constexpr int kAttnWarps = 8;
-constexpr int kAttnThreads = 32 * kAttnWarps;
-constexpr int kAttnStages = 3;
 constexpr int kHeadDim = 128;
+
+// Warps per CTA and ring depth per warp: 12 warps x 2 stages when a CTA holds at most 4
+// KV heads (more warps hide more latency), 8 warps x 3 stages for 8 KV heads.  Either
+// way the rings take 192 KiB.
+template <int HKV_CTA>
+struct AttnShape {
+  static constexpr int kWarps = HKV_CTA == 8 ? 8 : 12;
+  static constexpr int kStages = HKV_CTA == 8 ? 3 : 2;
+};
 
 struct AttnArgs {
   const int32_t* q_offsets;
@@ -55,20 +61,27 @@ struct AttnArgs {
 
 template <int HKV_CTA>
 struct AttnGeom {
-  static constexpr int kWPG = kAttnWarps / HKV_CTA;  // warps per KV head
+  static constexpr int kWarps = AttnShape<HKV_CTA>::kWarps;
+  static constexpr int kStages = AttnShape<HKV_CTA>::kStages;
+  static constexpr int kThreads = 32 * kWarps;
+  static constexpr int kWPG = kWarps / HKV_CTA;      // warps per KV head
   static constexpr int kChunk = 16 * kWPG;           // positions per chunk (all warps)
   static constexpr int kWarpHalf = 16 * kHeadDim * 2;  // one warp's K (or V) slice: 4 KiB
   static constexpr int kWarpStage = 2 * kWarpHalf;     // K + V: 8 KiB
 };
 
 __host__ inline size_t attn_smem_bytes() {
-  return (size_t)kAttnWarps * kAttnStages * AttnGeom<1>::kWarpStage + 128 /*align*/;
+  return (size_t)AttnGeom<1>::kWarps * AttnGeom<1>::kStages * AttnGeom<1>::kWarpStage +
+         128 /*align*/;
 }
 
 template <int HKV_CTA, int NT>
-__global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(AttnArgs a) {
+__global__ void __launch_bounds__(AttnGeom<HKV_CTA>::kThreads, 1) sparse_attn_kernel(AttnArgs a) {
   using Geo = AttnGeom<HKV_CTA>;
   constexpr int CH = Geo::kChunk;
+  constexpr int kAttnThreads = Geo::kThreads;
+  constexpr int kAttnWarps = Geo::kWarps;
+  constexpr int kAttnStages = Geo::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
