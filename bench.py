@@ -507,7 +507,7 @@ def main():
     if dom == 2:
         t_full = committed_traffic("indexer_top_gated_b200/csrc/sparse_attn.cuh",
                                    "sparse_attn_gated_prefill_t32768_k2048.txt")
-        traffic = t_full / stage_n[2] if t_full else None
+        traffic = t_full  # DRAM bytes per launch of this configuration, from the ncu capture
     roof = {"kernel": names[dom], "bound": stages[dom]["bound"], "achieved": stages[dom]["achieved"],
             "peak": stages[dom]["peak"], "unit": stages[dom]["unit"], "frac": stages[dom]["frac"],
             "traffic": traffic, "peak_source": f"{peak_src} ({'hbm_gbs' if dom else 'bf16_tflops_sustained'})",
