@@ -104,6 +104,11 @@ DSA_DEV void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t b
       : "memory");
 }
 
+// Bulk prefetch of [src, src + bytes) into L2 (16-byte aligned, size a multiple of 16).
+DSA_DEV void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Named barrier over `count` threads (a multiple of 32).
 DSA_DEV void named_barrier(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");

@@ -4,10 +4,10 @@
 // an order-preserving 32-bit key (-0.0 folded onto +0.0).
 //
 // Fast path (almost every row):
-//  - 1024 evenly spaced samples give an estimate t of the K-th largest key: the sample of
-//    rank S*K/n plus a margin of 4 sigma + 8, found by a radix select over the samples
-//    (12 + 10 + 10 bits), so that with overwhelming probability at least K keys of the row
-//    are >= t;
+//  - 1024 samples (64 evenly spaced runs of 16 consecutive scores) give an estimate t of
+//    the K-th largest key: the sample of rank S*K/n plus a margin of 4 sigma + 8, found to
+//    22 bits by a radix select over the samples (12 + 10 bits), so that with overwhelming
+//    probability at least K keys of the row are >= t;
 //  - one ordered pass keeps every key >= t, with its position, as a candidate in shared
 //    memory (each warp owns a contiguous run of positions; packed warp scans and one
 //    block scan per run of 16384 positions give the slots, so candidates stay in
@@ -61,6 +61,12 @@ DSA_DEV uint32_t topk_key(float f) {
   uint32_t u = __float_as_uint(f);
   if (u == 0x80000000u) u = 0u;  // -0.0 == +0.0
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Inverse of topk_key: the float whose key is k (finite for every key of a finite score
+// with low bits cleared, since such keys stay >= key(-FLT_MAX)).
+DSA_DEV float topk_key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k ^ 0x80000000u) : ~k);
 }
 
 DSA_DEV uint32_t warp_incl_scan(uint32_t x) {
@@ -170,6 +176,16 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkArgs a) {
   const float* row = a.scores + i * a.ld;
   const int nn = (int)n;  // rows are shorter than 2^31
   int bank = 0;
+  {
+    // pull the whole row towards L2 now, so that its DRAM latency overlaps the threshold
+    // estimate below and the candidate pass reads from L2 (the row is 16-byte aligned and
+    // its padded length round4(n) <= ld)
+    const int64_t bytes = (((int64_t)nn + 3) & ~int64_t(3)) * 4;
+    constexpr int64_t kPiece = 16384;
+    for (int64_t off = (int64_t)tid * kPiece; off < bytes; off += (int64_t)kTopkThreads * kPiece)
+      bulk_prefetch_l2(reinterpret_cast<const char*>(row) + off,
+                       (uint32_t)(bytes - off < kPiece ? bytes - off : kPiece));
+  }
   // four consecutive keys starting at j0 (a multiple of 4; 0 past the end)
   auto load4 = [&](int j0, uint32_t (&k4)[4]) {
     if (j0 + 3 < nn) {
@@ -187,7 +203,7 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkArgs a) {
   // thread), in hist12 / hist10a / hist10b (zeroed): returns the threshold key in *tau and
   // the count still needed from keys equal to it (0 when the threshold bin is kept whole).
   auto select = [&](uint32_t* h12, uint32_t* h10a, uint32_t* h10b, uint32_t want, auto&& get,
-                    uint32_t count, uint32_t* tau, bool* whole) -> uint32_t {
+                    uint32_t count, int levels, uint32_t* tau, bool* whole) -> uint32_t {
     for (uint32_t c = tid; c < count; c += kTopkThreads) atomicAdd(&h12[get(c) >> 20], 1u);
     __syncthreads();
     if (warp == 0) warp_select<4096>(h12, want, s_sel);
@@ -205,7 +221,7 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkArgs a) {
       t |= s_sel[0] << 10;
       need = s_sel[1];
       w = s_sel[2] != 0;
-      if (!w) {
+      if (!w && levels > 2) {
         for (uint32_t c = tid; c < count; c += kTopkThreads) {
           const uint32_t key = get(c);
           if ((key & 0xFFFFFC00u) == t) atomicAdd(&h10b[key & 1023u], 1u);
@@ -234,35 +250,54 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkArgs a) {
     const float m_exp = (float)S * (float)K / (float)nn;
     int m = (int)ceilf(m_exp + 4.f * sqrtf(m_exp) + 8.f);
     if (m > S) m = S;
-    // samples: thread t holds samples t and t + kTopkThreads
-    uint32_t sk[1024 / kTopkThreads];
-#pragma unroll
-    for (int q = 0; q < 1024 / kTopkThreads; ++q) {
-      const int sidx = tid + q * kTopkThreads;
-      sk[q] = sidx < S ? topk_key(__ldg(row + (int)(((int64_t)sidx * nn) / S))) : 0u;
+    // samples: 64 evenly spaced runs of 16 consecutive scores (one float4 per thread for
+    // 256 threads), or the whole row when it is shorter than 1024; kept in the candidate
+    // area, which the candidate pass overwrites only afterwards
+    if (nn >= 1024) {
+      if (tid < 256) {
+        const int blk = tid >> 2;
+        const int start = (int)(((int64_t)blk * (nn - 16)) / 63) & ~3;
+        uint32_t k4[4];
+        load4(start + 4 * (tid & 3), k4);
+        *reinterpret_cast<uint4*>(fk + 4 * tid) = make_uint4(k4[0], k4[1], k4[2], k4[3]);
+      }
+    } else {
+      for (int j = tid; j < nn; j += kTopkThreads) fk[j] = topk_key(__ldg(row + j));
     }
-    auto sget = [&](uint32_t c) -> uint32_t { return sk[(c - tid) / kTopkThreads]; };
+    __syncthreads();
+    auto sget = [&](uint32_t c) -> uint32_t { return fk[c]; };
     uint32_t t_est;
     bool sw;
-    select(hA, hB, hC, (uint32_t)m, sget, (uint32_t)S, &t_est, &sw);
-    // every sample >= t_est counts towards m, so t_est is the estimate itself
+    // 22 bits of the estimate are plenty: every sample >= t_est counts towards m
+    select(hA, hB, hC, (uint32_t)m, sget, (uint32_t)S, 2, &t_est, &sw);
+    __syncthreads();  // samples read; the candidate pass may overwrite them
 
-    // -- candidates: every key >= t_est, in position order
+    // -- candidates: every key >= t_est, in position order.  The comparison is done on the
+    // raw scores (key order = float order, -0.0 == +0.0); keys are formed only for the
+    // candidates.
+    const float t_val = topk_key_value(t_est);
     uint32_t run = 0;
     bool overflow = false;
     for (int cb = 0; cb < nn && !overflow; cb += kTopkRun) {
-      uint32_t kb[kTopkBatch][4];
+      float4 xb[kTopkBatch];
 #pragma unroll
-      for (int it = 0; it < kTopkBatch; ++it)  // warp w owns positions cb + 1024 w .. + 1023
-        load4(cb + warp * 1024 + it * 128 + lane * 4, kb[it]);
-      uint32_t fl = 0;                  // bit 4*it + q: key q of step it is kept
+      for (int it = 0; it < kTopkBatch; ++it) {  // warp w owns positions cb + 1024 w .. + 1023
+        const int j0 = cb + warp * 1024 + it * 128 + lane * 4;
+        if (j0 + 3 < nn) {
+          xb[it] = __ldg(reinterpret_cast<const float4*>(row + j0));
+        } else {
+          xb[it].x = j0 < nn ? __ldg(row + j0) : -INFINITY;
+          xb[it].y = j0 + 1 < nn ? __ldg(row + j0 + 1) : -INFINITY;
+          xb[it].z = j0 + 2 < nn ? __ldg(row + j0 + 2) : -INFINITY;
+          xb[it].w = j0 + 3 < nn ? __ldg(row + j0 + 3) : -INFINITY;
+        }
+      }
+      uint32_t fl = 0;                  // bit 4*it + q: score q of step it is kept
       uint32_t cnt_lo = 0, cnt_hi = 0;  // per-step counts packed in bytes
 #pragma unroll
       for (int it = 0; it < kTopkBatch; ++it) {
-        const int j0 = cb + warp * 1024 + it * 128 + lane * 4;
-        uint32_t f = 0;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) f |= (uint32_t)(j0 + q < nn && kb[it][q] >= t_est) << q;
+        const uint32_t f = (uint32_t)(xb[it].x >= t_val) | ((uint32_t)(xb[it].y >= t_val) << 1) |
+                           ((uint32_t)(xb[it].z >= t_val) << 2) | ((uint32_t)(xb[it].w >= t_val) << 3);
         fl |= f << (4 * it);
         if (it < 4) cnt_lo |= (uint32_t)__popc(f) << (8 * it);
         else cnt_hi |= (uint32_t)__popc(f) << (8 * (it - 4));
@@ -288,12 +323,15 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkArgs a) {
       for (int it = 0; it < kTopkBatch; ++it) {
         const uint32_t lo = it < 4 ? (exc_lo >> (8 * it)) & 255u : (exc_hi >> (8 * (it - 4))) & 255u;
         const uint32_t tt = it < 4 ? (tot_lo >> (8 * it)) & 255u : (tot_hi >> (8 * (it - 4))) & 255u;
-        uint32_t slot = pre + lo;
-        const int j0 = cb + warp * 1024 + it * 128 + lane * 4;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          if ((fl >> (4 * it + q)) & 1u) {
-            fk[slot] = kb[it][q];
+        uint32_t nib = (fl >> (4 * it)) & 15u;
+        if (nib) {
+          uint32_t slot = pre + lo;
+          const int j0 = cb + warp * 1024 + it * 128 + lane * 4;
+          while (nib) {
+            const int q = __ffs(nib) - 1;
+            nib &= nib - 1;
+            const float x = q == 0 ? xb[it].x : q == 1 ? xb[it].y : q == 2 ? xb[it].z : xb[it].w;
+            fk[slot] = topk_key(x);
             fp[slot] = (uint32_t)(j0 + q);
             ++slot;
           }
@@ -309,7 +347,7 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkArgs a) {
       auto cget = [&](uint32_t c) -> uint32_t { return fk[c]; };
       uint32_t tau;
       bool ge;
-      const uint32_t ties_needed = select(hD, hE, hF, (uint32_t)K, cget, C, &tau, &ge);
+      const uint32_t ties_needed = select(hD, hE, hF, (uint32_t)K, cget, C, 3, &tau, &ge);
       // -- ordered output over the candidates (they are in position order)
       uint32_t run_def = 0, run_tie = 0;
       for (uint32_t base = 0; base < C; base += 4 * kTopkThreads) {
