@@ -28,6 +28,7 @@
 namespace dsa {
 
 constexpr int kHeadDim = 128;
+constexpr float kLazyMax = 8.f;  // log2 units the running maximum may lag behind
 
 // Warps per CTA and ring depth per warp: 12 warps x 2 stages when a CTA holds at most 4
 // KV heads (more warps hide more latency), 8 warps x 3 stages for 8 KV heads.  Either
@@ -131,29 +132,29 @@ __global__ void __launch_bounds__(AttnGeom<HKV_CTA>::kThreads, 1) sparse_attn_ke
   const int64_t row_stride = (int64_t)a.Hkv * kHeadDim;
 
   // gather chunk c into ring slot st; returns the validity mask of its 16 positions.
-  // Lane t < 16 reads the index of position t and forms its row address once; every
-  // cp.async then moves two whole 256-byte head slices (512 contiguous bytes per warp
-  // instruction), the row address arriving by shuffle.
+  // Lane t < 16 reads the index of position t; every cp.async step then moves two whole
+  // 256-byte head slices (512 contiguous bytes per warp instruction), the row arriving by
+  // shuffle.  Padding and out-of-range entries copy the sequence's first row (finite data)
+  // and are masked in the softmax, so the copies need no per-piece predicate.
   const int lt = lane & 15, lhi = lane >> 4;
   const int64_t v_minus_k = a.v - a.k;  // V row = K row + this many elements
+  const __nv_bfloat16* kpiece = kh + kbase * row_stride + lt * 8;  // row 0, this lane's piece
+  const uint32_t swz = (uint32_t)((lt ^ lhi) << 4);  // lt ^ ((2k + lhi) & 7) = (lt ^ lhi) ^ 2k&7
   auto load_chunk = [&](int c, int st) -> uint32_t {
     const int e = c * CH + sub * 16 + lt;
     const int j = e < K ? __ldg(irow + e) : -1;
     const bool valid = j >= 0 && (int64_t)j <= p;
     const uint32_t vmask = __ballot_sync(0xFFFFFFFFu, valid) & 0xFFFFu;
-    const unsigned long long rowp =
-        reinterpret_cast<unsigned long long>(kh + (kbase + (valid ? j : 0)) * row_stride);
-    const uint32_t kdst = smem_u32(wsm + st * Geo::kWarpStage);
+    const int rowi = valid ? j : 0;
+    const uint32_t kdst = smem_u32(wsm + st * Geo::kWarpStage) + lhi * 256;
     const uint32_t vdst = kdst + Geo::kWarpHalf;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const int t = 2 * k + lhi;  // position handled by this lane in step k
-      const bool vt = (vmask >> t) & 1u;
-      const __nv_bfloat16* ks =
-          reinterpret_cast<const __nv_bfloat16*>(__shfl_sync(0xFFFFFFFFu, rowp, t)) + lt * 8;
-      const uint32_t so = (uint32_t)(t * 256 + ((lt ^ (t & 7)) << 4));
-      cp_async_16(kdst + so, vt ? (const void*)ks : (const void*)a.k, vt ? 16u : 0u);
-      cp_async_16(vdst + so, vt ? (const void*)(ks + v_minus_k) : (const void*)a.k, vt ? 16u : 0u);
+      const int rt = __shfl_sync(0xFFFFFFFFu, rowi, 2 * k + lhi);
+      const __nv_bfloat16* src = kpiece + (int64_t)rt * row_stride;
+      const uint32_t so = (uint32_t)(k * 512) + (swz ^ (uint32_t)(((2 * k) & 7) << 4));
+      cp_async_16(kdst + so, src, 16u);
+      cp_async_16(vdst + so, src + v_minus_k, 16u);
     }
     return vmask;
   };
@@ -237,38 +238,46 @@ __global__ void __launch_bounds__(AttnGeom<HKV_CTA>::kThreads, 1) sparse_attn_ke
       s[nt][1] = v_lo ? (s[nt][1] + s2[nt][1]) * a.scale_log2 : -INFINITY;
       s[nt][2] = v_hi ? (s[nt][2] + s2[nt][2]) * a.scale_log2 : -INFINITY;
       s[nt][3] = v_hi ? (s[nt][3] + s2[nt][3]) * a.scale_log2 : -INFINITY;
+      // Lazy running maximum: the reference m_run only moves (with a warp-wide max and a
+      // rescale of the partial sums) when some logit exceeds it by more than kLazyMax, so
+      // every weight stays <= 2^kLazyMax, well inside bf16 / fp32 range.
       float mx[2] = {fmaxf(s[nt][0], s[nt][2]), fmaxf(s[nt][1], s[nt][3])};
+      const bool need = !(mx[0] <= m_run[nt][0] + kLazyMax) || !(mx[1] <= m_run[nt][1] + kLazyMax) ||
+                        m_run[nt][0] == -INFINITY || m_run[nt][1] == -INFINITY;
+      float pr[4];
+      if (__any_sync(0xFFFFFFFFu, need)) {
+        float alpha[2];
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        mx[cc] = fmaxf(mx[cc], __shfl_xor_sync(0xFFFFFFFFu, mx[cc], 4));
-        mx[cc] = fmaxf(mx[cc], __shfl_xor_sync(0xFFFFFFFFu, mx[cc], 8));
-        mx[cc] = fmaxf(mx[cc], __shfl_xor_sync(0xFFFFFFFFu, mx[cc], 16));
-      }
-      float alpha[2], pr[4];
-      bool grew = false;
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        const float m_new = fmaxf(m_run[nt][cc], mx[cc]);
-        if (m_new == -INFINITY) {
-          alpha[cc] = 1.f;
-          pr[cc] = 0.f;
-          pr[cc + 2] = 0.f;
-        } else {
-          alpha[cc] = ex2_approx(m_run[nt][cc] - m_new);
-          pr[cc] = ex2_approx(s[nt][cc] - m_new);
-          pr[cc + 2] = ex2_approx(s[nt][cc + 2] - m_new);
+        for (int cc = 0; cc < 2; ++cc) {
+          mx[cc] = fmaxf(mx[cc], __shfl_xor_sync(0xFFFFFFFFu, mx[cc], 4));
+          mx[cc] = fmaxf(mx[cc], __shfl_xor_sync(0xFFFFFFFFu, mx[cc], 8));
+          mx[cc] = fmaxf(mx[cc], __shfl_xor_sync(0xFFFFFFFFu, mx[cc], 16));
+          const float m_new = fmaxf(m_run[nt][cc], mx[cc]);
+          if (m_new == -INFINITY) {
+            alpha[cc] = 1.f;
+            pr[cc] = 0.f;
+            pr[cc + 2] = 0.f;
+          } else {
+            alpha[cc] = ex2_approx(m_run[nt][cc] - m_new);
+            pr[cc] = ex2_approx(s[nt][cc] - m_new);
+            pr[cc + 2] = ex2_approx(s[nt][cc + 2] - m_new);
+          }
+          m_run[nt][cc] = m_new;
+          l_run[nt][cc] = l_run[nt][cc] * alpha[cc] + pr[cc] + pr[cc + 2];
         }
-        grew |= m_new != m_run[nt][cc];
-        m_run[nt][cc] = m_new;
-        l_run[nt][cc] = l_run[nt][cc] * alpha[cc] + pr[cc] + pr[cc + 2];
-      }
-      if (__any_sync(0xFFFFFFFFu, grew)) {  // a running max moved: rescale the partial sums
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
           o[nt][mt][0] *= alpha[0];
           o[nt][mt][1] *= alpha[1];
           o[nt][mt][2] *= alpha[0];
           o[nt][mt][3] *= alpha[1];
+        }
+      } else {
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          pr[cc] = ex2_approx(s[nt][cc] - m_run[nt][cc]);
+          pr[cc + 2] = ex2_approx(s[nt][cc + 2] - m_run[nt][cc]);
+          l_run[nt][cc] += pr[cc] + pr[cc + 2];
         }
       }
       // P = P_hi + P_lo, both bf16: the P.V product keeps ~16 significant bits of P
