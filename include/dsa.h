@@ -143,6 +143,39 @@ dsa_status dsa_topk(const dsa_params* params, const dsa_ragged* ragged, const fl
                     int64_t ld_idx, int32_t* cnt, void* stream);
 
 /*
+ * Steps 1-2 fused - the index rows of dsa_index_scores followed by dsa_topk, without
+ * writing the score matrix ([GSA] section 4: whether the Top-K selection can be fused
+ * into kernels; [HSA] "Engineering and Evaluation Recommendations": dedicated fused
+ * Top-K kernels).  The pages name the fusion as an engineering goal and give no method;
+ * this one is exact:
+ *   a. the indexer over every 16th key position gives each row a sample of its scores;
+ *   b. from the sample, a threshold t per row with, with overwhelming probability, at
+ *      least K of the row's scores >= t and not many more;
+ *   c. the indexer over all keys keeps only the (position, score) pairs with score >= t;
+ *   d. when a row has between K and the slot count of such candidates they contain its
+ *      Top-K with every tie, and an exact radix select over them gives the result;
+ *      a row whose threshold missed has its scores recomputed (CUDA cores, fp32) and
+ *      selected exactly.
+ * Output: exactly what dsa_index_scores + dsa_topk give on inputs whose scores are exact
+ * in fp32 (e.g. dyadic values); otherwise the Top-K of fp32 scores whose rounding may
+ * differ in the last bit for a row that was recomputed in step d.
+ *   q_idx, k_idx, w   as dsa_index_scores
+ *   idx, ld_idx, cnt  as dsa_topk (rows q_begin .. q_begin+q_count-1)
+ *   workspace device, 256-byte aligned, ws_bytes >= the minimum of
+ *             dsa_index_topk_workspace_size; rows are processed in passes of as many
+ *             as it holds (the recommended size holds all q_count rows).  Nothing in it
+ *             has to be initialised; its contents are undefined afterwards.
+ * Returns DSA_ERR_UNSUPPORTED when K is too large for the candidate slots (about
+ * K > 4500) or max_kv_len exceeds 314496; dsa_index_scores + dsa_topk cover those.
+ */
+dsa_status dsa_index_topk_workspace_size(const dsa_params* params, const dsa_ragged* ragged,
+                                         int64_t q_count, size_t* min_bytes, size_t* rec_bytes);
+dsa_status dsa_index_topk(const dsa_params* params, const dsa_ragged* ragged, const void* q_idx,
+                          const void* k_idx, const float* w, int64_t q_begin, int64_t q_count,
+                          int32_t* idx, int64_t ld_idx, int32_t* cnt, void* workspace,
+                          size_t ws_bytes, void* stream);
+
+/*
  * Steps 3-4 - exact softmax attention over the selected rows with the sigmoid output
  * gate fused in ([HSA] steps 3-4 and pseudocode; [SAE] section 5; [GSA] section 2).
  *   q        bf16 [total_q, Hq, d]
@@ -167,7 +200,11 @@ dsa_status dsa_sparse_attn_gated(const dsa_params* params, const dsa_ragged* rag
 /*
  * Workspace for dsa_prefill / dsa_decode.  *min_bytes: the least that works (one query
  * row of scores per pass); *rec_bytes: the size this build recommends for throughput
- * (bounded; fewer, larger passes).  Either pointer may be NULL.
+ * (fewer, larger passes).  Either pointer may be NULL.  dsa_prefill runs steps 1-2 as
+ * dsa_index_topk does when the batch is prefill-shaped (at least 256 query rows per
+ * sequence on average), its score matrix would exceed 256 MiB, the fused path supports
+ * K and max_kv_len, and the workspace holds fused passes of at least 2048 rows (or all
+ * rows); *rec_bytes then covers one fused pass over every row.
  */
 dsa_status dsa_workspace_size(const dsa_params* params, const dsa_ragged* ragged, int is_decode,
                               size_t* min_bytes, size_t* rec_bytes);

@@ -53,7 +53,7 @@ EXPORTS = [
     "dsa_status_string", "dsa_version", "dsa_index_scores", "dsa_topk",
     "dsa_sparse_attn_gated", "dsa_workspace_size", "dsa_prefill", "dsa_decode",
     "dsa_device_status", "dsa_launch_count", "dsa_stage_timing", "dsa_stage_times",
-    "dsa_decode_noalloc",
+    "dsa_decode_noalloc", "dsa_index_topk", "dsa_index_topk_workspace_size",
 ]
 
 
@@ -70,6 +70,8 @@ def _load():
     L.dsa_topk.argtypes = [PP, RP, vp, i64, i64, i64, vp, i64, vp, vp]
     L.dsa_sparse_attn_gated.argtypes = [PP, RP, vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, vp, vp]
     L.dsa_workspace_size.argtypes = [PP, RP, ctypes.c_int, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+    L.dsa_index_topk_workspace_size.argtypes = [PP, RP, i64, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+    L.dsa_index_topk.argtypes = [PP, RP, vp, vp, vp, i64, i64, vp, i64, vp, vp, sz, vp]
     L.dsa_prefill.argtypes = [PP, RP, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.dsa_decode.argtypes = L.dsa_prefill.argtypes
     L.dsa_decode_noalloc.argtypes = [PP, RP, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
@@ -168,6 +170,25 @@ def dsa_workspace_size(shape: LayerShape, rg: Ragged, is_decode: bool = False):
     _check(lib.dsa_workspace_size(ctypes.byref(p), ctypes.byref(rg), int(is_decode),
                                   ctypes.byref(mn), ctypes.byref(rec)), "dsa_workspace_size")
     return mn.value, rec.value
+
+
+def dsa_index_topk_workspace_size(shape: LayerShape, rg: Ragged, q_count: int):
+    p = shape.params()
+    mn, rec = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check(lib.dsa_index_topk_workspace_size(ctypes.byref(p), ctypes.byref(rg), q_count,
+                                             ctypes.byref(mn), ctypes.byref(rec)),
+           "dsa_index_topk_workspace_size")
+    return mn.value, rec.value
+
+
+def dsa_index_topk(shape: LayerShape, rg: Ragged, q_idx, k_idx, w, q_begin: int, q_count: int,
+                   idx, ld_idx: int, cnt=None, workspace=None, ws_bytes=None, stream=None):
+    p = shape.params()
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.dsa_index_topk(ctypes.byref(p), ctypes.byref(rg), _ptr(q_idx), _ptr(k_idx),
+                              _ptr(w), q_begin, q_count, _ptr(idx), ld_idx, _ptr(cnt),
+                              _ptr(workspace), ws_bytes, _stream(stream)), "dsa_index_topk")
 
 
 def _layer(fn, name, shape, rg, q_idx, k_idx, w, q, k_cache, v_cache, gate, out, idx_out,

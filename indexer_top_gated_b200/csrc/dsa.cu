@@ -101,11 +101,18 @@ dsa_status device_setup(DeviceState** out) {
     d.max_smem = (size_t)smem_optin;
     const size_t idx_max = idx_smem_bytes(4, 64, false);
     cudaError_t e = cudaSuccess;
-    e = e ? e : allow_smem(idx_scores_kernel<64, false>, idx_max);
-    e = e ? e : allow_smem(idx_scores_kernel<16, false>, idx_max);
-    e = e ? e : allow_smem(idx_scores_kernel<64, true>, idx_max);
-    e = e ? e : allow_smem(idx_scores_kernel<16, true>, idx_max);
-    e = e ? e : allow_smem(topk_kernel, topk_smem_bytes(0));
+    e = e ? e : allow_smem(idx_scores_kernel<64, false, false>, idx_max);
+    e = e ? e : allow_smem(idx_scores_kernel<16, false, false>, idx_max);
+    e = e ? e : allow_smem(idx_scores_kernel<64, true, false>, idx_max);
+    e = e ? e : allow_smem(idx_scores_kernel<16, true, false>, idx_max);
+    const size_t cand_max = idx_smem_bytes(4, 64, false, true);
+    e = e ? e : allow_smem(idx_scores_kernel<64, false, true>, cand_max);
+    e = e ? e : allow_smem(idx_scores_kernel<16, false, true>, cand_max);
+    e = e ? e : allow_smem(idx_scores_kernel<64, true, true>, cand_max);
+    e = e ? e : allow_smem(idx_scores_kernel<16, true, true>, cand_max);
+    e = e ? e : allow_smem(topk_kernel<kTopkScores>, topk_smem_bytes(0));
+    e = e ? e : allow_smem(topk_kernel<kTopkFused>, topk_fused_smem_bytes(kTopkFastCap, kTopkFusedMaxN));
+    e = e ? e : allow_smem(topk_kernel<kTopkFallback>, topk_smem_bytes(0));
     e = e ? e : allow_smem(sparse_attn_kernel<1, 1>, attn_smem_bytes());
     e = e ? e : allow_smem(sparse_attn_kernel<2, 1>, attn_smem_bytes());
     e = e ? e : allow_smem(sparse_attn_kernel<4, 1>, attn_smem_bytes());
@@ -171,6 +178,15 @@ dsa_status check_attn(const dsa_params* P) {
     if (_s != DSA_OK) return _s;     \
   } while (0)
 
+// Status of the launch just made: DSA_ERR_CUDA, with one line on stderr naming the kernel
+// and CUDA's error, when it failed.
+dsa_status launch_status(const char* kernel) {
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return DSA_OK;
+  std::fprintf(stderr, "dsa: launch of %s failed: %s\n", kernel, cudaGetErrorString(e));
+  return DSA_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------- launches
 dsa_status make_idx_map(CUtensorMap* map, const void* base, int64_t rows, int n_heads, bool fp8,
                         int box_rows) {
@@ -187,15 +203,30 @@ dsa_status make_idx_map(CUtensorMap* map, const void* base, int64_t rows, int n_
   return r == CUDA_SUCCESS ? DSA_OK : DSA_ERR_INVALID_ARG;
 }
 
+// Variants of the indexer launch used by the fused indexer -> Top-K path.
+struct IdxVariant {
+  int shift = 0;                   // > 0: keys are the sampled key tensor below
+  const void* k_rows = nullptr;    // sampled key tensor
+  int64_t k_rows_n = 0;            // its rows
+  const float* thr = nullptr;      // non-null: candidate variant
+  float2* cand = nullptr;
+  int cap = 0;
+  int32_t* cand_cnt = nullptr;
+};
+
 dsa_status launch_index_scores(const DeviceState& dev, const dsa_params* P, const dsa_ragged* R,
                                const void* q_idx, const void* k_idx, const float* w,
                                int64_t q_begin, int64_t q_count, float* scores, int64_t ld,
-                               int bq, cudaStream_t stream) {
+                               int bq, cudaStream_t stream, const IdxVariant& var = IdxVariant()) {
   if (q_count == 0 || R->total_kv == 0) return DSA_OK;
   const bool fp8 = P->idx_dtype == DSA_FP8_E4M3;
+  const bool cand = var.thr != nullptr;
   CUtensorMap mq, mk;
   DSA_TRY(make_idx_map(&mq, q_idx, R->total_q, P->n_idx_heads, fp8, bq));
-  DSA_TRY(make_idx_map(&mk, k_idx, R->total_kv, P->n_idx_heads, fp8, kIdxKeyTile));
+  if (var.shift)
+    DSA_TRY(make_idx_map(&mk, var.k_rows, var.k_rows_n, P->n_idx_heads, fp8, kIdxKeyTile));
+  else
+    DSA_TRY(make_idx_map(&mk, k_idx, R->total_kv, P->n_idx_heads, fp8, kIdxKeyTile));
   IdxArgs a;
   a.q_offsets = R->q_offsets;
   a.kv_offsets = R->kv_offsets;
@@ -204,12 +235,14 @@ dsa_status launch_index_scores(const DeviceState& dev, const dsa_params* P, cons
   a.q_begin = q_begin;
   a.q_count = q_count;
   a.n_tiles = (int)((q_count + bq - 1) / bq);
-  const int max_kt = std::max(1, (R->max_kv_len + kIdxKeyTile - 1) / kIdxKeyTile);
-  // enough CTAs to fill the GPU a few times over, at least 8 key tiles per CTA
+  const int64_t max_keys = R->max_kv_len > 0 ? ((int64_t)(R->max_kv_len - 1) >> var.shift) + 1 : 1;
+  const int max_kt = (int)std::max<int64_t>(1, (max_keys + kIdxKeyTile - 1) / kIdxKeyTile);
+  // enough CTAs to fill the GPU a few times over, at least 8 key tiles per CTA; the
+  // candidate variant keeps every key tile of a row in one CTA
   const int64_t target = (int64_t)dev.num_sms * 8;
   int ysplit = (int)std::min<int64_t>((target + a.n_tiles - 1) / a.n_tiles,
                                       std::max(1, max_kt / 8));
-  ysplit = std::max(ysplit, 1);
+  ysplit = cand ? 1 : std::max(ysplit, 1);
   a.kt_per_split = (max_kt + ysplit - 1) / ysplit;
   ysplit = (max_kt + a.kt_per_split - 1) / a.kt_per_split;
   a.w = w;
@@ -218,18 +251,28 @@ dsa_status launch_index_scores(const DeviceState& dev, const dsa_params* P, cons
   a.scores = scores;
   a.ld = ld;
   a.status = dev.status;
-  const size_t smem = idx_smem_bytes(P->n_idx_heads, bq, fp8);
+  a.shift = var.shift;
+  a.thr = var.thr;
+  a.cand = var.cand;
+  a.cap = var.cap;
+  a.cand_cnt = var.cand_cnt;
+  const size_t smem = idx_smem_bytes(P->n_idx_heads, bq, fp8, cand);
   dim3 grid((unsigned)a.n_tiles, (unsigned)ysplit);
   StageScope scope(0, stream);
-  if (bq == 64) {
-    if (fp8) idx_scores_kernel<64, true><<<grid, kIdxThreads, smem, stream>>>(mq, mk, a);
-    else idx_scores_kernel<64, false><<<grid, kIdxThreads, smem, stream>>>(mq, mk, a);
-  } else {
-    if (fp8) idx_scores_kernel<16, true><<<grid, kIdxThreads, smem, stream>>>(mq, mk, a);
-    else idx_scores_kernel<16, false><<<grid, kIdxThreads, smem, stream>>>(mq, mk, a);
-  }
+#define DSA_IDX_CASE(BQ, F8, C)                                                      \
+  if (bq == BQ && fp8 == F8 && cand == C)                                            \
+    idx_scores_kernel<BQ, F8, C><<<grid, kIdxThreads, smem, stream>>>(mq, mk, a);
+  DSA_IDX_CASE(64, false, false)
+  DSA_IDX_CASE(64, true, false)
+  DSA_IDX_CASE(16, false, false)
+  DSA_IDX_CASE(16, true, false)
+  DSA_IDX_CASE(64, false, true)
+  DSA_IDX_CASE(64, true, true)
+  DSA_IDX_CASE(16, false, true)
+  DSA_IDX_CASE(16, true, true)
+#undef DSA_IDX_CASE
   ++t_launches;
-  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  return launch_status("idx_scores_kernel");
 }
 
 dsa_status launch_topk(const dsa_params* P, const dsa_ragged* R, const float* scores, int64_t ld,
@@ -237,6 +280,7 @@ dsa_status launch_topk(const dsa_params* P, const dsa_ragged* R, const float* sc
                        int32_t* cnt, cudaStream_t stream) {
   if (q_count == 0) return DSA_OK;
   TopkArgs a;
+  std::memset(&a, 0, sizeof(a));
   a.q_offsets = R->q_offsets;
   a.kv_offsets = R->kv_offsets;
   a.batch = R->batch;
@@ -250,9 +294,196 @@ dsa_status launch_topk(const dsa_params* P, const dsa_ragged* R, const float* sc
   a.cnt = cnt;
   const size_t smem = topk_smem_bytes(R->max_kv_len);
   StageScope scope(1, stream);
-  topk_kernel<<<(unsigned)q_count, kTopkThreads, smem, stream>>>(a);
+  topk_kernel<kTopkScores><<<(unsigned)q_count, kTopkThreads, smem, stream>>>(a);
   ++t_launches;
-  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  return launch_status("topk_kernel");
+}
+
+// ---------------------------------------------------------------- fused indexer -> Top-K
+//
+// Per pass of rows: (1) the indexer over every 16th key (samples), (2) a threshold estimate
+// per row from its samples, (3) the indexer again over all keys keeping only the scores
+// >= the estimate as candidates, (4) an exact selection over the candidates, (5) the rows
+// whose estimate missed, recomputed and selected exactly.  The sampled key tensor is built
+// once per call.
+constexpr int kSampleShift = 4;
+constexpr int kFallbackCtas = 128;
+
+struct FusedGeom {
+  int cap;              // candidate slots per row
+  int64_t ld_s;         // floats per sample row
+  int64_t ld_fb;        // floats per fallback scratch row
+  int64_t samp_rows;    // rows of the sampled key tensor
+  int64_t key_row;      // bytes per key row
+  int64_t fixed_bytes;  // sampled keys + fallback scratch
+  int64_t row_bytes;    // per query row: samples / candidates (shared), threshold, count, list
+};
+
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+// false when the fused path cannot take this problem (K or the rows too long)
+bool fused_geom(const dsa_params* P, const dsa_ragged* R, FusedGeom* g) {
+  const int K = P->top_k;
+  const double s = double(1 << kSampleShift);
+  // samples of rank R = e + 5 sqrt(e) + 16 (e = K / 16 + 1 at most) leave about 16 R
+  // candidates; the slots cover 6 standard deviations more
+  const double e = K / s + 1.0;
+  const double rr = std::ceil(e + 5.0 * std::sqrt(e) + 16.0);
+  const int64_t cap = round_up((int64_t)std::ceil(s * (rr + 6.0 * std::sqrt(rr))), 256);
+  if (cap > kTopkFastCap || cap < K) return false;
+  if (R->max_kv_len > kTopkFusedMaxN) return false;
+  g->cap = (int)cap;
+  const int64_t max_n = std::max(R->max_kv_len, 1);
+  g->ld_s = round_up(((max_n - 1) >> kSampleShift) + 1, 32);
+  g->ld_fb = round_up(max_n, 4);
+  g->samp_rows = (R->total_kv >> kSampleShift) + R->batch + 1;
+  g->key_row = (int64_t)P->n_idx_heads * 64 * (P->idx_dtype == DSA_FP8_E4M3 ? 1 : 2);
+  g->fixed_bytes = round_up(g->samp_rows * g->key_row, 256) +
+                   round_up((int64_t)kFallbackCtas * g->ld_fb * 4, 256) + 256 * 4;
+  g->row_bytes = std::max<int64_t>(g->ld_s * 4, cap * 8) + 6 * 4;
+  return true;
+}
+
+// Rows of one fused pass that `bytes` of workspace hold (0 if not even one).
+int64_t fused_rows(const FusedGeom& g, int64_t bytes) {
+  return bytes > g.fixed_bytes ? (bytes - g.fixed_bytes) / g.row_bytes : 0;
+}
+
+// The layer takes the fused path for prefill-shaped batches (few sequences, many query
+// rows each) whose score matrix would be far larger than L2; smaller problems keep their
+// scores in L2 anyway, and batches of many short sequences suit the split key ranges of
+// the materialised path.
+constexpr int64_t kFusedMinScoreBytes = int64_t(256) << 20;
+constexpr int64_t kFusedMinRows = 2048;
+
+bool fused_wanted(const dsa_params* P, const dsa_ragged* R, FusedGeom* g) {
+  if (!fused_geom(P, R, g)) return false;
+  if ((int64_t)R->batch * 256 > R->total_q) return false;
+  return R->total_q * (int64_t)R->max_kv_len * 2 > kFusedMinScoreBytes;
+}
+
+struct FusedWs {
+  uint4* k_samp;
+  float* fb_scores;
+  char* sc;        // samples [rows, ld_s] floats, later candidates [rows, cap] float2
+  float* thr;
+  int32_t* ccnt;   // [rows, 4]
+  int32_t* list;   // [1 + rows]
+};
+
+FusedWs fused_carve(const FusedGeom& g, void* ws, int64_t rows) {
+  char* p = static_cast<char*>(ws);
+  FusedWs f;
+  f.k_samp = reinterpret_cast<uint4*>(p);
+  p += round_up(g.samp_rows * g.key_row, 256);
+  f.fb_scores = reinterpret_cast<float*>(p);
+  p += round_up((int64_t)kFallbackCtas * g.ld_fb * 4, 256);
+  f.sc = p;
+  p += round_up(rows * std::max<int64_t>(g.ld_s * 4, (int64_t)g.cap * 8), 256);
+  f.thr = reinterpret_cast<float*>(p);
+  p += round_up(rows * 4, 256);
+  f.ccnt = reinterpret_cast<int32_t*>(p);
+  p += round_up(rows * 16, 256);
+  f.list = reinterpret_cast<int32_t*>(p);
+  return f;
+}
+
+dsa_status fused_prepare(const DeviceState& dev, const dsa_ragged* R, const void* k_idx, const FusedGeom& g, const FusedWs& f,
+                         cudaStream_t stream) {
+  const int vec = (int)(g.key_row / 16);
+  const int64_t blocks = std::min<int64_t>((g.samp_rows + 7) / 8, (int64_t)dev.num_sms * 8);
+  StageScope scope(0, stream);
+  idx_sample_keys_kernel<<<(unsigned)std::max<int64_t>(blocks, 1), 256, 0, stream>>>(
+      R->kv_offsets, R->batch, kSampleShift, static_cast<const uint4*>(k_idx), f.k_samp, vec,
+      g.samp_rows);
+  ++t_launches;
+  return launch_status("idx_sample_keys_kernel");
+}
+
+dsa_status fused_pass(const DeviceState& dev, const dsa_params* P, const dsa_ragged* R,
+                      const void* q_idx, const void* k_idx, const float* w, int64_t q_begin,
+                      int64_t q_count, int32_t* idx, int64_t ld_idx, int32_t* cnt,
+                      const FusedGeom& g, const FusedWs& f, cudaStream_t stream) {
+  if (q_count == 0) return DSA_OK;
+  const int bq = R->max_q_len <= 16 ? 16 : 64;
+  float* samp = reinterpret_cast<float*>(f.sc);
+  {  // (1) sampled scores
+    IdxVariant v;
+    v.shift = kSampleShift;
+    v.k_rows = f.k_samp;
+    v.k_rows_n = g.samp_rows;
+    DSA_TRY(launch_index_scores(dev, P, R, q_idx, k_idx, w, q_begin, q_count, samp, g.ld_s, bq,
+                                stream, v));
+  }
+  {  // (2) thresholds
+    TopkThrArgs t;
+    t.q_offsets = R->q_offsets;
+    t.kv_offsets = R->kv_offsets;
+    t.batch = R->batch;
+    t.q_begin = q_begin;
+    t.q_count = q_count;
+    t.K = P->top_k;
+    t.cap = g.cap;
+    t.shift = kSampleShift;
+    t.samp = samp;
+    t.ld_s = g.ld_s;
+    t.thr = f.thr;
+    t.fb_list = f.list;
+    StageScope scope(1, stream);
+    topk_thr_kernel<<<(unsigned)((q_count + kThrWarps - 1) / kThrWarps), 32 * kThrWarps, 0,
+                      stream>>>(t);
+    ++t_launches;
+    DSA_TRY(launch_status("topk_thr_kernel"));
+  }
+  {  // (3) candidates
+    IdxVariant v;
+    v.thr = f.thr;
+    v.cand = reinterpret_cast<float2*>(f.sc);
+    v.cap = g.cap;
+    v.cand_cnt = f.ccnt;
+    DSA_TRY(launch_index_scores(dev, P, R, q_idx, k_idx, w, q_begin, q_count, nullptr, 0, bq,
+                                stream, v));
+  }
+  TopkArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.q_offsets = R->q_offsets;
+  a.kv_offsets = R->kv_offsets;
+  a.batch = R->batch;
+  a.q_begin = q_begin;
+  a.q_count = q_count;
+  a.K = P->top_k;
+  a.idx = idx;
+  a.ld_idx = ld_idx;
+  a.cnt = cnt;
+  a.cand = reinterpret_cast<const float2*>(f.sc);
+  a.cap = g.cap;
+  a.cand_cnt = f.ccnt;
+  a.fb_list = f.list;
+  a.q_idx = q_idx;
+  a.k_idx = k_idx;
+  a.idx_heads = P->n_idx_heads;
+  a.idx_fp8 = P->idx_dtype == DSA_FP8_E4M3 ? 1 : 0;
+  a.w = w;
+  a.w_row_stride = P->w_row_stride;
+  a.idx_scale = P->idx_scale_q * P->idx_scale_k;
+  a.fb_scores = f.fb_scores;
+  a.ld_fb = g.ld_fb;
+  const size_t smem = topk_smem_bytes(R->max_kv_len);
+  a.bm_words = topk_fused_bm_words(std::max(R->max_kv_len, 1));
+  {  // (4) exact selection over the candidates
+    StageScope scope(1, stream);
+    topk_kernel<kTopkFused><<<(unsigned)q_count, kTopkThreads,
+                              topk_fused_smem_bytes(g.cap, R->max_kv_len), stream>>>(a);
+    ++t_launches;
+    DSA_TRY(launch_status("topk_kernel (fused selection)"));
+  }
+  {  // (5) rows whose estimate missed
+    StageScope scope(1, stream);
+    topk_kernel<kTopkFallback><<<kFallbackCtas, kTopkThreads, smem, stream>>>(a);
+    ++t_launches;
+    DSA_TRY(launch_status("topk_kernel (fallback rows)"));
+  }
+  return DSA_OK;
 }
 
 dsa_status launch_attn(const DeviceState& dev, const dsa_params* P, const dsa_ragged* R,
@@ -301,10 +532,8 @@ dsa_status launch_attn(const DeviceState& dev, const dsa_params* P, const dsa_ra
   DSA_ATTN_CASE(8, 2)
 #undef DSA_ATTN_CASE
   ++t_launches;
-  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  return launch_status("sparse_attn_kernel");
 }
-
-int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 
 // Workspace per pass row: scores row (ld floats) plus an index row when idx_out is absent.
 int64_t scores_ld(const dsa_ragged* R) { return round_up(std::max(R->max_kv_len, 1), 32); }
@@ -360,6 +589,28 @@ dsa_status run_layer(const dsa_params* P, const dsa_ragged* R, const void* q_idx
   if (!plan_passes(R->total_q, ld * 4, irow, (int64_t)ws_bytes, dev->num_sms, &plan))
     return DSA_ERR_WORKSPACE;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  FusedGeom fg;
+  if (!decode && fused_wanted(P, R, &fg)) {
+    // fused indexer -> Top-K, in passes of as many rows as the workspace holds (with their
+    // index rows when the caller keeps none)
+    const int64_t rows = std::min<int64_t>(
+        R->total_q, std::max<int64_t>(0, ((int64_t)ws_bytes - fg.fixed_bytes - 256) /
+                                             (fg.row_bytes + irow)));
+    if (rows >= std::min<int64_t>(R->total_q, kFusedMinRows)) {
+      const FusedWs f = fused_carve(fg, ws, rows);
+      int32_t* idx_ws = reinterpret_cast<int32_t*>(
+          static_cast<char*>(ws) + round_up(fg.fixed_bytes + rows * fg.row_bytes, 256));
+      DSA_TRY(fused_prepare(*dev, R, k_idx, fg, f, stream));
+      for (int64_t a0 = 0; a0 < R->total_q; a0 += rows) {
+        const int64_t cnt_a = std::min<int64_t>(rows, R->total_q - a0);
+        int32_t* idx = idx_out ? idx_out + a0 * K : idx_ws;
+        DSA_TRY(fused_pass(*dev, P, R, q_idx, k_idx, w, a0, cnt_a, idx, K, nullptr, fg, f, stream));
+        DSA_TRY(launch_attn(*dev, P, R, q, k, v, idx, K, a0, cnt_a, gate, out, nullptr, err_count,
+                            stream));
+      }
+      return DSA_OK;
+    }
+  }
   float* scores = static_cast<float*>(ws);
   int32_t* idx_ws = idx_out ? nullptr
                             : reinterpret_cast<int32_t*>(static_cast<char*>(ws) +
@@ -453,11 +704,16 @@ dsa_status dsa_sparse_attn_gated(const dsa_params* P, const dsa_ragged* R, const
 
 dsa_status dsa_workspace_size(const dsa_params* P, const dsa_ragged* R, int is_decode,
                               size_t* min_bytes, size_t* rec_bytes) {
-  (void)is_decode;
   DSA_TRY(check_common(P, R));
   const int64_t srow = scores_ld(R) * 4;
   const int64_t irow = round_up((int64_t)P->top_k * 4, 16);
   if (min_bytes) *min_bytes = (size_t)(srow + irow);
+  FusedGeom fg;
+  if (rec_bytes && !is_decode && fused_wanted(P, R, &fg)) {
+    // one fused pass over every query row
+    *rec_bytes = (size_t)(fg.fixed_bytes + 256 + std::max<int64_t>(1, R->total_q) * (fg.row_bytes + irow));
+    return DSA_OK;
+  }
   if (rec_bytes) {
     // a score sub-pass of up to kScorePassBytes (at least one row per SM) plus index rows
     // for attention passes of up to 16384 query rows
@@ -466,6 +722,48 @@ dsa_status dsa_workspace_size(const dsa_params* P, const dsa_ragged* R, int is_d
     rows_s = std::max<int64_t>(1, std::min(rows_s, tq));
     const int64_t rows_a = std::max(rows_s, std::min<int64_t>(tq, 16384));
     *rec_bytes = (size_t)(rows_s * srow + rows_a * irow);
+  }
+  return DSA_OK;
+}
+
+dsa_status dsa_index_topk_workspace_size(const dsa_params* P, const dsa_ragged* R,
+                                         int64_t q_count, size_t* min_bytes, size_t* rec_bytes) {
+  DSA_TRY(check_common(P, R));
+  DSA_TRY(check_indexer(P));
+  if (q_count < 0) return DSA_ERR_INVALID_ARG;
+  FusedGeom g;
+  if (!fused_geom(P, R, &g)) return DSA_ERR_UNSUPPORTED;
+  if (min_bytes) *min_bytes = (size_t)(g.fixed_bytes + g.row_bytes);
+  if (rec_bytes) *rec_bytes = (size_t)(g.fixed_bytes + std::max<int64_t>(1, q_count) * g.row_bytes);
+  return DSA_OK;
+}
+
+dsa_status dsa_index_topk(const dsa_params* P, const dsa_ragged* R, const void* q_idx,
+                          const void* k_idx, const float* w, int64_t q_begin, int64_t q_count,
+                          int32_t* idx, int64_t ld_idx, int32_t* cnt, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  DSA_TRY(check_common(P, R));
+  DSA_TRY(check_indexer(P));
+  if (!q_idx || !k_idx || !w || !idx) return DSA_ERR_INVALID_ARG;
+  if (q_begin < 0 || q_count < 0 || q_begin + q_count > R->total_q) return DSA_ERR_INVALID_ARG;
+  if (ld_idx < P->top_k) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx)) return DSA_ERR_INVALID_ARG;
+  if (q_count > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  FusedGeom g;
+  if (!fused_geom(P, R, &g)) return DSA_ERR_UNSUPPORTED;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255)) return DSA_ERR_WORKSPACE;
+  const int64_t rows = std::min<int64_t>(q_count, fused_rows(g, (int64_t)ws_bytes));
+  if (fused_rows(g, (int64_t)ws_bytes) < 1) return DSA_ERR_WORKSPACE;
+  if (q_count == 0) return DSA_OK;
+  DeviceState* dev = nullptr;
+  DSA_TRY(device_setup(&dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const FusedWs f = fused_carve(g, workspace, rows);
+  DSA_TRY(fused_prepare(*dev, R, k_idx, g, f, st));
+  for (int64_t s0 = q_begin; s0 < q_begin + q_count; s0 += rows) {
+    const int64_t n = std::min<int64_t>(rows, q_begin + q_count - s0);
+    DSA_TRY(fused_pass(*dev, P, R, q_idx, k_idx, w, s0, n, idx + (s0 - q_begin) * ld_idx, ld_idx,
+                       cnt ? cnt + (s0 - q_begin) : nullptr, g, f, st));
   }
   return DSA_OK;
 }

@@ -18,6 +18,20 @@
 //    first (the last rows of a sequence see the most keys).
 //  - Every wait is bounded; on a timeout the CTA records it, waits (bounded) for its
 //    own copies and MMAs in flight, frees TMEM and returns.
+//
+// Two variants serve the fused indexer -> Top-K path (no score matrix in HBM):
+//  - sampled keys (shift > 0): the key tensor holds every 2^shift-th cache position of
+//    each sequence (sequence b's samples start at row (kv_offsets[b] >> shift) + b), and
+//    sample m stands for position m << shift, so the causal bound becomes m <= p >> shift;
+//  - candidates (CAND): instead of storing every score, the epilogue keeps only the
+//    scores >= a per-row threshold as (position, score) pairs.  A CTA then owns every
+//    key tile of its rows (kt_per_split covers the whole range).  A row's list has one
+//    segment per TMEM lane quadrant (cap / 4 slots each), written only by the epilogue
+//    warp of that quadrant that owns the row's chunk of 16 rows, so a plain shared
+//    counter per (quadrant, row) suffices.  The warp stashes its 16 x 32 block of scores
+//    in shared memory and reads it back transposed: each lane then compares 16 keys of
+//    one row, counts its hits with one popcount and stores them in a short loop.  The
+//    2 KiB per warp come out of the key ring, which has 2 stages in this variant.
 #pragma once
 
 #include "common.cuh"
@@ -39,9 +53,24 @@ struct IdxArgs {
   float* scores;
   int64_t ld;
   int* status;
+  int shift;           // > 0: key rows are every 2^shift-th position (sampled keys)
+  // candidate variant
+  const float* thr;    // [q_count] keep scores >= thr[row - q_begin]
+  float2* cand;        // [q_count, cap]: 4 segments of cap/4 (position as int bits, score)
+  int cap;             // a multiple of 4
+  int32_t* cand_cnt;   // [q_count, 4] candidates found per segment (may exceed cap/4)
 };
 
-constexpr int kIdxStages = 3;
+// first key-tensor row of sequence b
+DSA_DEV int64_t idx_key_base(const IdxArgs& a, int b) {
+  const int64_t ko = __ldg(a.kv_offsets + b);
+  return a.shift ? (ko >> a.shift) + b : ko;
+}
+
+constexpr int kIdxStages = 3;      // key ring depth (the candidate variant uses 2)
+constexpr int kIdxCandStages = 2;
+constexpr int kIdxTileStride = 36;  // floats per row of a warp's score block (no bank conflicts)
+constexpr int kIdxTileBytes = 16 * kIdxTileStride * 4;
 constexpr int kIdxKeyTile = 128;
 constexpr int kIdxEpiWarps = 8;  // two warps per TMEM lane quadrant
 constexpr int kIdxThreads = 64 + 32 * kIdxEpiWarps;
@@ -65,11 +94,12 @@ __host__ __device__ inline int idx_tmem_cols(int n_heads, int bq) {
 // Dynamic shared memory of one CTA.  A CTA whose TMEM allocation exceeds a quarter of
 // the 512 columns asks for enough shared memory that CTAs sharing an SM can never
 // oversubscribe TMEM (an allocation that cannot be met would block).
-__host__ inline size_t idx_smem_bytes(int n_heads, int bq, bool fp8) {
+__host__ inline size_t idx_smem_bytes(int n_heads, int bq, bool fp8, bool cand = false) {
   size_t row = fp8 ? 64 : 128;
   size_t q = (size_t)n_heads * bq * row;
-  size_t k = (size_t)kIdxStages * n_heads * kIdxKeyTile * row;
-  size_t bytes = 1024 /*align slack*/ + q + k + 256 /*barriers*/;
+  size_t k = (size_t)(cand ? kIdxCandStages : kIdxStages) * n_heads * kIdxKeyTile * row;
+  size_t bytes = 1024 /*align slack*/ + q + k + 256 /*barriers*/ +
+                 (cand ? (size_t)kIdxEpiWarps * kIdxTileBytes : 0);
   const int cols = idx_tmem_cols(n_heads, bq);
   if (cols > 256 && bytes < 120 * 1024) bytes = 120 * 1024;       // 1 CTA per SM
   else if (cols > 128 && bytes < 80 * 1024) bytes = 80 * 1024;    // <= 2 CTAs per SM
@@ -77,12 +107,12 @@ __host__ inline size_t idx_smem_bytes(int n_heads, int bq, bool fp8) {
   return bytes;
 }
 
-template <int BQ, bool FP8>
+template <int BQ, bool FP8, bool CAND>
 __global__ void __launch_bounds__(kIdxThreads, 1)
     idx_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
                       const __grid_constant__ CUtensorMap tmap_k, IdxArgs a) {
   using Geo = IdxGeom<FP8>;
-  constexpr int ST = kIdxStages;
+  constexpr int ST = CAND ? kIdxCandStages : kIdxStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -97,10 +127,13 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   uint64_t* tfull = bars + 2 * ST;  // [2]
   uint64_t* tempty = tfull + 2;     // [2]
   uint64_t* qfull = tempty + 2;     // [1]
+  float* tiles = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);  // CAND
   __shared__ uint32_t s_tmem;
   __shared__ int s_bfirst, s_blast;
   __shared__ volatile int s_abort;
   __shared__ int s_consumed;  // jobs whose smem stage the MMA warp has released
+  __shared__ float s_thr[CAND ? BQ : 1];
+  __shared__ uint32_t s_cnt[CAND ? 4 : 1][CAND ? BQ : 1];  // candidates per (quadrant, row)
 
   const int warp = threadIdx.x >> 5;
   const int lane = lane_id();
@@ -129,7 +162,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     pbase = (kn - ko) - (qn - qo) - qo;  // p(r) = pbase + r
     int64_t pmax = pbase + re - 1;
     if (pmax < 0) return false;
-    int n_kt = (int)(pmax / kIdxKeyTile) + 1;
+    int n_kt = (int)((pmax >> a.shift) / kIdxKeyTile) + 1;
     kt_hi = n_kt < kt_lo + a.kt_per_split ? n_kt : kt_lo + a.kt_per_split;
     return kt_lo < kt_hi;
   };
@@ -140,7 +173,17 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     int kh;
     if (seq_range(b, rs, re, kh, pb)) n_jobs += kh - kt_lo;
   }
-  if (n_jobs == 0) return;  // uniform across the CTA
+  if (n_jobs == 0) {  // uniform across the CTA
+    if (CAND)
+      for (int c = threadIdx.x; c < 4 * BQ; c += blockDim.x)
+        if (r0 + c / 4 <= r_last) a.cand_cnt[(r0 - a.q_begin) * 4 + c] = 0;
+    return;
+  }
+  if (CAND) {
+    for (int c = threadIdx.x; c < BQ; c += blockDim.x)
+      s_thr[c] = r0 + c <= r_last ? __ldg(a.thr + (r0 + c - a.q_begin)) : INFINITY;
+    for (int c = threadIdx.x; c < 4 * BQ; c += blockDim.x) s_cnt[c / BQ][c % BQ] = 0;
+  }
 
   const int ncols = idx_tmem_cols(H, BQ);
   if (threadIdx.x == 0) {
@@ -178,7 +221,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         int64_t rs, re, pb;
         int kh;
         if (!seq_range(b, rs, re, kh, pb)) continue;
-        const int64_t kbase = __ldg(a.kv_offsets + b);
+        const int64_t kbase = idx_key_base(a, b);
         for (int kt = kt_lo; kt < kh; ++kt, ++i) {
           const int s = i % ST;
           if (!mbar_wait_bounded(smem_u32(&empty[s]), ((i / ST) & 1) ^ 1, a.status, &s_abort)) {
@@ -252,6 +295,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     float wsh[4] = {0.f, 0.f, 0.f, 0.f};
     if (a.w_row_stride == 0)
       for (int h = 0; h < H; ++h) wsh[h] = __ldg(a.w + h) * a.scale;
+    // candidate variant: this warp's score block (the chunk of rows c0 always goes to
+    // the warp with half = (c0 / 16) & 1, so each (quadrant, row) has one writer)
+    float* tile = tiles + (warp - 2) * (kIdxTileBytes / 4);
     int i = 0;
     bool ok = true;
     for (int b = b_first; b <= b_last && ok; ++b) {
@@ -268,9 +314,10 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         const int64_t j = (int64_t)kt * kIdxKeyTile + quad * 32 + lane;  // key position
         // columns c of this tile that belong to sequence b: rows rs..re-1
         const int c_lo = (int)(rs - r0), c_hi = (int)(re - r0);
-        for (int c0 = (c_lo / 16) * 16 + 16 * half; c0 < c_hi; c0 += 32) {
+        for (int c0 = 16 * half; c0 < c_hi; c0 += 32) {
+          if (c0 + 16 <= c_lo) continue;  // rows of an earlier sequence of the tile
           // skip chunks whose rows all precede this key tile (causal)
-          const int64_t p_chunk_max = pbase + r0 + (c0 + 15 < c_hi - 1 ? c0 + 15 : c_hi - 1);
+          const int64_t p_chunk_max = (pbase + r0 + (c0 + 15 < c_hi - 1 ? c0 + 15 : c_hi - 1)) >> a.shift;
           if (p_chunk_max < (int64_t)kt * kIdxKeyTile) continue;
           // all heads' TMEM loads in flight together, one wait
           uint32_t v[4][16];
@@ -301,10 +348,53 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           }
           // rows r0+c0 .. r0+c0+15; key j.  Interior chunk: every row belongs to this
           // sequence and sees the whole key tile, so no per-element predicate is needed.
+          const bool inside = c0 >= c_lo && c0 + 16 <= c_hi &&
+                              (int64_t)kt * kIdxKeyTile + (kIdxKeyTile - 1) <= ((pbase + r0 + c0) >> a.shift);
+          if (CAND) {
+            // keep the scores >= the row's threshold (float order; -0.0 == +0.0)
+#pragma unroll
+            for (int c = 0; c < 16; ++c) tile[c * kIdxTileStride + lane] = acc[c];
+            __syncwarp();
+            // lane l: row rr = l & 15 of the chunk, keys kh .. kh+15 of the warp's 32
+            const int rr = lane & 15, kh = (lane >> 4) * 16;
+            const float* trow = tile + rr * kIdxTileStride + kh;
+            const int cc = c0 + rr;
+            const float th = s_thr[cc];
+            // keys of this lane that the row may see: k < k_lim
+            int k_lim = 16;
+            if (!inside) {
+              const int64_t pr = (pbase + r0 + cc) >> a.shift;  // last key row the row sees
+              const int64_t first = (int64_t)kt * kIdxKeyTile + quad * 32 + kh;
+              const int64_t lim = pr - first + 1;
+              k_lim = (cc < c_lo || cc >= c_hi || lim <= 0) ? 0 : lim >= 16 ? 16 : (int)lim;
+            }
+            uint32_t m = 0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float4 x = *reinterpret_cast<const float4*>(trow + 4 * q);
+              m |= ((uint32_t)(x.x >= th) | ((uint32_t)(x.y >= th) << 1) | ((uint32_t)(x.z >= th) << 2) |
+                    ((uint32_t)(x.w >= th) << 3)) << (4 * q);
+            }
+            m &= k_lim >= 16 ? 0xFFFFu : ((1u << k_lim) - 1u);
+            const uint32_t n_lo = __shfl_sync(0xFFFFFFFFu, (uint32_t)__popc(m), lane & 15);
+            uint32_t base = lane < 16 ? s_cnt[quad][cc] : 0u;
+            base = __shfl_sync(0xFFFFFFFFu, base, lane & 15) + (lane >= 16 ? n_lo : 0u);
+            const uint32_t n_hi = __shfl_sync(0xFFFFFFFFu, (uint32_t)__popc(m), 16 + (lane & 15));
+            if (lane < 16) s_cnt[quad][cc] = base + n_lo + n_hi;
+            const int seg = a.cap >> 2;
+            float2* dst = a.cand + (r0 + cc - a.q_begin) * (int64_t)a.cap + quad * seg;
+            const int j0 = kt * kIdxKeyTile + quad * 32 + kh;
+            while (m) {
+              const int k = __ffs(m) - 1;
+              m &= m - 1;
+              if (base < (uint32_t)seg) dst[base] = make_float2(__int_as_float(j0 + k), trow[k]);
+              ++base;
+            }
+            __syncwarp();  // the block is read before the next chunk overwrites it
+            continue;
+          }
           float* dst = a.scores + (r0 + c0 - a.q_begin) * a.ld + j;
-          const bool interior = c0 >= c_lo && c0 + 16 <= c_hi &&
-                                (int64_t)kt * kIdxKeyTile + (kIdxKeyTile - 1) <= pbase + r0 + c0 &&
-                                (int64_t)kt * kIdxKeyTile + kIdxKeyTile <= a.ld;
+          const bool interior = inside && (int64_t)kt * kIdxKeyTile + kIdxKeyTile <= a.ld;
           if (interior) {
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
@@ -316,7 +406,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             for (int c = 0; c < 16; ++c) {
               const int cc = c0 + c;
               const int64_t r = r0 + cc;
-              if (cc >= c_lo && cc < c_hi && j <= pbase + r && j < a.ld) *dst = acc[c];
+              if (cc >= c_lo && cc < c_hi && j <= ((pbase + r) >> a.shift) && j < a.ld) *dst = acc[c];
               dst += a.ld;
             }
           }
@@ -333,6 +423,35 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, (uint32_t)ncols);
+  }
+  if (CAND)
+    for (int c = threadIdx.x; c < 4 * BQ; c += blockDim.x)
+      if (r0 + c / 4 <= r_last) a.cand_cnt[(r0 - a.q_begin) * 4 + c] = (int32_t)s_cnt[c % 4][c / 4];
+}
+
+// Sampled key tensor of the fused path: row (kv_offsets[b] >> shift) + b + m is row
+// kv_offsets[b] + (m << shift) of k_idx, for every sequence b and m < ceil(L_b / 2^shift);
+// rows between sequences are zero.  One warp per row, `vec` 16-byte words per row.
+__global__ void __launch_bounds__(256) idx_sample_keys_kernel(const int32_t* kv_offsets,
+                                                              int batch, int shift,
+                                                              const uint4* k, uint4* ks,
+                                                              int vec, int64_t rows) {
+  const int lane = lane_id();
+  const int64_t n_warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); g < rows;
+       g += n_warps) {
+    int lo = 0, hi = batch - 1;  // last sequence whose sample rows start at or before g
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (((int64_t)__ldg(kv_offsets + mid) >> shift) + mid <= g) lo = mid;
+      else hi = mid - 1;
+    }
+    const int64_t ko = __ldg(kv_offsets + lo), kn = __ldg(kv_offsets + lo + 1);
+    const int64_t m = g - ((ko >> shift) + lo);
+    const int64_t src = ko + (m << shift);
+    const bool real = m >= 0 && src < kn;
+    for (int v = lane; v < vec; v += 32)
+      ks[g * vec + v] = real ? __ldg(k + src * vec + v) : make_uint4(0u, 0u, 0u, 0u);
   }
 }
 

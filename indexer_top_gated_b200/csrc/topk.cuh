@@ -22,6 +22,19 @@
 // Bins are picked by a single warp (two-level warp scan), every histogram is zeroed once
 // up front and block scans cost one barrier, so a row needs few block-wide barriers; two
 // CTAs share an SM.  No sort and no global scratch.
+//
+// Fused indexer -> Top-K (no score matrix): the indexer first scores every 16th key
+// (samples), topk_thr_kernel turns each row's samples into a threshold estimate t, the
+// candidate indexer pass keeps only the (position, score) pairs with score >= t, and
+// topk_kernel<kTopkFused> selects among them: when the row has between K and `cap`
+// candidates they contain every score >= t, hence the whole Top-K with all of its ties,
+// and the selection is exact.  The candidates arrive in no particular order: the radix
+// select does not need one, and the selected positions are then marked in a bitmap over
+// the row (ties at the threshold in a second one, of which the lowest positions are
+// kept), which one ordered scan turns into the ascending index row.  A row whose
+// estimate missed (fewer than K candidates, or more than its slots) goes to a list that
+// topk_kernel<kTopkFallback> works through: it recomputes the row's scores on CUDA cores
+// into a scratch row and runs the full selection on it.
 #pragma once
 
 #include "common.cuh"
@@ -43,6 +56,20 @@ __host__ inline size_t topk_smem_bytes(int64_t /*max_kv_len*/) {
   return (size_t)kTopkSmemWords * sizeof(uint32_t);
 }
 
+// Fused selection: shared memory of one CTA = three histograms (4096 + 1024 + 1024 words),
+// the candidates' keys and positions (cap words each) and two position bitmaps of
+// ceil(max_n / 32) words each (rounded up to a multiple of 4).
+constexpr int kTopkFusedMaxN = 314496;
+constexpr int kTopkCandBatch = 8;  // candidate loads in flight per thread
+__host__ __device__ inline int topk_fused_bm_words(int64_t max_n) {
+  return (int)(((max_n + 31) / 32 + 3) / 4 * 4);
+}
+__host__ inline size_t topk_fused_smem_bytes(int cap, int64_t max_n) {
+  return (size_t)(6144 + 2 * cap + 2 * topk_fused_bm_words(max_n)) * 4;
+}
+
+enum TopkMode { kTopkScores = 0, kTopkFused = 1, kTopkFallback = 2 };
+
 struct TopkArgs {
   const int32_t* q_offsets;
   const int32_t* kv_offsets;
@@ -55,6 +82,38 @@ struct TopkArgs {
   int32_t* idx;
   int64_t ld_idx;
   int32_t* cnt;
+  // fused selection: candidate lists of the candidate indexer pass
+  const float2* cand;       // [q_count, cap]: 4 segments of cap/4 (position bits, score)
+  int cap;
+  const int32_t* cand_cnt;  // [q_count, 4] per segment
+  int32_t* fb_list;         // [1 + q_count]: count, then rows (within the launch) to redo
+  int bm_words;             // words of each position bitmap (topk_fused_bm_words)
+  // fallback: recompute a row's scores on CUDA cores (same formula as the indexer)
+  const void* q_idx;
+  const void* k_idx;
+  int idx_heads;
+  int idx_fp8;
+  const float* w;
+  int w_row_stride;
+  float idx_scale;
+  float* fb_scores;         // [gridDim.x, ld_fb]
+  int64_t ld_fb;
+};
+
+// Threshold estimate from sampled scores (fused path).
+struct TopkThrArgs {
+  const int32_t* q_offsets;
+  const int32_t* kv_offsets;
+  int batch;
+  int64_t q_begin;
+  int64_t q_count;
+  int K;
+  int cap;
+  int shift;          // sample m of a row is the score of position m << shift
+  const float* samp;  // [q_count, ld_s]
+  int64_t ld_s;
+  float* thr;         // [q_count]
+  int32_t* fb_list;   // its count is reset here
 };
 
 DSA_DEV uint32_t topk_key(float f) {
@@ -141,8 +200,112 @@ DSA_DEV void warp_select(const uint32_t* hist, uint32_t remaining, uint32_t* s_s
   }
 }
 
-__global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkArgs a) {
-  extern __shared__ uint32_t dyn[];
+// Shared state of a Top-K CTA besides the dynamic area.
+struct TopkShared {
+  uint32_t tot[64];
+  uint32_t sel[3];
+  uint32_t ncand;
+  uint32_t kmin, kmax;
+};
+
+// Radix select over `count` keys get(c) (strided over the block) with the zeroed histograms
+// h12 / h10a / h10b: finds the key threshold *tau of the want-th largest key and returns
+// how many keys equal to it are still needed (0 when the threshold bin is kept whole,
+// *whole = true, and every key >= *tau belongs to the selection).
+template <class Get>
+DSA_DEV uint32_t topk_select(uint32_t* h12, uint32_t* h10a, uint32_t* h10b, uint32_t want,
+                             Get&& get, uint32_t count, int levels, TopkShared& sh,
+                             uint32_t* tau, bool* whole) {
+  const int tid = threadIdx.x, warp = tid >> 5;
+  for (uint32_t c = tid; c < count; c += kTopkThreads) atomicAdd(&h12[get(c) >> 20], 1u);
+  __syncthreads();
+  if (warp == 0) warp_select<4096>(h12, want, sh.sel);
+  __syncthreads();
+  uint32_t t = sh.sel[0] << 20, need = sh.sel[1];
+  bool w = sh.sel[2] != 0;
+  if (!w) {
+    for (uint32_t c = tid; c < count; c += kTopkThreads) {
+      const uint32_t key = get(c);
+      if ((key & 0xFFF00000u) == t) atomicAdd(&h10a[(key >> 10) & 1023u], 1u);
+    }
+    __syncthreads();
+    if (warp == 0) warp_select<1024>(h10a, need, sh.sel);
+    __syncthreads();
+    t |= sh.sel[0] << 10;
+    need = sh.sel[1];
+    w = sh.sel[2] != 0;
+    if (!w && levels > 2) {
+      for (uint32_t c = tid; c < count; c += kTopkThreads) {
+        const uint32_t key = get(c);
+        if ((key & 0xFFFFFC00u) == t) atomicAdd(&h10b[key & 1023u], 1u);
+      }
+      __syncthreads();
+      if (warp == 0) warp_select<1024>(h10b, need, sh.sel);
+      __syncthreads();
+      t |= sh.sel[0];
+      need = sh.sel[1];
+      w = sh.sel[2] != 0;
+    }
+  }
+  *tau = t;
+  *whole = w;
+  return w ? 0u : need;
+}
+
+// Ordered output over C candidates fk / fp held in position order: the keys above tau (or
+// >= tau when ge) and the first ties_needed keys equal to tau, ascending by position.
+DSA_DEV void topk_emit_candidates(const uint32_t* fk, const uint32_t* fp, uint32_t C,
+                                  uint32_t tau, bool ge, uint32_t ties_needed, int32_t* out,
+                                  TopkShared& sh, int& bank) {
+  const int tid = threadIdx.x;
+  uint32_t run_def = 0, run_tie = 0;
+  for (uint32_t base = 0; base < C; base += 4 * kTopkThreads) {
+    const uint32_t c0 = base + 4 * tid;
+    uint32_t dflag = 0, tflag = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const bool valid = c0 + q < C;
+      const uint32_t key = valid ? fk[c0 + q] : 0u;
+      dflag |= (uint32_t)(valid && (ge ? key >= tau : key > tau)) << q;
+      tflag |= (uint32_t)(valid && !ge && key == tau) << q;
+    }
+    const uint32_t packed = (uint32_t)__popc(dflag) | ((uint32_t)__popc(tflag) << 16);
+    uint32_t total;
+    const uint32_t before = block_scan(packed, sh.tot, bank, total);
+    uint32_t d_before = run_def + (before & 0xFFFFu);
+    uint32_t t_before = run_tie + (before >> 16);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if ((dflag >> q) & 1u) {
+        out[d_before + (t_before < ties_needed ? t_before : ties_needed)] = (int32_t)fp[c0 + q];
+        ++d_before;
+      } else if ((tflag >> q) & 1u) {
+        if (t_before < ties_needed) out[d_before + t_before] = (int32_t)fp[c0 + q];
+        ++t_before;
+      }
+    }
+    run_def += total & 0xFFFFu;
+    run_tie += total >> 16;
+  }
+}
+
+template <bool NC>
+DSA_DEV float4 topk_ld4(const float* p) {
+  if (NC) return __ldg(reinterpret_cast<const float4*>(p));
+  return *reinterpret_cast<const float4*>(p);
+}
+template <bool NC>
+DSA_DEV float topk_ld1(const float* p) {
+  if (NC) return __ldg(p);
+  return *p;
+}
+
+// Top-K of one materialised score row row[0 .. nn), nn > K, into out[0 .. K).  NC: the row
+// was written by an earlier launch (read through the non-coherent cache); otherwise this
+// CTA wrote it, and it is read with coherent loads.
+template <bool NC>
+DSA_DEV void topk_scores_row(const TopkArgs& a, int nn, const float* row, int32_t* out,
+                             uint32_t* dyn, TopkShared& sh) {
   uint32_t* hA = dyn;            // 4096: sample, top 12 bits
   uint32_t* hB = hA + 4096;      // 1024: sample, next 10 bits
   uint32_t* hC = hB + 1024;      // 1024: sample, last 10 bits
@@ -152,34 +315,13 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkArgs a) {
   uint32_t* cand = dyn + kTopkHistWords;
   uint32_t* fk = cand;                 // fast path: candidate keys      [kTopkFastCap]
   uint32_t* fp = cand + kTopkFastCap;  // fast path: candidate positions [kTopkFastCap]
-  __shared__ uint32_t s_tot[64];
-  __shared__ uint32_t s_sel[3];
-  __shared__ uint32_t s_ncand;
-
   const int tid = threadIdx.x, lane = lane_id(), warp = tid >> 5;
-  const int64_t i = a.q_count - 1 - (int64_t)blockIdx.x;  // rows late in a sequence first
-  const int64_t r = a.q_begin + i;
-  const int b = seq_of_row(a.q_offsets, a.batch, r);
-  const int64_t qo = __ldg(a.q_offsets + b), qn = __ldg(a.q_offsets + b + 1);
-  const int64_t L = (int64_t)__ldg(a.kv_offsets + b + 1) - __ldg(a.kv_offsets + b);
-  const int64_t p = L - (qn - qo) + (r - qo);
-  const int64_t n = p + 1 > 0 ? p + 1 : 0;
   const int K = a.K;
-  int32_t* out = a.idx + i * a.ld_idx;
-
-  if (n <= K) {
-    for (int j = tid; j < K; j += kTopkThreads) out[j] = j < n ? j : -1;
-    if (a.cnt && tid == 0) a.cnt[i] = (int32_t)n;
-    return;
-  }
-
-  const float* row = a.scores + i * a.ld;
-  const int nn = (int)n;  // rows are shorter than 2^31
   int bank = 0;
   {
     // pull the whole row towards L2 now, so that its DRAM latency overlaps the threshold
     // estimate below and the candidate pass reads from L2 (the row is 16-byte aligned and
-    // its padded length round4(n) <= ld)
+    // its padded length round4(n) fits its allocation)
     const int64_t bytes = (((int64_t)nn + 3) & ~int64_t(3)) * 4;
     constexpr int64_t kPiece = 16384;
     for (int64_t off = (int64_t)tid * kPiece; off < bytes; off += (int64_t)kTopkThreads * kPiece)
@@ -189,59 +331,20 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkArgs a) {
   // four consecutive keys starting at j0 (a multiple of 4; 0 past the end)
   auto load4 = [&](int j0, uint32_t (&k4)[4]) {
     if (j0 + 3 < nn) {
-      const float4 f = __ldg(reinterpret_cast<const float4*>(row + j0));
+      const float4 f = topk_ld4<NC>(row + j0);
       k4[0] = topk_key(f.x);
       k4[1] = topk_key(f.y);
       k4[2] = topk_key(f.z);
       k4[3] = topk_key(f.w);
     } else {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) k4[q] = j0 + q < nn ? topk_key(__ldg(row + j0 + q)) : 0u;
+      for (int q = 0; q < 4; ++q) k4[q] = j0 + q < nn ? topk_key(topk_ld1<NC>(row + j0 + q)) : 0u;
     }
-  };
-  // radix select over keys held by the threads (`get(c)` for c in [0, count) strided by
-  // thread), in hist12 / hist10a / hist10b (zeroed): returns the threshold key in *tau and
-  // the count still needed from keys equal to it (0 when the threshold bin is kept whole).
-  auto select = [&](uint32_t* h12, uint32_t* h10a, uint32_t* h10b, uint32_t want, auto&& get,
-                    uint32_t count, int levels, uint32_t* tau, bool* whole) -> uint32_t {
-    for (uint32_t c = tid; c < count; c += kTopkThreads) atomicAdd(&h12[get(c) >> 20], 1u);
-    __syncthreads();
-    if (warp == 0) warp_select<4096>(h12, want, s_sel);
-    __syncthreads();
-    uint32_t t = s_sel[0] << 20, need = s_sel[1];
-    bool w = s_sel[2] != 0;
-    if (!w) {
-      for (uint32_t c = tid; c < count; c += kTopkThreads) {
-        const uint32_t key = get(c);
-        if ((key & 0xFFF00000u) == t) atomicAdd(&h10a[(key >> 10) & 1023u], 1u);
-      }
-      __syncthreads();
-      if (warp == 0) warp_select<1024>(h10a, need, s_sel);
-      __syncthreads();
-      t |= s_sel[0] << 10;
-      need = s_sel[1];
-      w = s_sel[2] != 0;
-      if (!w && levels > 2) {
-        for (uint32_t c = tid; c < count; c += kTopkThreads) {
-          const uint32_t key = get(c);
-          if ((key & 0xFFFFFC00u) == t) atomicAdd(&h10b[key & 1023u], 1u);
-        }
-        __syncthreads();
-        if (warp == 0) warp_select<1024>(h10b, need, s_sel);
-        __syncthreads();
-        t |= s_sel[0];
-        need = s_sel[1];
-        w = s_sel[2] != 0;
-      }
-    }
-    *tau = t;
-    *whole = w;
-    return w ? 0u : need;
   };
 
   // ---- zero every histogram once
   for (int t = tid; t < kTopkHistWords; t += kTopkThreads) dyn[t] = 0;
-  if (tid == 0) s_ncand = 0;
+  if (tid == 0) sh.ncand = 0;
   __syncthreads();
 
   // ================================================================ fast path
@@ -262,14 +365,14 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkArgs a) {
         *reinterpret_cast<uint4*>(fk + 4 * tid) = make_uint4(k4[0], k4[1], k4[2], k4[3]);
       }
     } else {
-      for (int j = tid; j < nn; j += kTopkThreads) fk[j] = topk_key(__ldg(row + j));
+      for (int j = tid; j < nn; j += kTopkThreads) fk[j] = topk_key(topk_ld1<NC>(row + j));
     }
     __syncthreads();
-    auto sget = [&](uint32_t c) -> uint32_t { return fk[c]; };
     uint32_t t_est;
     bool sw;
     // 22 bits of the estimate are plenty: every sample >= t_est counts towards m
-    select(hA, hB, hC, (uint32_t)m, sget, (uint32_t)S, 2, &t_est, &sw);
+    topk_select(hA, hB, hC, (uint32_t)m, [&](uint32_t c) { return fk[c]; }, (uint32_t)S, 2, sh,
+                &t_est, &sw);
     __syncthreads();  // samples read; the candidate pass may overwrite them
 
     // -- candidates: every key >= t_est, in position order.  The comparison is done on the
@@ -284,12 +387,12 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkArgs a) {
       for (int it = 0; it < kTopkBatch; ++it) {  // warp w owns positions cb + 1024 w .. + 1023
         const int j0 = cb + warp * 1024 + it * 128 + lane * 4;
         if (j0 + 3 < nn) {
-          xb[it] = __ldg(reinterpret_cast<const float4*>(row + j0));
+          xb[it] = topk_ld4<NC>(row + j0);
         } else {
-          xb[it].x = j0 < nn ? __ldg(row + j0) : -INFINITY;
-          xb[it].y = j0 + 1 < nn ? __ldg(row + j0 + 1) : -INFINITY;
-          xb[it].z = j0 + 2 < nn ? __ldg(row + j0 + 2) : -INFINITY;
-          xb[it].w = j0 + 3 < nn ? __ldg(row + j0 + 3) : -INFINITY;
+          xb[it].x = j0 < nn ? topk_ld1<NC>(row + j0) : -INFINITY;
+          xb[it].y = j0 + 1 < nn ? topk_ld1<NC>(row + j0 + 1) : -INFINITY;
+          xb[it].z = j0 + 2 < nn ? topk_ld1<NC>(row + j0 + 2) : -INFINITY;
+          xb[it].w = j0 + 3 < nn ? topk_ld1<NC>(row + j0 + 3) : -INFINITY;
         }
       }
       uint32_t fl = 0;                  // bit 4*it + q: score q of step it is kept
@@ -311,7 +414,7 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkArgs a) {
       for (int it = 0; it < 4; ++it)
         wtot += ((tot_lo >> (8 * it)) & 255u) + ((tot_hi >> (8 * it)) & 255u);
       uint32_t chunk_total;
-      const uint32_t wb = block_scan(lane == 31 ? wtot : 0u, s_tot, bank, chunk_total);
+      const uint32_t wb = block_scan(lane == 31 ? wtot : 0u, sh.tot, bank, chunk_total);
       // only lane 31 contributed, so lane 0's exclusive prefix is the count before warp w
       const uint32_t warp_base = __shfl_sync(0xFFFFFFFFu, wb, 0);
       if (run + chunk_total > (uint32_t)kTopkFastCap) {
@@ -342,43 +445,14 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkArgs a) {
     }
     __syncthreads();
     if (!overflow && run >= (uint32_t)K) {
-      // -- exact selection among the candidates
-      const uint32_t C = run;
-      auto cget = [&](uint32_t c) -> uint32_t { return fk[c]; };
+      // -- exact selection among the candidates, then ordered output over them (they are
+      // in position order)
       uint32_t tau;
       bool ge;
-      const uint32_t ties_needed = select(hD, hE, hF, (uint32_t)K, cget, C, 3, &tau, &ge);
-      // -- ordered output over the candidates (they are in position order)
-      uint32_t run_def = 0, run_tie = 0;
-      for (uint32_t base = 0; base < C; base += 4 * kTopkThreads) {
-        const uint32_t c0 = base + 4 * tid;
-        uint32_t dflag = 0, tflag = 0;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const bool valid = c0 + q < C;
-          const uint32_t key = valid ? fk[c0 + q] : 0u;
-          dflag |= (uint32_t)(valid && (ge ? key >= tau : key > tau)) << q;
-          tflag |= (uint32_t)(valid && !ge && key == tau) << q;
-        }
-        const uint32_t packed = (uint32_t)__popc(dflag) | ((uint32_t)__popc(tflag) << 16);
-        uint32_t total;
-        const uint32_t before = block_scan(packed, s_tot, bank, total);
-        uint32_t d_before = run_def + (before & 0xFFFFu);
-        uint32_t t_before = run_tie + (before >> 16);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          if ((dflag >> q) & 1u) {
-            out[d_before + (t_before < ties_needed ? t_before : ties_needed)] = (int32_t)fp[c0 + q];
-            ++d_before;
-          } else if ((tflag >> q) & 1u) {
-            if (t_before < ties_needed) out[d_before + t_before] = (int32_t)fp[c0 + q];
-            ++t_before;
-          }
-        }
-        run_def += total & 0xFFFFu;
-        run_tie += total >> 16;
-      }
-      if (tid == 0 && a.cnt) a.cnt[i] = K;
+      const uint32_t ties_needed =
+          topk_select(hD, hE, hF, (uint32_t)K, [&](uint32_t c) { return fk[c]; }, run, 3, sh,
+                      &tau, &ge);
+      topk_emit_candidates(fk, fp, run, tau, ge, ties_needed, out, sh, bank);
       return;  // uniform
     }
   }
@@ -400,12 +474,12 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkArgs a) {
     }
   }
   __syncthreads();
-  if (warp == 0) warp_select<4096>(hD, (uint32_t)K, s_sel);
+  if (warp == 0) warp_select<4096>(hD, (uint32_t)K, sh.sel);
   __syncthreads();
-  const uint32_t b12 = s_sel[0];
-  uint32_t remaining = s_sel[1];
+  const uint32_t b12 = sh.sel[0];
+  uint32_t remaining = sh.sel[1];
   uint32_t prefix = b12 << 20;
-  bool ge_mode = s_sel[2] != 0;
+  bool ge_mode = sh.sel[2] != 0;
   if (!ge_mode) {
     const uint32_t n_bin = hD[b12];
     const bool use_cand = n_bin <= (uint32_t)kTopkExactCap;
@@ -424,7 +498,7 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkArgs a) {
             const unsigned bal = __ballot_sync(0xFFFFFFFFu, mm);
             if (bal) {
               uint32_t slot = 0;
-              if (lane == 0) slot = atomicAdd(&s_ncand, (uint32_t)__popc(bal));
+              if (lane == 0) slot = atomicAdd(&sh.ncand, (uint32_t)__popc(bal));
               slot = __shfl_sync(0xFFFFFFFFu, slot, 0);
               if (mm) ck[slot + __popc(bal & ((1u << lane) - 1u))] = kb[it][q];
             }
@@ -458,11 +532,11 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkArgs a) {
         }
       }
       __syncthreads();
-      if (warp == 0) warp_select<1024>(h, remaining, s_sel);
+      if (warp == 0) warp_select<1024>(h, remaining, sh.sel);
       __syncthreads();
-      prefix |= s_sel[0] << shift;
-      remaining = s_sel[1];
-      ge_mode = s_sel[2] != 0;
+      prefix |= sh.sel[0] << shift;
+      remaining = sh.sel[1];
+      ge_mode = sh.sel[2] != 0;
     }
   }
 
@@ -489,7 +563,7 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkArgs a) {
       // packed counts: low 16 bits definite, high 16 bits ties (each <= 2048 per step)
       const uint32_t packed = (uint32_t)__popc(dflag) | ((uint32_t)__popc(tflag) << 16);
       uint32_t total;
-      const uint32_t before = block_scan(packed, s_tot, bank, total);
+      const uint32_t before = block_scan(packed, sh.tot, bank, total);
       uint32_t d_before = run_def + (before & 0xFFFFu);
       uint32_t t_before = run_tie + (before >> 16);
 #pragma unroll
@@ -506,7 +580,370 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkArgs a) {
       run_tie += total >> 16;
     }
   }
+}
+
+// Fused selection over the row's candidates: cnt[s] of them at the start of segment s
+// (seg slots each) of cl, C = sum >= K in all, nn <= kTopkFusedMaxN.  Their keys are
+// mapped onto the full 32-bit range by the order-preserving (key - kmin) << clz(kmax -
+// kmin), so that the radix digits spread although all candidates lie close together.
+DSA_DEV void topk_candidates_row(const TopkArgs& a, int nn, const float2* cl, int seg,
+                                 const uint32_t (&cnt)[4], uint32_t C, int32_t* out,
+                                 uint32_t* dyn, TopkShared& sh) {
+  uint32_t* hD = dyn;
+  uint32_t* hE = hD + 4096;
+  uint32_t* hF = hE + 1024;
+  uint32_t* sk = dyn + 6144;             // [cap] keys
+  uint32_t* sp = sk + a.cap;             // [cap] positions
+  uint32_t* bm = sp + a.cap;             // [bm_words] selected positions
+  uint32_t* bt = bm + a.bm_words;        // [bm_words] positions tied at the threshold
+  const int tid = threadIdx.x, lane = lane_id();
+  const int W = (nn + 31) >> 5;
+  int bank = 0;
+  const uint32_t e1 = cnt[0], e2 = e1 + cnt[1], e3 = e2 + cnt[2];
+  for (int t = tid; t < 6144; t += kTopkThreads) dyn[t] = 0;
+  for (int t = tid; t < W; t += kTopkThreads) {
+    bm[t] = 0;
+    bt[t] = 0;
+  }
+  if (tid == 0) {
+    sh.kmin = 0xFFFFFFFFu;
+    sh.kmax = 0u;
+  }
+  // load the candidates (several loads in flight per thread)
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  for (uint32_t c0 = 0; c0 < C; c0 += kTopkCandBatch * kTopkThreads) {
+    float2 e[kTopkCandBatch];
+#pragma unroll
+    for (int u = 0; u < kTopkCandBatch; ++u) {
+      const uint32_t c = c0 + u * kTopkThreads + tid;
+      const int s = (c >= e1) + (c >= e2) + (c >= e3);
+      const uint32_t sb = s == 0 ? 0u : s == 1 ? e1 : s == 2 ? e2 : e3;
+      e[u] = c < C ? __ldg(cl + (int64_t)s * seg + (c - sb)) : make_float2(0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kTopkCandBatch; ++u) {
+      const uint32_t c = c0 + u * kTopkThreads + tid;
+      if (c < C) {
+        const uint32_t key = topk_key(e[u].y);
+        lo = key < lo ? key : lo;
+        hi = key > hi ? key : hi;
+        sk[c] = key;
+        sp[c] = (uint32_t)__float_as_int(e[u].x);
+      }
+    }
+  }
+  lo = __reduce_min_sync(0xFFFFFFFFu, lo);
+  hi = __reduce_max_sync(0xFFFFFFFFu, hi);
+  __syncthreads();  // kmin / kmax initialised, histograms and bitmaps zeroed
+  if (lane == 0) {
+    atomicMin(&sh.kmin, lo);
+    atomicMax(&sh.kmax, hi);
+  }
+  __syncthreads();
+  {
+    const uint32_t kmin = sh.kmin, span = sh.kmax - sh.kmin;
+    const int z = span ? __clz(span) : 0;
+    for (uint32_t c = tid; c < C; c += kTopkThreads) sk[c] = (sk[c] - kmin) << z;
+  }
+  __syncthreads();
+  uint32_t tau;
+  bool ge;
+  const uint32_t ties_needed =
+      topk_select(hD, hE, hF, (uint32_t)a.K, [&](uint32_t c) { return sk[c]; }, C, 3, sh, &tau, &ge);
+  // mark the selected positions, and the ties at the threshold separately
+  for (uint32_t c = tid; c < C; c += kTopkThreads) {
+    const uint32_t key = sk[c], pos = sp[c];
+    if (ge ? key >= tau : key > tau) atomicOr(&bm[pos >> 5], 1u << (pos & 31u));
+    else if (!ge && key == tau) atomicOr(&bt[pos >> 5], 1u << (pos & 31u));
+  }
+  __syncthreads();
+  // each thread owns a run of bitmap words
+  const int wpt = (W + kTopkThreads - 1) / kTopkThreads;
+  const int w0 = tid * wpt, w1 = w0 + wpt < W ? w0 + wpt : W;
+  if (ties_needed) {  // uniform: keep the lowest ties_needed tied positions
+    uint32_t mine = 0;
+    for (int w = w0; w < w1; ++w) mine += __popc(bt[w]);
+    uint32_t total;
+    uint32_t before = block_scan(mine, sh.tot, bank, total);
+    for (int w = w0; w < w1 && before < ties_needed; ++w) {
+      uint32_t t = bt[w];
+      const uint32_t n = (uint32_t)__popc(t);
+      if (before + n > ties_needed) {  // keep only the lowest ties_needed - before bits
+        uint32_t keep = 0;
+        for (uint32_t q = before; q < ties_needed; ++q) {
+          keep |= t & (0u - t);
+          t &= t - 1;
+        }
+        t = keep;
+      }
+      bm[w] |= t;
+      before += n;
+    }
+    __syncthreads();
+  }
+  // ascending output: each thread writes the positions of its words
+  uint32_t mine = 0;
+  for (int w = w0; w < w1; ++w) mine += __popc(bm[w]);
+  uint32_t total;
+  uint32_t at = block_scan(mine, sh.tot, bank, total);
+  for (int w = w0; w < w1; ++w) {
+    uint32_t b = bm[w];
+    while (b) {
+      const int q = __ffs(b) - 1;
+      b &= b - 1;
+      out[at++] = w * 32 + q;
+    }
+  }
+}
+
+// e4m3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; no infinities) to float.
+DSA_DEV float topk_e4m3(uint32_t v) {
+  const uint32_t e = (v >> 3) & 15u, m = v & 7u;
+  const float x = e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : (float)m * 0.001953125f;
+  return (v & 0x80u) ? -x : x;
+}
+
+// Recompute the indexer scores of packed row r (sequence b, positions 0 .. nn-1) into
+// srow on CUDA cores, with the head weights applied as the indexer's epilogue does.
+DSA_DEV void topk_recompute_scores(const TopkArgs& a, int64_t r, int b, int nn, float* srow,
+                                   float* s_q, float* s_w) {
+  const int tid = threadIdx.x;
+  const int H = a.idx_heads;
+  const int D = 64 * H;
+  if (tid < D) {
+    if (a.idx_fp8) s_q[tid] = topk_e4m3(static_cast<const uint8_t*>(a.q_idx)[r * D + tid]);
+    else s_q[tid] = __uint_as_float((uint32_t)static_cast<const uint16_t*>(a.q_idx)[r * D + tid] << 16);
+  }
+  if (tid < H)
+    s_w[tid] = a.w_row_stride ? __ldg(a.w + r * a.w_row_stride + tid) : __ldg(a.w + tid) * a.idx_scale;
+  __syncthreads();
+  const int64_t ko = __ldg(a.kv_offsets + b);
+  for (int j = tid; j < nn; j += kTopkThreads) {
+    float acc = 0.f;
+    for (int h = 0; h < H; ++h) {
+      float dot = 0.f;
+      if (a.idx_fp8) {
+        const uint4* kr = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.k_idx) +
+                                                         (ko + j) * D + h * 64);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint4 u = __ldg(kr + v);
+          const uint32_t wds[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int q = 0; q < 16; ++q)
+            dot = fmaf(s_q[h * 64 + v * 16 + q], topk_e4m3((wds[q >> 2] >> (8 * (q & 3))) & 255u), dot);
+        }
+      } else {
+        const uint4* kr = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.k_idx) +
+                                                         (ko + j) * D + h * 64);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const uint4 u = __ldg(kr + v);
+          const uint32_t wds[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const uint32_t bits = (q & 1) ? (wds[q >> 1] & 0xFFFF0000u) : (wds[q >> 1] << 16);
+            dot = fmaf(s_q[h * 64 + v * 8 + q], __uint_as_float(bits), dot);
+          }
+        }
+      }
+      acc = a.w_row_stride ? fmaf(s_w[h], fmaxf(dot * a.idx_scale, 0.f), acc)
+                           : fmaf(s_w[h], fmaxf(dot, 0.f), acc);
+    }
+    srow[j] = acc;
+  }
+  __syncthreads();
+}
+
+DSA_DEV int64_t topk_row_len(const TopkArgs& a, int64_t r, int* b_out) {
+  const int b = seq_of_row(a.q_offsets, a.batch, r);
+  const int64_t qo = __ldg(a.q_offsets + b), qn = __ldg(a.q_offsets + b + 1);
+  const int64_t L = (int64_t)__ldg(a.kv_offsets + b + 1) - __ldg(a.kv_offsets + b);
+  const int64_t p = L - (qn - qo) + (r - qo);
+  *b_out = b;
+  return p + 1 > 0 ? p + 1 : 0;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkArgs a) {
+  extern __shared__ uint32_t dyn[];
+  __shared__ TopkShared sh;
+  const int tid = threadIdx.x;
+  const int K = a.K;
+
+  if (MODE == kTopkFallback) {
+    __shared__ float s_q[256];
+    __shared__ float s_w[4];
+    __shared__ int s_rows;
+    if (tid == 0) s_rows = a.fb_list[0];
+    __syncthreads();
+    const int rows = s_rows;
+    float* srow = a.fb_scores + (int64_t)blockIdx.x * a.ld_fb;
+    for (int k = blockIdx.x; k < rows; k += gridDim.x) {
+      const int64_t i = a.fb_list[1 + k];
+      const int64_t r = a.q_begin + i;
+      int b;
+      const int nn = (int)topk_row_len(a, r, &b);
+      __syncthreads();  // the previous row is finished with the shared areas
+      topk_recompute_scores(a, r, b, nn, srow, s_q, s_w);
+      topk_scores_row<false>(a, nn, srow, a.idx + i * a.ld_idx, dyn, sh);
+      if (tid == 0 && a.cnt) a.cnt[i] = K;
+    }
+    return;
+  }
+
+  const int64_t i = a.q_count - 1 - (int64_t)blockIdx.x;  // rows late in a sequence first
+  const int64_t r = a.q_begin + i;
+  int b;
+  const int64_t n = topk_row_len(a, r, &b);
+  int32_t* out = a.idx + i * a.ld_idx;
+  if (n <= K) {
+    for (int j = tid; j < K; j += kTopkThreads) out[j] = j < n ? j : -1;
+    if (a.cnt && tid == 0) a.cnt[i] = (int32_t)n;
+    return;
+  }
+  if (MODE == kTopkFused) {
+    const int seg = a.cap >> 2;
+    const int4 c4 = __ldg(reinterpret_cast<const int4*>(a.cand_cnt) + i);
+    const uint32_t cnt[4] = {(uint32_t)c4.x, (uint32_t)c4.y, (uint32_t)c4.z, (uint32_t)c4.w};
+    const uint32_t C = cnt[0] + cnt[1] + cnt[2] + cnt[3];
+    const bool over = cnt[0] > (uint32_t)seg || cnt[1] > (uint32_t)seg || cnt[2] > (uint32_t)seg ||
+                      cnt[3] > (uint32_t)seg;
+    if (over || C < (uint32_t)K) {
+      if (tid == 0) a.fb_list[1 + atomicAdd(a.fb_list, 1)] = (int32_t)i;
+      return;
+    }
+    topk_candidates_row(a, (int)n, a.cand + i * (int64_t)a.cap, seg, cnt, C, out, dyn, sh);
+  } else {
+    topk_scores_row<true>(a, (int)n, a.scores + i * a.ld, out, dyn, sh);
+  }
   if (tid == 0 && a.cnt) a.cnt[i] = K;
+}
+
+// One warp per row: a lower bound of the R-th largest of the row's S samples, R = S K / n
+// plus a margin of 5 sigma + 16, so that at least K scores of the row are >= it with
+// overwhelming probability while about R n / S are.  The sample keys are mapped onto the
+// full 32-bit range ((key - kmin) << clz(kmax - kmin), order-preserving), and two 8-bit
+// radix levels give the top 16 bits of the R-th largest; the estimate rounds it down.
+// Rows with n <= K need no candidates (+inf); rows with n <= cap keep every score (-inf).
+constexpr int kThrWarps = 4;
+constexpr int kThrStage = 2048;  // samples a warp stages in shared memory as keys
+__global__ void __launch_bounds__(32 * kThrWarps) topk_thr_kernel(TopkThrArgs a) {
+  __shared__ uint32_t hist[kThrWarps][256];
+  __shared__ __align__(16) uint32_t stage[kThrWarps][kThrStage];
+  const int warp = threadIdx.x >> 5, lane = lane_id();
+  if (blockIdx.x == 0 && threadIdx.x == 0) a.fb_list[0] = 0;
+  const int64_t i = (int64_t)blockIdx.x * kThrWarps + warp;
+  if (i >= a.q_count) return;  // warp-uniform; only warp-level syncs below
+  const int64_t r = a.q_begin + i;
+  const int b = seq_of_row(a.q_offsets, a.batch, r);
+  const int64_t qo = __ldg(a.q_offsets + b), qn = __ldg(a.q_offsets + b + 1);
+  const int64_t L = (int64_t)__ldg(a.kv_offsets + b + 1) - __ldg(a.kv_offsets + b);
+  const int64_t p = L - (qn - qo) + (r - qo);
+  const int64_t n = p + 1;
+  if (n <= a.K || n <= a.cap) {
+    if (lane == 0) a.thr[i] = n <= a.K ? INFINITY : -INFINITY;
+    return;
+  }
+  const int S = (int)(p >> a.shift) + 1;
+  const float e = (float)a.K * (float)S / (float)n;
+  int R = (int)ceilf(e + 5.f * sqrtf(e) + 16.f);
+  if (R > S) R = S;
+  uint32_t* h = hist[warp];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) h[lane * 8 + q] = 0;
+  const float* row = a.samp + i * a.ld_s;
+  // short sample rows (the usual case) are staged once as keys; longer ones are read
+  // from global memory on every pass, several loads in flight per lane
+  const bool staged = S <= kThrStage;
+  uint32_t* st = stage[warp];
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  auto for_keys = [&](auto&& f) {
+    if (staged) {
+      for (int m = lane; m < S; m += 32) f(st[m], true);
+    } else {
+      for (int m0 = 0; m0 < S; m0 += 8 * 32) {
+        float x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int m = m0 + u * 32 + lane;
+          x[u] = m < S ? __ldg(row + m) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) f(topk_key(x[u]), m0 + u * 32 + lane < S);
+      }
+    }
+  };
+  if (staged) {
+    const int S4 = (S + 3) & ~3;  // rows are 16-byte aligned and padded to ld_s >= S4
+    for (int m0 = 0; m0 < S4; m0 += 4 * 32 * 4) {
+      float4 f[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int m = m0 + (u * 32 + lane) * 4;
+        f[u] = m < S4 ? __ldg(reinterpret_cast<const float4*>(row + m)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int m = m0 + (u * 32 + lane) * 4;
+        if (m < S4)
+          *reinterpret_cast<uint4*>(st + m) =
+              make_uint4(topk_key(f[u].x), topk_key(f[u].y), topk_key(f[u].z), topk_key(f[u].w));
+      }
+    }
+    __syncwarp();
+  }
+  for_keys([&](uint32_t k, bool ok) {
+    if (ok) {
+      lo = k < lo ? k : lo;
+      hi = k > hi ? k : hi;
+    }
+  });
+  lo = __reduce_min_sync(0xFFFFFFFFu, lo);
+  hi = __reduce_max_sync(0xFFFFFFFFu, hi);
+  const int z = hi != lo ? __clz(hi - lo) : 0;
+  __syncwarp();
+  uint32_t prefix = 0, mask = 0, remaining = (uint32_t)R;
+  for (int level = 0; level < 2; ++level) {
+    const int sh = 24 - 8 * level;
+    for_keys([&](uint32_t k, bool ok) {
+      const uint32_t nk = (k - lo) << z;
+      if (ok && (nk & mask) == prefix) atomicAdd(&h[(nk >> sh) & 255u], 1u);
+    });
+    __syncwarp();
+    // lane l owns bins 255 - 8l - q, q = 0..7 (from the top)
+    uint32_t c[8], sum = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      c[q] = h[255 - 8 * lane - q];
+      sum += c[q];
+    }
+    const uint32_t incl = warp_incl_scan(sum);
+    const unsigned own = __ballot_sync(0xFFFFFFFFu, incl - sum < remaining && remaining <= incl);
+    const int o = __ffs(own) - 1;
+    uint32_t bin = 0, rem = 0;
+    if (lane == o) {
+      uint32_t above = incl - sum;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (above < remaining && remaining <= above + c[q]) {
+          bin = 255u - 8u * (uint32_t)lane - (uint32_t)q;
+          rem = remaining - above;
+        }
+        above += c[q];
+      }
+    }
+    bin = __shfl_sync(0xFFFFFFFFu, bin, o);
+    rem = __shfl_sync(0xFFFFFFFFu, rem, o);
+    prefix |= bin << sh;
+    mask |= 255u << sh;
+    remaining = rem;
+    __syncwarp();
+#pragma unroll
+    for (int q = 0; q < 8; ++q) h[lane * 8 + q] = 0;
+    __syncwarp();
+  }
+  if (lane == 0) a.thr[i] = topk_key_value(lo + (prefix >> z));
 }
 
 }  // namespace dsa

@@ -118,6 +118,40 @@ def test_workspace_size_is_host_only():
     import indexer_top_gated_b200 as dsa
     shape = dsa.LayerShape(top_k=2048)
     rg = dsa.Ragged(1, 0x1000, 0x2000, 32768, 32768, 32768, 32768)
-    mn, rec = dsa.dsa_workspace_size(shape, rg)
+    mn, rec = dsa.dsa_workspace_size(shape, rg, is_decode=True)
     assert mn == 32768 * 4 + 2048 * 4
     assert mn <= rec <= (1 << 30) + mn
+    # prefill of one long sequence: one fused pass over all rows, each row holding its
+    # candidate slots (8 bytes each, at least 2K of them) and its index row
+    mn_p, rec_p = dsa.dsa_workspace_size(shape, rg, is_decode=False)
+    assert mn_p == mn
+    assert rec_p >= 32768 * (2 * 2048 * 8 + 2048 * 4)
+    # a small prefill keeps its scores materialised (they fit in L2)
+    rg_small = dsa.Ragged(1, 0x1000, 0x2000, 4096, 4096, 4096, 4096)
+    assert dsa.dsa_workspace_size(dsa.LayerShape(top_k=256), rg_small)[1] <= 1 << 30
+
+
+def test_fused_index_topk_workspace_and_limits():
+    import indexer_top_gated_b200 as dsa
+    rg = dsa.Ragged(1, 0x1000, 0x2000, 32768, 32768, 32768, 32768)
+    mn, rec = dsa.dsa_index_topk_workspace_size(dsa.LayerShape(top_k=2048), rg, 32768)
+    assert 0 < mn < rec
+    # rec holds every row: per row at least the candidate slots
+    assert rec - mn >= 32767 * 2 * 2048 * 8
+    # K beyond the candidate slots, or rows beyond the position bitmap: unsupported
+    with pytest.raises(RuntimeError, match="unsupported"):
+        dsa.dsa_index_topk_workspace_size(dsa.LayerShape(top_k=6000), rg, 1)
+    long_rg = dsa.Ragged(1, 0x1000, 0x2000, 1, 400000, 1, 400000)
+    with pytest.raises(RuntimeError, match="unsupported"):
+        dsa.dsa_index_topk_workspace_size(dsa.LayerShape(top_k=64), long_rg, 1)
+    L = dsa.lib
+    P = dsa.LayerShape(top_k=2048).params()
+    A = 0x10000
+    args = lambda ws, nbytes, q0=0, qn=1, ld=2048: (  # noqa: E731
+        ctypes.byref(P), ctypes.byref(rg), A, A, A, q0, qn, A, ld, None, ws, nbytes, None)
+    assert L.dsa_index_topk(*args(A, mn)[:10], None, mn, None) == dsa.DSA_ERR_WORKSPACE
+    assert L.dsa_index_topk(*args(A + 16, mn)) == dsa.DSA_ERR_WORKSPACE
+    assert L.dsa_index_topk(*args(A, mn - 1)) == dsa.DSA_ERR_WORKSPACE
+    assert L.dsa_index_topk(*args(A, mn, ld=2047)) == dsa.DSA_ERR_INVALID_ARG
+    assert L.dsa_index_topk(*args(A, mn, q0=32768)) == dsa.DSA_ERR_INVALID_ARG
+    assert L.dsa_index_topk(*args(A, mn, qn=0)) == 0  # nothing to do
