@@ -86,6 +86,9 @@ def algorithmic(w):
         "idx_flops": 2 * Hi * Di * n_sum,
         "idx_bytes": 4 * n_sum + (tq + tk) * Hi * Di * e_idx,
         "topk_bytes": 4 * n_sum + 4 * K * tq,
+        # fused path: the selection never sees the score matrix; its floor is reading the
+        # K selected (position, score) pairs and writing the index rows
+        "topk_bytes_fused": 12 * sel_sum,
         "attn_bytes": sel_sum * Hkv * d * 2 * 2 + 3 * tq * Hq * d * 2 + 4 * K * tq,
         "attn_flops": 4 * sel_sum * Hq * d,
         "scores": n_sum,
@@ -488,13 +491,19 @@ def main():
     names = ["idx_scores", "topk_select", "sparse_attn_gated"]
     attn_gbs = alg["attn_bytes"] / (stage_ms[2] / 1e3) / 1e9 if stage_ms[2] > 0 else None
     idx_tflops = alg["idx_flops"] / (stage_ms[0] / 1e3) / 1e12 if stage_ms[0] > 0 else None
-    topk_gbs = alg["topk_bytes"] / (stage_ms[1] / 1e3) / 1e9 if stage_ms[1] > 0 else None
+    # steps 1-2 ran fused (sampled keys + samples + candidates | thresholds + selection +
+    # fallback rows: several launches per stage) or on a materialised score matrix
+    fused = stage_n[1] > 1
+    topk_alg = alg["topk_bytes_fused"] if fused else alg["topk_bytes"]
+    topk_gbs = topk_alg / (stage_ms[1] / 1e3) / 1e9 if stage_ms[1] > 0 else None
     stages = [
         {"kernel": names[0], "ms_per_step": stage_ms[0], "launches_per_step": stage_n[0],
          "bound": "tensor", "achieved": idx_tflops, "unit": "TFLOP/s",
          "peak": peaks["bf16_tflops_sustained"],
          "frac": idx_tflops / peaks["bf16_tflops_sustained"] if idx_tflops else None,
-         "score_write_gbs": 4 * alg["scores"] / (stage_ms[0] / 1e3) / 1e9 if stage_ms[0] else None},
+         "path": "fused: sampled threshold, candidates only" if fused else "materialised scores",
+         "score_write_gbs": (None if fused else
+                             4 * alg["scores"] / (stage_ms[0] / 1e3) / 1e9 if stage_ms[0] else None)},
         {"kernel": names[1], "ms_per_step": stage_ms[1], "launches_per_step": stage_n[1],
          "bound": "hbm", "achieved": topk_gbs, "unit": "GB/s", "peak": peaks["hbm_gbs"],
          "frac": topk_gbs / peaks["hbm_gbs"] if topk_gbs else None},
@@ -511,7 +520,7 @@ def main():
     roof = {"kernel": names[dom], "bound": stages[dom]["bound"], "achieved": stages[dom]["achieved"],
             "peak": stages[dom]["peak"], "unit": stages[dom]["unit"], "frac": stages[dom]["frac"],
             "traffic": traffic, "peak_source": f"{peak_src} ({'hbm_gbs' if dom else 'bf16_tflops_sustained'})",
-            "algorithmic_per_launch": (alg["attn_bytes"] if dom == 2 else alg["topk_bytes"] if dom == 1
+            "algorithmic_per_launch": (alg["attn_bytes"] if dom == 2 else topk_alg if dom == 1
                                        else alg["idx_flops"]) / stage_n[dom]}
     cpu = None
     if world == 1 and not args.no_cpu_baseline:

@@ -111,7 +111,7 @@ dsa_status device_setup(DeviceState** out) {
     e = e ? e : allow_smem(idx_scores_kernel<64, true, true>, cand_max);
     e = e ? e : allow_smem(idx_scores_kernel<16, true, true>, cand_max);
     e = e ? e : allow_smem(topk_kernel<kTopkScores>, topk_smem_bytes(0));
-    e = e ? e : allow_smem(topk_kernel<kTopkFused>, topk_fused_smem_bytes(kTopkFastCap, kTopkFusedMaxN));
+    e = e ? e : allow_smem(topk_fused_kernel, topk_fused_smem_bytes(kTopkFastCap, kTopkFusedMaxN));
     e = e ? e : allow_smem(topk_kernel<kTopkFallback>, topk_smem_bytes(0));
     e = e ? e : allow_smem(sparse_attn_kernel<1, 1>, attn_smem_bytes());
     e = e ? e : allow_smem(sparse_attn_kernel<2, 1>, attn_smem_bytes());
@@ -472,8 +472,8 @@ dsa_status fused_pass(const DeviceState& dev, const dsa_params* P, const dsa_rag
   a.bm_words = topk_fused_bm_words(std::max(R->max_kv_len, 1));
   {  // (4) exact selection over the candidates
     StageScope scope(1, stream);
-    topk_kernel<kTopkFused><<<(unsigned)q_count, kTopkThreads,
-                              topk_fused_smem_bytes(g.cap, R->max_kv_len), stream>>>(a);
+    topk_fused_kernel<<<(unsigned)q_count, kTopkThreads,
+                        topk_fused_smem_bytes(g.cap, R->max_kv_len), stream>>>(a);
     ++t_launches;
     DSA_TRY(launch_status("topk_kernel (fused selection)"));
   }

@@ -10,9 +10,11 @@
 //    positions of one query row: every score store is a coalesced 128-byte line.
 //  - Warp 0 issues TMA loads (128-byte swizzled, one box per indexer head) into a
 //    3-stage ring; warp 1 issues tcgen05.mma (one per head and 16-wide K step) into one
-//    of two TMEM accumulator buffers; warps 2-9 drain TMEM (tcgen05.ld; two warps per
-//    lane quadrant, alternate 16-column chunks), apply ReLU, the head weights and the
-//    head sum, mask causally and store fp32 scores.
+//    of two TMEM accumulator buffers; warps 2-17 drain TMEM (tcgen05.ld; four warps per
+//    lane quadrant, each taking every fourth 16-column chunk), apply ReLU, the head
+//    weights and the head sum, mask causally and store fp32 scores.  Sixteen draining
+//    warps (at most 96 registers each) hide the TMEM-load and store latencies better
+//    than fewer, larger ones.
 //  - Tiles may straddle sequences of a ragged batch: the CTA runs one pass per
 //    sequence it touches and masks the other rows.  Tiles are scheduled largest
 //    first (the last rows of a sequence see the most keys).
@@ -72,7 +74,8 @@ constexpr int kIdxCandStages = 2;
 constexpr int kIdxTileStride = 36;  // floats per row of a warp's score block (no bank conflicts)
 constexpr int kIdxTileBytes = 16 * kIdxTileStride * 4;
 constexpr int kIdxKeyTile = 128;
-constexpr int kIdxEpiWarps = 8;  // two warps per TMEM lane quadrant
+constexpr int kIdxEpiWarps = 16;  // four warps per TMEM lane quadrant
+constexpr int kIdxSubs = kIdxEpiWarps / 4;
 constexpr int kIdxThreads = 64 + 32 * kIdxEpiWarps;
 
 template <bool FP8>
@@ -288,7 +291,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue (warps 2-9)
     const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
-    const int half = (warp - 2) >> 2;  // the two warps of a quadrant take alternate chunks
+    const int sub = (warp - 2) >> 2;  // the warps of a quadrant take every kIdxSubs-th chunk
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     // shared head weights with the (positive) dequantisation scale folded in:
     // w * max(0, c * x) = (w * c) * max(0, x) for c > 0
@@ -296,7 +299,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     if (a.w_row_stride == 0)
       for (int h = 0; h < H; ++h) wsh[h] = __ldg(a.w + h) * a.scale;
     // candidate variant: this warp's score block (the chunk of rows c0 always goes to
-    // the warp with half = (c0 / 16) & 1, so each (quadrant, row) has one writer)
+    // the warp with sub = (c0 / 16) % kIdxSubs, so each (quadrant, row) has one writer)
     float* tile = tiles + (warp - 2) * (kIdxTileBytes / 4);
     int i = 0;
     bool ok = true;
@@ -314,35 +317,42 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         const int64_t j = (int64_t)kt * kIdxKeyTile + quad * 32 + lane;  // key position
         // columns c of this tile that belong to sequence b: rows rs..re-1
         const int c_lo = (int)(rs - r0), c_hi = (int)(re - r0);
-        for (int c0 = 16 * half; c0 < c_hi; c0 += 32) {
+        for (int c0 = 16 * sub; c0 < c_hi; c0 += 16 * kIdxSubs) {
           if (c0 + 16 <= c_lo) continue;  // rows of an earlier sequence of the tile
           // skip chunks whose rows all precede this key tile (causal)
           const int64_t p_chunk_max = (pbase + r0 + (c0 + 15 < c_hi - 1 ? c0 + 15 : c_hi - 1)) >> a.shift;
           if (p_chunk_max < (int64_t)kt * kIdxKeyTile) continue;
-          // all heads' TMEM loads in flight together, one wait
-          uint32_t v[4][16];
-#pragma unroll
-          for (int h = 0; h < 4; ++h)
-            if (h < H) tmem_ld16_async(tmem + lane_base + (uint32_t)(buf * H * BQ + h * BQ + c0), v[h]);
-          tmem_wait_ld();
+          // heads in pairs: two TMEM loads in flight, then their ReLU-weighted sum
+          // (the accumulation order over heads is 0, 1, 2, 3 as before)
           float acc[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) acc[c] = 0.f;
 #pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            if (h >= H) break;
-            reg_fence(v[h]);
-            if (a.w_row_stride == 0) {
+          for (int hp = 0; hp < 4; hp += 2) {
+            if (hp >= H) break;
+            uint32_t v[2][16];
 #pragma unroll
-              for (int c = 0; c < 16; ++c)
-                acc[c] = fmaf(wsh[h], fmaxf(__uint_as_float(v[h][c]), 0.f), acc[c]);
-            } else {
+            for (int q = 0; q < 2; ++q)
+              if (hp + q < H)
+                tmem_ld16_async(tmem + lane_base + (uint32_t)(buf * H * BQ + (hp + q) * BQ + c0), v[q]);
+            tmem_wait_ld();
 #pragma unroll
-              for (int c = 0; c < 16; ++c) {
-                int64_t r = r0 + c0 + c;
-                if (r > r_last) r = r_last;
-                const float wv = __ldg(a.w + r * a.w_row_stride + h);
-                acc[c] = fmaf(wv, fmaxf(__uint_as_float(v[h][c]) * a.scale, 0.f), acc[c]);
+            for (int q = 0; q < 2; ++q) {
+              const int h = hp + q;
+              if (h >= H) break;
+              reg_fence(v[q]);
+              if (a.w_row_stride == 0) {
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                  acc[c] = fmaf(wsh[h], fmaxf(__uint_as_float(v[q][c]), 0.f), acc[c]);
+              } else {
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                  int64_t r = r0 + c0 + c;
+                  if (r > r_last) r = r_last;
+                  const float wv = __ldg(a.w + r * a.w_row_stride + h);
+                  acc[c] = fmaf(wv, fmaxf(__uint_as_float(v[q][c]) * a.scale, 0.f), acc[c]);
+                }
               }
             }
           }

@@ -26,15 +26,16 @@
 // Fused indexer -> Top-K (no score matrix): the indexer first scores every 16th key
 // (samples), topk_thr_kernel turns each row's samples into a threshold estimate t, the
 // candidate indexer pass keeps only the (position, score) pairs with score >= t, and
-// topk_kernel<kTopkFused> selects among them: when the row has between K and `cap`
-// candidates they contain every score >= t, hence the whole Top-K with all of its ties,
-// and the selection is exact.  The candidates arrive in no particular order: the radix
-// select does not need one, and the selected positions are then marked in a bitmap over
-// the row (ties at the threshold in a second one, of which the lowest positions are
-// kept), which one ordered scan turns into the ascending index row.  A row whose
-// estimate missed (fewer than K candidates, or more than its slots) goes to a list that
-// topk_kernel<kTopkFallback> works through: it recomputes the row's scores on CUDA cores
-// into a scratch row and runs the full selection on it.
+// topk_fused_kernel selects among them: when the row has between K and `cap` candidates
+// they contain every score >= t, hence the whole Top-K with all of its ties, and the
+// selection is exact.  The candidates arrive in no particular order, which one radix
+// level (12 bits of the keys, spread over the candidates' range) does not need; the few
+// candidates in the threshold bin are then ranked exactly (score descending, position
+// ascending), the selected positions are marked in a bitmap over the row, and one ordered
+// scan turns it into the ascending index row.  A row whose estimate missed (fewer than
+// K candidates, or more than its slots) or whose threshold bin is too crowded goes to a
+// list that topk_kernel<kTopkFallback> works through: it recomputes the row's scores on
+// CUDA cores into a scratch row and runs the full selection on it.
 #pragma once
 
 #include "common.cuh"
@@ -56,19 +57,20 @@ __host__ inline size_t topk_smem_bytes(int64_t /*max_kv_len*/) {
   return (size_t)kTopkSmemWords * sizeof(uint32_t);
 }
 
-// Fused selection: shared memory of one CTA = three histograms (4096 + 1024 + 1024 words),
-// the candidates' keys and positions (cap words each) and two position bitmaps of
-// ceil(max_n / 32) words each (rounded up to a multiple of 4).
+// Fused selection: shared memory of one CTA = a 4096-bin histogram, the candidates' keys
+// and positions (cap words each), a position bitmap of ceil(max_n / 32) words (rounded up
+// to a multiple of 4) and the threshold bin's keys and positions (kTopkBinMax each).
 constexpr int kTopkFusedMaxN = 314496;
-constexpr int kTopkCandBatch = 8;  // candidate loads in flight per thread
+constexpr int kTopkCandBatch = 8;    // candidate loads in flight per thread
+constexpr int kTopkBinMax = 512;     // threshold-bin candidates ranked directly
 __host__ __device__ inline int topk_fused_bm_words(int64_t max_n) {
   return (int)(((max_n + 31) / 32 + 3) / 4 * 4);
 }
 __host__ inline size_t topk_fused_smem_bytes(int cap, int64_t max_n) {
-  return (size_t)(6144 + 2 * cap + 2 * topk_fused_bm_words(max_n)) * 4;
+  return (size_t)(4096 + 2 * cap + topk_fused_bm_words(max_n) + 2 * kTopkBinMax) * 4;
 }
 
-enum TopkMode { kTopkScores = 0, kTopkFused = 1, kTopkFallback = 2 };
+enum TopkMode { kTopkScores = 0, kTopkFallback = 2 };
 
 struct TopkArgs {
   const int32_t* q_offsets;
@@ -163,12 +165,16 @@ DSA_DEV void warp_select(const uint32_t* hist, uint32_t remaining, uint32_t* s_s
   constexpr int PER = NB / 32;   // bins per lane in the first level
   constexpr int SUB = PER / 32;  // bins per lane in the second level
   const int lane = lane_id();
-  // level 1: lane l owns the l-th block of PER bins counted from the top
+  // level 1: lane l owns the l-th block of PER bins counted from the top.  The blocks
+  // are PER words apart (the same banks), so each lane walks its block in a rotated
+  // order: at step q lane l reads quad (q + l) mod (PER / 4), and a warp's 16-byte reads
+  // spread over all banks.
   const int hi1 = NB - 1 - lane * PER;
   uint32_t sum = 0;
 #pragma unroll
-  for (int q = 0; q < PER; q += 4) {
-    const uint4 u = *reinterpret_cast<const uint4*>(hist + hi1 - PER + 1 + q);
+  for (int q = 0; q < PER / 4; ++q) {
+    const int qq = (q + lane) & (PER / 4 - 1);
+    const uint4 u = *reinterpret_cast<const uint4*>(hist + hi1 - PER + 1 + 4 * qq);
     sum += u.x + u.y + u.z + u.w;
   }
   uint32_t incl = warp_incl_scan(sum);
@@ -583,31 +589,29 @@ DSA_DEV void topk_scores_row(const TopkArgs& a, int nn, const float* row, int32_
 }
 
 // Fused selection over the row's candidates: cnt[s] of them at the start of segment s
-// (seg slots each) of cl, C = sum >= K in all, nn <= kTopkFusedMaxN.  Their keys are
-// mapped onto the full 32-bit range by the order-preserving (key - kmin) << clz(kmax -
-// kmin), so that the radix digits spread although all candidates lie close together.
-DSA_DEV void topk_candidates_row(const TopkArgs& a, int nn, const float2* cl, int seg,
+// (seg slots each) of cl, C = sum >= K in all, nn <= kTopkFusedMaxN.  Keys are mapped onto
+// the full 32-bit range by the order-preserving (key - kmin) << clz(kmax - kmin), so that
+// the 12-bit digit spreads although all candidates lie close together.  Returns false
+// (nothing written) when the threshold bin holds more than kTopkBinMax candidates.
+DSA_DEV bool topk_candidates_row(const TopkArgs& a, int nn, const float2* cl, int seg,
                                  const uint32_t (&cnt)[4], uint32_t C, int32_t* out,
                                  uint32_t* dyn, TopkShared& sh) {
-  uint32_t* hD = dyn;
-  uint32_t* hE = hD + 4096;
-  uint32_t* hF = hE + 1024;
-  uint32_t* sk = dyn + 6144;             // [cap] keys
+  uint32_t* h = dyn;                     // [4096]
+  uint32_t* sk = dyn + 4096;             // [cap] keys
   uint32_t* sp = sk + a.cap;             // [cap] positions
   uint32_t* bm = sp + a.cap;             // [bm_words] selected positions
-  uint32_t* bt = bm + a.bm_words;        // [bm_words] positions tied at the threshold
-  const int tid = threadIdx.x, lane = lane_id();
+  uint32_t* bk = bm + a.bm_words;        // [kTopkBinMax] threshold-bin keys
+  uint32_t* bp = bk + kTopkBinMax;       // [kTopkBinMax] threshold-bin positions
+  const int tid = threadIdx.x, lane = lane_id(), warp = tid >> 5;
   const int W = (nn + 31) >> 5;
   int bank = 0;
   const uint32_t e1 = cnt[0], e2 = e1 + cnt[1], e3 = e2 + cnt[2];
-  for (int t = tid; t < 6144; t += kTopkThreads) dyn[t] = 0;
-  for (int t = tid; t < W; t += kTopkThreads) {
-    bm[t] = 0;
-    bt[t] = 0;
-  }
+  for (int t = tid; t < 4096; t += kTopkThreads) h[t] = 0;
+  for (int t = tid; t < W; t += kTopkThreads) bm[t] = 0;
   if (tid == 0) {
     sh.kmin = 0xFFFFFFFFu;
     sh.kmax = 0u;
+    sh.ncand = 0;
   }
   // load the candidates (several loads in flight per thread)
   uint32_t lo = 0xFFFFFFFFu, hi = 0u;
@@ -634,7 +638,7 @@ DSA_DEV void topk_candidates_row(const TopkArgs& a, int nn, const float2* cl, in
   }
   lo = __reduce_min_sync(0xFFFFFFFFu, lo);
   hi = __reduce_max_sync(0xFFFFFFFFu, hi);
-  __syncthreads();  // kmin / kmax initialised, histograms and bitmaps zeroed
+  __syncthreads();  // kmin / kmax initialised, histogram and bitmap zeroed
   if (lane == 0) {
     atomicMin(&sh.kmin, lo);
     atomicMax(&sh.kmax, hi);
@@ -643,57 +647,83 @@ DSA_DEV void topk_candidates_row(const TopkArgs& a, int nn, const float2* cl, in
   {
     const uint32_t kmin = sh.kmin, span = sh.kmax - sh.kmin;
     const int z = span ? __clz(span) : 0;
-    for (uint32_t c = tid; c < C; c += kTopkThreads) sk[c] = (sk[c] - kmin) << z;
+    for (uint32_t c0 = 0; c0 < C; c0 += kTopkCandBatch * kTopkThreads) {
+      uint32_t kk[kTopkCandBatch];
+#pragma unroll
+      for (int u = 0; u < kTopkCandBatch; ++u) {
+        const uint32_t c = c0 + u * kTopkThreads + tid;
+        kk[u] = c < C ? sk[c] : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < kTopkCandBatch; ++u) {
+        const uint32_t c = c0 + u * kTopkThreads + tid;
+        if (c < C) {
+          const uint32_t nk = (kk[u] - kmin) << z;
+          sk[c] = nk;
+          atomicAdd(&h[nk >> 20], 1u);
+        }
+      }
+    }
   }
   __syncthreads();
-  uint32_t tau;
-  bool ge;
-  const uint32_t ties_needed =
-      topk_select(hD, hE, hF, (uint32_t)a.K, [&](uint32_t c) { return sk[c]; }, C, 3, sh, &tau, &ge);
-  // mark the selected positions, and the ties at the threshold separately
-  for (uint32_t c = tid; c < C; c += kTopkThreads) {
-    const uint32_t key = sk[c], pos = sp[c];
-    if (ge ? key >= tau : key > tau) atomicOr(&bm[pos >> 5], 1u << (pos & 31u));
-    else if (!ge && key == tau) atomicOr(&bt[pos >> 5], 1u << (pos & 31u));
+  if (warp == 0) warp_select<4096>(h, (uint32_t)a.K, sh.sel);
+  __syncthreads();
+  const uint32_t b = sh.sel[0], need = sh.sel[1];
+  const bool whole = sh.sel[2] != 0;
+  const uint32_t n_bin = h[b];
+  if (!whole && n_bin > (uint32_t)kTopkBinMax) return false;  // uniform
+  // keys in higher bins (or the whole threshold bin) are selected; the threshold bin's
+  // keys are set aside for ranking
+  for (uint32_t c0 = 0; c0 < C; c0 += kTopkCandBatch * kTopkThreads) {
+    uint32_t kk[kTopkCandBatch], pp[kTopkCandBatch];
+#pragma unroll
+    for (int u = 0; u < kTopkCandBatch; ++u) {
+      const uint32_t c = c0 + u * kTopkThreads + tid;
+      kk[u] = c < C ? sk[c] : 0u;
+      pp[u] = c < C ? sp[c] : 0xFFFFFFFFu;
+    }
+#pragma unroll
+    for (int u = 0; u < kTopkCandBatch; ++u) {
+      if (pp[u] == 0xFFFFFFFFu) continue;
+      const uint32_t bin = kk[u] >> 20, pos = pp[u];
+      if (bin > b || (whole && bin == b)) {
+        atomicOr(&bm[pos >> 5], 1u << (pos & 31u));
+      } else if (bin == b) {
+        const uint32_t slot = atomicAdd(&sh.ncand, 1u);
+        bk[slot] = kk[u];
+        bp[slot] = pos;
+      }
+    }
   }
   __syncthreads();
-  // each thread owns a run of bitmap words
+  if (!whole && tid < (int)n_bin) {
+    // rank among the bin: larger keys first, then lower positions
+    const uint32_t k0 = bk[tid], p0 = bp[tid];
+    uint32_t rank = 0;
+#pragma unroll 4
+    for (uint32_t x = 0; x < n_bin; ++x) {
+      const uint32_t k1 = bk[x];
+      rank += (k1 > k0) || (k1 == k0 && bp[x] < p0);
+    }
+    if (rank < need) atomicOr(&bm[p0 >> 5], 1u << (p0 & 31u));
+  }
+  __syncthreads();
+  // ascending output: each thread writes the positions of its run of bitmap words
   const int wpt = (W + kTopkThreads - 1) / kTopkThreads;
   const int w0 = tid * wpt, w1 = w0 + wpt < W ? w0 + wpt : W;
-  if (ties_needed) {  // uniform: keep the lowest ties_needed tied positions
-    uint32_t mine = 0;
-    for (int w = w0; w < w1; ++w) mine += __popc(bt[w]);
-    uint32_t total;
-    uint32_t before = block_scan(mine, sh.tot, bank, total);
-    for (int w = w0; w < w1 && before < ties_needed; ++w) {
-      uint32_t t = bt[w];
-      const uint32_t n = (uint32_t)__popc(t);
-      if (before + n > ties_needed) {  // keep only the lowest ties_needed - before bits
-        uint32_t keep = 0;
-        for (uint32_t q = before; q < ties_needed; ++q) {
-          keep |= t & (0u - t);
-          t &= t - 1;
-        }
-        t = keep;
-      }
-      bm[w] |= t;
-      before += n;
-    }
-    __syncthreads();
-  }
-  // ascending output: each thread writes the positions of its words
   uint32_t mine = 0;
   for (int w = w0; w < w1; ++w) mine += __popc(bm[w]);
   uint32_t total;
   uint32_t at = block_scan(mine, sh.tot, bank, total);
   for (int w = w0; w < w1; ++w) {
-    uint32_t b = bm[w];
-    while (b) {
-      const int q = __ffs(b) - 1;
-      b &= b - 1;
+    uint32_t bits = bm[w];
+    while (bits) {
+      const int q = __ffs(bits) - 1;
+      bits &= bits - 1;
       out[at++] = w * 32 + q;
     }
   }
+  return true;
 }
 
 // e4m3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; no infinities) to float.
@@ -802,20 +832,36 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkArgs a) {
     if (a.cnt && tid == 0) a.cnt[i] = (int32_t)n;
     return;
   }
-  if (MODE == kTopkFused) {
-    const int seg = a.cap >> 2;
-    const int4 c4 = __ldg(reinterpret_cast<const int4*>(a.cand_cnt) + i);
-    const uint32_t cnt[4] = {(uint32_t)c4.x, (uint32_t)c4.y, (uint32_t)c4.z, (uint32_t)c4.w};
-    const uint32_t C = cnt[0] + cnt[1] + cnt[2] + cnt[3];
-    const bool over = cnt[0] > (uint32_t)seg || cnt[1] > (uint32_t)seg || cnt[2] > (uint32_t)seg ||
-                      cnt[3] > (uint32_t)seg;
-    if (over || C < (uint32_t)K) {
-      if (tid == 0) a.fb_list[1 + atomicAdd(a.fb_list, 1)] = (int32_t)i;
-      return;
-    }
-    topk_candidates_row(a, (int)n, a.cand + i * (int64_t)a.cap, seg, cnt, C, out, dyn, sh);
-  } else {
-    topk_scores_row<true>(a, (int)n, a.scores + i * a.ld, out, dyn, sh);
+  topk_scores_row<true>(a, (int)n, a.scores + i * a.ld, out, dyn, sh);
+  if (tid == 0 && a.cnt) a.cnt[i] = K;
+}
+
+// Fused selection, one CTA per row (three CTAs share an SM).
+__global__ void __launch_bounds__(kTopkThreads, 3) topk_fused_kernel(TopkArgs a) {
+  extern __shared__ uint32_t dyn[];
+  __shared__ TopkShared sh;
+  const int tid = threadIdx.x;
+  const int K = a.K;
+  const int64_t i = a.q_count - 1 - (int64_t)blockIdx.x;
+  const int64_t r = a.q_begin + i;
+  int b;
+  const int64_t n = topk_row_len(a, r, &b);
+  int32_t* out = a.idx + i * a.ld_idx;
+  if (n <= K) {
+    for (int j = tid; j < K; j += kTopkThreads) out[j] = j < n ? j : -1;
+    if (a.cnt && tid == 0) a.cnt[i] = (int32_t)n;
+    return;
+  }
+  const int seg = a.cap >> 2;
+  const int4 c4 = __ldg(reinterpret_cast<const int4*>(a.cand_cnt) + i);
+  const uint32_t cnt[4] = {(uint32_t)c4.x, (uint32_t)c4.y, (uint32_t)c4.z, (uint32_t)c4.w};
+  const uint32_t C = cnt[0] + cnt[1] + cnt[2] + cnt[3];
+  const bool over = cnt[0] > (uint32_t)seg || cnt[1] > (uint32_t)seg || cnt[2] > (uint32_t)seg ||
+                    cnt[3] > (uint32_t)seg;
+  if (over || C < (uint32_t)K ||
+      !topk_candidates_row(a, (int)n, a.cand + i * (int64_t)a.cap, seg, cnt, C, out, dyn, sh)) {
+    if (tid == 0) a.fb_list[1 + atomicAdd(a.fb_list, 1)] = (int32_t)i;
+    return;
   }
   if (tid == 0 && a.cnt) a.cnt[i] = K;
 }
