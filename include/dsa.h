@@ -198,6 +198,24 @@ dsa_status dsa_sparse_attn_gated(const dsa_params* params, const dsa_ragged* rag
                                  int32_t* err_count, void* stream);
 
 /*
+ * Steps 3-4 with the layer's second branch mixed in by the gate ([HSA] "Indexer + Top-K:
+ * How Fine-Grained Sparse Attention Works", step 4 and the last line of its pseudocode,
+ * g * o_sparse + (1 - g) * o_linear; [FGS] "How Indexer + Top-K Works at Runtime", step 3
+ * "Fuse": g * precise + (1 - g) * compressed_context):
+ *   out[t,h,e] = sigmoid(gate[t,h,e]) * o[t,h,e] + (1 - sigmoid(gate[t,h,e])) * other[t,h,e]
+ * with o the exact sparse attention of dsa_sparse_attn_gated.  The second branch (the
+ * linear or compressed-context attention output) is an input computed elsewhere.
+ *   other  bf16 [total_q, Hq, d], 16-byte aligned; gate is required here.
+ * Every other argument, the LSE (of the sparse branch) and the error behaviour are as for
+ * dsa_sparse_attn_gated.
+ */
+dsa_status dsa_sparse_attn_gated_mix(const dsa_params* params, const dsa_ragged* ragged,
+                                     const void* q, const void* k_cache, const void* v_cache,
+                                     const int32_t* idx, int64_t ld_idx, int64_t q_begin,
+                                     int64_t q_count, const void* gate, const void* other,
+                                     void* out, float* lse, int32_t* err_count, void* stream);
+
+/*
  * Workspace for dsa_prefill / dsa_decode.  *min_bytes: the least that works (one query
  * row of scores per pass); *rec_bytes: the size this build recommends for throughput
  * (fewer, larger passes).  Either pointer may be NULL.  dsa_prefill runs steps 1-2 as

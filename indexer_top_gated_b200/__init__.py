@@ -54,6 +54,7 @@ EXPORTS = [
     "dsa_sparse_attn_gated", "dsa_workspace_size", "dsa_prefill", "dsa_decode",
     "dsa_device_status", "dsa_launch_count", "dsa_stage_timing", "dsa_stage_times",
     "dsa_decode_noalloc", "dsa_index_topk", "dsa_index_topk_workspace_size",
+    "dsa_sparse_attn_gated_mix",
 ]
 
 
@@ -69,6 +70,8 @@ def _load():
     L.dsa_index_scores.argtypes = [PP, RP, vp, vp, vp, i64, i64, vp, i64, vp]
     L.dsa_topk.argtypes = [PP, RP, vp, i64, i64, i64, vp, i64, vp, vp]
     L.dsa_sparse_attn_gated.argtypes = [PP, RP, vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, vp, vp]
+    L.dsa_sparse_attn_gated_mix.argtypes = [PP, RP, vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, vp,
+                                            vp, vp]
     L.dsa_workspace_size.argtypes = [PP, RP, ctypes.c_int, ctypes.POINTER(sz), ctypes.POINTER(sz)]
     L.dsa_index_topk_workspace_size.argtypes = [PP, RP, i64, ctypes.POINTER(sz), ctypes.POINTER(sz)]
     L.dsa_index_topk.argtypes = [PP, RP, vp, vp, vp, i64, i64, vp, i64, vp, vp, sz, vp]
@@ -162,6 +165,17 @@ def dsa_sparse_attn_gated(shape: LayerShape, rg: Ragged, q, k_cache, v_cache, id
                                      _ptr(v_cache), _ptr(idx), ld_idx, q_begin, q_count,
                                      _ptr(gate), _ptr(out), _ptr(lse), _ptr(err_count),
                                      _stream(stream)), "dsa_sparse_attn_gated")
+
+
+def dsa_sparse_attn_gated_mix(shape: LayerShape, rg: Ragged, q, k_cache, v_cache, idx, ld_idx: int,
+                              q_begin: int, q_count: int, gate, other, out, lse=None,
+                              err_count=None, stream=None):
+    p = shape.params()
+    _check(lib.dsa_sparse_attn_gated_mix(ctypes.byref(p), ctypes.byref(rg), _ptr(q),
+                                         _ptr(k_cache), _ptr(v_cache), _ptr(idx), ld_idx, q_begin,
+                                         q_count, _ptr(gate), _ptr(other), _ptr(out), _ptr(lse),
+                                         _ptr(err_count), _stream(stream)),
+           "dsa_sparse_attn_gated_mix")
 
 
 def dsa_workspace_size(shape: LayerShape, rg: Ragged, is_decode: bool = False):

@@ -490,7 +490,7 @@ dsa_status launch_attn(const DeviceState& dev, const dsa_params* P, const dsa_ra
                        const void* q, const void* k,
                        const void* v, const int32_t* idx, int64_t ld_idx, int64_t q_begin,
                        int64_t q_count, const void* gate, void* out, float* lse,
-                       int32_t* err_count, cudaStream_t stream) {
+                       int32_t* err_count, cudaStream_t stream, const void* other = nullptr) {
   if (q_count == 0) return DSA_OK;
   AttnArgs a;
   a.q_offsets = R->q_offsets;
@@ -505,6 +505,7 @@ dsa_status launch_attn(const DeviceState& dev, const dsa_params* P, const dsa_ra
   a.ld_idx = ld_idx;
   a.K = P->top_k;
   a.gate = static_cast<const __nv_bfloat16*>(gate);
+  a.other = static_cast<const __nv_bfloat16*>(other);
   a.out = static_cast<__nv_bfloat16*>(out);
   a.lse = lse;
   a.err_count = err_count;
@@ -700,6 +701,26 @@ dsa_status dsa_sparse_attn_gated(const dsa_params* P, const dsa_ragged* R, const
   DSA_TRY(device_setup(&dev));
   return launch_attn(*dev, P, R, q, k_cache, v_cache, idx, ld_idx, q_begin, q_count, gate, out,
                      lse, err_count, static_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_sparse_attn_gated_mix(const dsa_params* P, const dsa_ragged* R, const void* q,
+                                     const void* k_cache, const void* v_cache,
+                                     const int32_t* idx, int64_t ld_idx, int64_t q_begin,
+                                     int64_t q_count, const void* gate, const void* other,
+                                     void* out, float* lse, int32_t* err_count, void* stream) {
+  DSA_TRY(check_common(P, R));
+  DSA_TRY(check_attn(P));
+  if (!q || !k_cache || !v_cache || !idx || !gate || !other || !out) return DSA_ERR_INVALID_ARG;
+  if (q_begin < 0 || q_count < 0 || q_begin + q_count > R->total_q) return DSA_ERR_INVALID_ARG;
+  if (ld_idx < P->top_k) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+      !aligned16(gate) || !aligned16(other))
+    return DSA_ERR_INVALID_ARG;
+  if (q_count > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  DeviceState* dev = nullptr;
+  DSA_TRY(device_setup(&dev));
+  return launch_attn(*dev, P, R, q, k_cache, v_cache, idx, ld_idx, q_begin, q_count, gate, out,
+                     lse, err_count, static_cast<cudaStream_t>(stream), other);
 }
 
 dsa_status dsa_workspace_size(const dsa_params* P, const dsa_ragged* R, int is_decode,

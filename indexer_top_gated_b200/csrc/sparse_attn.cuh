@@ -18,7 +18,8 @@
 //    ~2^-17 relative instead of 2^-9: the error no longer scales with sum_j p_j |v_j|
 //    (which dominates outputs that nearly cancel).
 //  - warps of the same KV head merge (m, l, O) through shared memory; the epilogue
-//    divides by l, multiplies by sigmoid(gate) and stores bf16 (and the LSE).
+//    divides by l, multiplies by sigmoid(gate) (and adds the second branch weighted by
+//    1 - sigmoid(gate) when one is given) and stores bf16 (and the LSE).
 // The work per row is bound by the gather bytes (K * Hkv * d * 2 * 2 per query), so the
 // tensor-core path here only has to keep up with memory.
 #pragma once
@@ -52,6 +53,7 @@ struct AttnArgs {
   int64_t ld_idx;
   int K;
   const __nv_bfloat16* gate;
+  const __nv_bfloat16* other;  // second branch to mix in (needs gate), or nullptr
   __nv_bfloat16* out;
   float* lse;
   int32_t* err_count;
@@ -372,6 +374,26 @@ __global__ void __launch_bounds__(AttnGeom<HKV_CTA>::kThreads, 1) sparse_attn_ke
       const __nv_bfloat16* gb = reinterpret_cast<const __nv_bfloat16*>(&graw);
 #pragma unroll
       for (int k = 0; k < 8; ++k) gv[k] = 1.f / (1.f + __expf(-__bfloat162float(gb[k])));
+      if (a.other) {
+        // the second branch enters with weight 1 - sigmoid(g) = sigmoid(-g), formed
+        // directly so that it keeps its relative precision when sigmoid(g) is near 1
+        const uint4 oraw = __ldg(reinterpret_cast<const uint4*>(a.other + off));
+        const __nv_bfloat16* ob = reinterpret_cast<const __nv_bfloat16*>(&oraw);
+        float mix[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          mix[k] = __bfloat162float(ob[k]) / (1.f + __expf(__bfloat162float(gb[k])));
+        uint4 packed;
+        uint32_t* pw = reinterpret_cast<uint32_t*>(&packed);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          pw[k] = pack_bf16x2(acc[2 * k] * inv * gv[2 * k] + mix[2 * k],
+                              acc[2 * k + 1] * inv * gv[2 * k + 1] + mix[2 * k + 1]);
+        *reinterpret_cast<uint4*>(a.out + off) = packed;
+        if (a.lse && d0 == 0)
+          a.lse[i * a.Hq + h] = Lsum > 0.f ? (M + __log2f(Lsum)) * 0.69314718055994531f : -INFINITY;
+        continue;
+      }
     } else {
 #pragma unroll
       for (int k = 0; k < 8; ++k) gv[k] = 1.f;

@@ -65,6 +65,8 @@ def lib():
         L.oracle_layer_rows.argtypes = [ctypes.POINTER(Problem), vp, vp, vp, vp, vp, vp, vp, vp, i64,
                                         i32, vp, vp, vp]
         L.oracle_layer_rows.restype = None
+        L.oracle_gate_mix.argtypes = [vp, vp, vp, i64, vp]
+        L.oracle_gate_mix.restype = None
         L.oracle_hardware_threads.argtypes = []
         L.oracle_hardware_threads.restype = i32
         _lib = L
@@ -121,6 +123,18 @@ class Oracle:
                                      r, out.ctypes.data, lse.ctypes.data)
         return out, lse
 
+    def sparse_attn_mix_row(self, r: int, idx: np.ndarray, o2: np.ndarray):
+        """Gated mixing with the second branch: sigmoid(g) * o + (1 - sigmoid(g)) * o2 for
+        packed query row r (o the ungated attention over idx; o2 [Hq, d] bf16 bits)."""
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+        o = np.empty((self.Hq, self.d), dtype=np.float64)
+        lib().oracle_sparse_attn_row(ctypes.byref(self.P), _ptr(self.a["q"]), _ptr(self.a["k"]),
+                                     _ptr(self.a["v"]), None, idx.ctypes.data, r, o.ctypes.data,
+                                     None)
+        g = np.ascontiguousarray(self.a["gate"][r], dtype=np.uint16)
+        o2 = np.ascontiguousarray(o2, dtype=np.uint16)
+        return gate_mix(o, g, o2)
+
     def layer_rows(self, rows: Sequence[int], nthreads: int = 0):
         rows = np.ascontiguousarray(rows, dtype=np.int64)
         nr = len(rows)
@@ -134,6 +148,18 @@ class Oracle:
                                 _ptr(self.a["v"]), _ptr(self.a.get("gate")), rows.ctypes.data, nr,
                                 nthreads, idx.ctypes.data, out.ctypes.data, lse.ctypes.data)
         return idx, out, lse
+
+
+def gate_mix(o: np.ndarray, gate_bits: np.ndarray, o2_bits: np.ndarray) -> np.ndarray:
+    """Oracle step 4 with the second branch, elementwise over equally shaped arrays: o fp64,
+    gate logits and o2 as bf16 bit patterns (uint16)."""
+    o = np.ascontiguousarray(o, dtype=np.float64)
+    g = np.ascontiguousarray(gate_bits, dtype=np.uint16)
+    o2 = np.ascontiguousarray(o2_bits, dtype=np.uint16)
+    assert o.shape == g.shape == o2.shape
+    out = np.empty_like(o)
+    lib().oracle_gate_mix(o.ctypes.data, g.ctypes.data, o2.ctypes.data, o.size, out.ctypes.data)
+    return out
 
 
 def topk_row(s: np.ndarray, K: int) -> np.ndarray:

@@ -29,7 +29,11 @@
  *      ([HSA] same section, step 3 and its pseudocode; [SAE] "5. Abstract
  *       Implementation Sketch of Indexer + Top-K").
  *   4. sigmoid output gate, per head and dimension: out = sigmoid(g) * o
- *      ([HSA] same section, step 4; [GSA] "2. The Core Change", pseudocode).
+ *      ([HSA] same section, step 4; [GSA] "2. The Core Change", pseudocode), or, with
+ *      the layer's second branch o2 (the linear / compressed-context output),
+ *      out = sigmoid(g) * o + (1 - sigmoid(g)) * o2 ([HSA] same section, step 4 and the
+ *      last line of its pseudocode; [FGS] "How Indexer + Top-K Works at Runtime",
+ *      step 3 "Fuse" of its pseudocode).
  * Parity is pinned by the tests against brute force, closed forms and library
  * routines (dense causal attention when K covers the whole history).
  */
@@ -190,6 +194,18 @@ void oracle_sparse_attn_row(const oracle_problem* P, const uint16_t* q, const ui
       out[(int64_t)h * d + e] = o;
     }
     if (lse) lse[h] = rows.empty() ? -INFINITY : m + std::log(l);
+  }
+}
+
+/* Step 4 with the second branch: out[e] = s * o[e] + (1 - s) * o2[e], s = sigmoid(gate[e]),
+ * over the n elements of one query row ([Hq, d]): o is the row's ungated attention output
+ * (oracle_sparse_attn_row with gate NULL), gate and o2 the row's bf16 logits and second-
+ * branch values. */
+void oracle_gate_mix(const double* o, const uint16_t* gate, const uint16_t* o2, int64_t n,
+                     double* out) {
+  for (int64_t e = 0; e < n; ++e) {
+    const double s = 1.0 / (1.0 + std::exp(-bf16_value(gate[e])));
+    out[e] = s * o[e] + (1.0 - s) * bf16_value(o2[e]);
   }
 }
 

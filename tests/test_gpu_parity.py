@@ -207,6 +207,41 @@ def test_sparse_attn_matches_oracle(case):
     assert int(err.item()) == 0
 
 
+@pytest.mark.parametrize("case", ["gqa8", "mha", "gqa16"])
+def test_sparse_attn_gated_mix_matches_oracle(case):
+    """The gate mixing in a second branch: sigmoid(g) o + (1 - sigmoid(g)) o2."""
+    cfg = ATTN_CASES[case]
+    w = _workload([40, 1, 90], [300, 50, 90], K=96, **cfg)
+    host = S.make_host_inputs(w)
+    dev = _dev(host)
+    orc = O.Oracle.for_workload(w, host)
+    idx_ref, out_gated, _ = orc.layer_rows(range(w.total_q))
+    rng = np.random.default_rng(5)
+    o2_bits = S.f32_to_bf16_bits((rng.normal(size=(w.total_q, w.n_q_heads, 128)) * 2e-3)
+                                 .astype(np.float32))
+    ref = np.stack([orc.sparse_attn_mix_row(r, idx_ref[r], o2_bits[r]) for r in range(w.total_q)])
+    o2 = torch.from_numpy(o2_bits.view(np.int16)).cuda().view(torch.bfloat16)
+    idx_t = torch.from_numpy(idx_ref).cuda()
+    shape = dsa.workload_shape(w)
+    out = torch.zeros((w.total_q, w.n_q_heads, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros((w.total_q, w.n_q_heads), device="cuda")
+    dsa.dsa_sparse_attn_gated_mix(shape, _rg(w, dev), dev["q"], dev["k"], dev["v"], idx_t, w.top_k,
+                                  0, w.total_q, dev["gate"], o2, out, lse)
+    torch.cuda.synchronize()
+    PT.assert_close(PT.bf16_tensor_to_f64(out), ref, case + " mix")
+    # the second branch matters: the gated-only reference must fail the same check
+    with pytest.raises(AssertionError):
+        PT.assert_close(PT.bf16_tensor_to_f64(out), out_gated, case + " mix vs gated")
+    # a zero second branch gives dsa_sparse_attn_gated's output bit for bit
+    zero = torch.zeros_like(o2)
+    out0 = torch.zeros_like(out)
+    dsa.dsa_sparse_attn_gated_mix(shape, _rg(w, dev), dev["q"], dev["k"], dev["v"], idx_t, w.top_k,
+                                  0, w.total_q, dev["gate"], zero, out0)
+    out_g, _, _ = _attn_run(w, dev, idx_t, lse=False, err=False)
+    torch.cuda.synchronize()
+    assert torch.equal(out0, out_g)
+
+
 def test_sparse_attn_sharp_softmax_and_no_gate():
     """q, k ~ N(0,1): the softmax is far from uniform; also the ungated path."""
     w = _workload([64], [1000], K=512, scale=1.0, gate=False)

@@ -110,6 +110,13 @@ def test_host_validation_rejects_bad_arguments():
     rg2 = _rg(dsa, batch=2, max_q=3)
     assert L.dsa_decode(ctypes.byref(p), ctypes.byref(rg2), A, A, A, A, A, A, null, A, null, null,
                         A, 1 << 20, null) == dsa.DSA_ERR_INVALID_ARG
+    # the mixing entry needs both the gate logits and the second branch
+    for gate_p, other_p in ((None, A), (A, None)):
+        assert L.dsa_sparse_attn_gated_mix(ctypes.byref(p), ctypes.byref(rg), A, A, A, A, 4, 0, 1,
+                                           gate_p, other_p, A, null, null, null) == \
+            dsa.DSA_ERR_INVALID_ARG
+    assert L.dsa_sparse_attn_gated_mix(ctypes.byref(p), ctypes.byref(rg), A, A, A, A, 4, 0, 1, A,
+                                       A + 8, A, null, null, null) == dsa.DSA_ERR_INVALID_ARG
     # null ragged / params
     assert L.dsa_topk(None, ctypes.byref(rg), A, 8, 0, 1, A, 4, null, null) == dsa.DSA_ERR_INVALID_ARG
 

@@ -292,6 +292,36 @@ def test_attention_invariants():
     np.testing.assert_array_equal(out2, out * 0.5)
 
 
+def test_gate_mix_with_second_branch():
+    """out = sigmoid(g) o + (1 - sigmoid(g)) o2: gate 0 gives the exact midpoint, g and -g
+    sum to o + o2 (sigmoid(g) + sigmoid(-g) = 1), o2 = o gives o, very large logits select
+    one branch, and o2 = 0 reduces to the gated output sigmoid(g) o of the attention row."""
+    rng = np.random.default_rng(11)
+    n = 64
+    o = rng.normal(size=n)
+    o2_bits = _bf16(rng.normal(size=n))
+    o2 = _val(o2_bits)
+    zero = _bf16(np.zeros(n))
+    np.testing.assert_array_equal(O.gate_mix(o, zero, o2_bits), 0.5 * o + 0.5 * o2)
+    g = _bf16(rng.normal(size=n) * 3)
+    gm = _bf16(-_val(g))
+    np.testing.assert_allclose(O.gate_mix(o, g, o2_bits) + O.gate_mix(o, gm, o2_bits), o + o2,
+                               rtol=0, atol=1e-14)
+    same = _val(_bf16(o))
+    np.testing.assert_allclose(O.gate_mix(same, g, _bf16(o)), same, rtol=1e-14, atol=1e-15)
+    big = _bf16(np.full(n, 60.0))
+    np.testing.assert_allclose(O.gate_mix(o, big, o2_bits), o, rtol=1e-20, atol=1e-24)
+    np.testing.assert_allclose(O.gate_mix(o, _bf16(np.full(n, -60.0)), o2_bits), o2, rtol=1e-20,
+                               atol=1e-24)
+    # o2 = 0: the gated attention output of the same row
+    a = _rand_layer(12, [3], [40], gate=True)
+    orc = _problem(a, top_k=8, n_idx_heads=3, idx_dim=8, n_q_heads=4, n_kv_heads=2, head_dim=8)
+    idx = np.array([0, 3, 5, 9, 17, 20, 31, 38], dtype=np.int32)
+    gated, _ = orc.sparse_attn_row(2, idx)
+    mixed = orc.sparse_attn_mix_row(2, idx, np.zeros((4, 8), np.uint16))
+    np.testing.assert_allclose(mixed, gated, rtol=1e-15, atol=1e-17)
+
+
 def test_padding_entries_are_ignored():
     L, Hq, d = 9, 1, 4
     rng = np.random.default_rng(7)
