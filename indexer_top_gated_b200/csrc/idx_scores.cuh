@@ -289,15 +289,16 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       mbar_wait_bounded(smem_u32(&tfull[j & 1]), (j >> 1) & 1, nullptr, nullptr);
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2-9)
+    // ------------------------------------------------------------ epilogue (warps 2-17)
     const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
     const int sub = (warp - 2) >> 2;  // the warps of a quadrant take every kIdxSubs-th chunk
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     // shared head weights with the (positive) dequantisation scale folded in:
     // w * max(0, c * x) = (w * c) * max(0, x) for c > 0
-    float wsh[4] = {0.f, 0.f, 0.f, 0.f};
-    if (a.w_row_stride == 0)
-      for (int h = 0; h < H; ++h) wsh[h] = __ldg(a.w + h) * a.scale;
+    // (unrolled with constant indices, so that the weights stay in registers)
+    float wsh[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) wsh[h] = (a.w_row_stride == 0 && h < H) ? __ldg(a.w + h) * a.scale : 0.f;
     // candidate variant: this warp's score block (the chunk of rows c0 always goes to
     // the warp with sub = (c0 / 16) % kIdxSubs, so each (quadrant, row) has one writer)
     float* tile = tiles + (warp - 2) * (kIdxTileBytes / 4);
@@ -307,6 +308,10 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       int64_t rs, re, pbase;
       int kh;
       if (!seq_range(b, rs, re, kh, pbase)) continue;
+      // 32-bit from here on (positions and rows of a launch stay below 2^31): p0 is the
+      // position of tile row 0 in sequence b (row cc sees keys up to (p0 + cc) >> shift)
+      const int p0 = (int)(pbase + r0);
+      const int row0 = (int)(r0 - a.q_begin);
       for (int kt = kt_lo; kt < kh; ++kt, ++i) {
         const int buf = i & 1;
         if (!mbar_wait_bounded(smem_u32(&tfull[buf]), (i >> 1) & 1, a.status, &s_abort)) {
@@ -314,14 +319,14 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           break;
         }
         tc_fence_after();
-        const int64_t j = (int64_t)kt * kIdxKeyTile + quad * 32 + lane;  // key position
+        const int j = kt * kIdxKeyTile + quad * 32 + lane;  // key position
         // columns c of this tile that belong to sequence b: rows rs..re-1
         const int c_lo = (int)(rs - r0), c_hi = (int)(re - r0);
         for (int c0 = 16 * sub; c0 < c_hi; c0 += 16 * kIdxSubs) {
           if (c0 + 16 <= c_lo) continue;  // rows of an earlier sequence of the tile
           // skip chunks whose rows all precede this key tile (causal)
-          const int64_t p_chunk_max = (pbase + r0 + (c0 + 15 < c_hi - 1 ? c0 + 15 : c_hi - 1)) >> a.shift;
-          if (p_chunk_max < (int64_t)kt * kIdxKeyTile) continue;
+          const int p_chunk_max = (p0 + (c0 + 15 < c_hi - 1 ? c0 + 15 : c_hi - 1)) >> a.shift;
+          if (p_chunk_max < kt * kIdxKeyTile) continue;
           // heads in pairs: two TMEM loads in flight, then their ReLU-weighted sum
           // (the accumulation order over heads is 0, 1, 2, 3 as before)
           float acc[16];
@@ -342,9 +347,16 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
               if (h >= H) break;
               reg_fence(v[q]);
               if (a.w_row_stride == 0) {
+                // two columns per packed fma (each lane of it rounds like fmaf)
+                const float2 w2 = make_float2(wsh[h], wsh[h]);
 #pragma unroll
-                for (int c = 0; c < 16; ++c)
-                  acc[c] = fmaf(wsh[h], fmaxf(__uint_as_float(v[q][c]), 0.f), acc[c]);
+                for (int c = 0; c < 16; c += 2) {
+                  const float2 x = make_float2(fmaxf(__uint_as_float(v[q][c]), 0.f),
+                                               fmaxf(__uint_as_float(v[q][c + 1]), 0.f));
+                  const float2 r2 = __ffma2_rn(w2, x, make_float2(acc[c], acc[c + 1]));
+                  acc[c] = r2.x;
+                  acc[c + 1] = r2.y;
+                }
               } else {
 #pragma unroll
                 for (int c = 0; c < 16; ++c) {
@@ -359,7 +371,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           // rows r0+c0 .. r0+c0+15; key j.  Interior chunk: every row belongs to this
           // sequence and sees the whole key tile, so no per-element predicate is needed.
           const bool inside = c0 >= c_lo && c0 + 16 <= c_hi &&
-                              (int64_t)kt * kIdxKeyTile + (kIdxKeyTile - 1) <= ((pbase + r0 + c0) >> a.shift);
+                              kt * kIdxKeyTile + (kIdxKeyTile - 1) <= ((p0 + c0) >> a.shift);
           if (CAND) {
             // keep the scores >= the row's threshold (float order; -0.0 == +0.0)
 #pragma unroll
@@ -373,10 +385,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             // keys of this lane that the row may see: k < k_lim
             int k_lim = 16;
             if (!inside) {
-              const int64_t pr = (pbase + r0 + cc) >> a.shift;  // last key row the row sees
-              const int64_t first = (int64_t)kt * kIdxKeyTile + quad * 32 + kh;
-              const int64_t lim = pr - first + 1;
-              k_lim = (cc < c_lo || cc >= c_hi || lim <= 0) ? 0 : lim >= 16 ? 16 : (int)lim;
+              const int pr = (p0 + cc) >> a.shift;  // last key row the row sees
+              const int lim = pr - (kt * kIdxKeyTile + quad * 32 + kh) + 1;
+              k_lim = (cc < c_lo || cc >= c_hi || lim <= 0) ? 0 : lim >= 16 ? 16 : lim;
             }
             uint32_t m = 0;
 #pragma unroll
@@ -392,7 +403,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             const uint32_t n_hi = __shfl_sync(0xFFFFFFFFu, (uint32_t)__popc(m), 16 + (lane & 15));
             if (lane < 16) s_cnt[quad][cc] = base + n_lo + n_hi;
             const int seg = a.cap >> 2;
-            float2* dst = a.cand + (r0 + cc - a.q_begin) * (int64_t)a.cap + quad * seg;
+            float2* dst = a.cand + (int64_t)(row0 + cc) * a.cap + quad * seg;
             const int j0 = kt * kIdxKeyTile + quad * 32 + kh;
             while (m) {
               const int k = __ffs(m) - 1;
@@ -403,7 +414,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             __syncwarp();  // the block is read before the next chunk overwrites it
             continue;
           }
-          float* dst = a.scores + (r0 + c0 - a.q_begin) * a.ld + j;
+          float* dst = a.scores + (int64_t)(row0 + c0) * a.ld + j;
           const bool interior = inside && (int64_t)kt * kIdxKeyTile + kIdxKeyTile <= a.ld;
           if (interior) {
 #pragma unroll
@@ -415,8 +426,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
               const int cc = c0 + c;
-              const int64_t r = r0 + cc;
-              if (cc >= c_lo && cc < c_hi && j <= ((pbase + r) >> a.shift) && j < a.ld) *dst = acc[c];
+              if (cc >= c_lo && cc < c_hi && j <= ((p0 + cc) >> a.shift) && j < a.ld) *dst = acc[c];
               dst += a.ld;
             }
           }
