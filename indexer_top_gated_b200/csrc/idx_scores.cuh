@@ -327,22 +327,24 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           // skip chunks whose rows all precede this key tile (causal)
           const int p_chunk_max = (p0 + (c0 + 15 < c_hi - 1 ? c0 + 15 : c_hi - 1)) >> a.shift;
           if (p_chunk_max < kt * kIdxKeyTile) continue;
-          // heads in pairs: two TMEM loads in flight, then their ReLU-weighted sum
-          // (the accumulation order over heads is 0, 1, 2, 3 as before)
+          // heads in groups of HPB (two, or one in the candidate variant, which needs the
+          // registers): HPB TMEM loads in flight, then their ReLU-weighted sum (the
+          // accumulation order over heads is 0, 1, 2, 3 either way)
+          constexpr int HPB = CAND ? 1 : 2;
           float acc[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) acc[c] = 0.f;
 #pragma unroll
-          for (int hp = 0; hp < 4; hp += 2) {
+          for (int hp = 0; hp < 4; hp += HPB) {
             if (hp >= H) break;
-            uint32_t v[2][16];
+            uint32_t v[HPB][16];
 #pragma unroll
-            for (int q = 0; q < 2; ++q)
+            for (int q = 0; q < HPB; ++q)
               if (hp + q < H)
                 tmem_ld16_async(tmem + lane_base + (uint32_t)(buf * H * BQ + (hp + q) * BQ + c0), v[q]);
             tmem_wait_ld();
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
+            for (int q = 0; q < HPB; ++q) {
               const int h = hp + q;
               if (h >= H) break;
               reg_fence(v[q]);
