@@ -85,7 +85,20 @@ typedef struct {
   int32_t max_q_len;          /* host: >= max_b Q_b                                */
   int32_t max_kv_len;         /* host: >= max_b L_b                                */
   int64_t total_q;            /* host: q_offsets[B]                                */
-  int64_t total_kv;           /* host: kv_offsets[B]                               */
+  int64_t total_kv;           /* host: kv_offsets[B] (contiguous); with a block table,
+                                 the rows of the cache arrays (pages * page_size)   */
+  /* Paged cache (optional).  NULL block_table: sequence b's cache rows are rows
+   * kv_offsets[b] .. kv_offsets[b+1]-1 of k_idx / k_cache / v_cache.  Otherwise position
+   * j of sequence b lives in row block_table[b * max_pages + j / page_size] * page_size
+   * + j % page_size of those arrays, and kv_offsets only gives the lengths
+   * L_b = kv_offsets[b+1] - kv_offsets[b].  This is the serving layout of a cache that is
+   * "no longer contiguous" ([FGS] "How Indexer + Top-K Works at Runtime", engineering
+   * details).  page_size: a power of two >= 128 (a 128-position indexer tile never
+   * straddles pages); max_pages >= ceil(max_kv_len / page_size); every referenced page id
+   * in [0, total_kv / page_size). */
+  const int32_t* block_table; /* device [B, max_pages] or NULL                     */
+  int32_t max_pages;
+  int32_t page_size;
 } dsa_ragged;
 
 /* Layer shape and numerics.  Supported by this build: idx_dim = 64,

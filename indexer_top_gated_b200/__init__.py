@@ -45,7 +45,8 @@ class Ragged(ctypes.Structure):
         ("batch", ctypes.c_int32), ("q_offsets", ctypes.c_void_p),
         ("kv_offsets", ctypes.c_void_p), ("max_q_len", ctypes.c_int32),
         ("max_kv_len", ctypes.c_int32), ("total_q", ctypes.c_int64),
-        ("total_kv", ctypes.c_int64),
+        ("total_kv", ctypes.c_int64), ("block_table", ctypes.c_void_p),
+        ("max_pages", ctypes.c_int32), ("page_size", ctypes.c_int32),
     ]
 
 
@@ -135,11 +136,21 @@ class LayerShape:
                       self.idx_scale_k, self.attn_scale, self.w_row_stride)
 
 
-def ragged(q_offsets, kv_offsets, q_lens: Sequence[int], kv_lens: Sequence[int]) -> Ragged:
-    """Build a dsa_ragged from device int32 offset tensors and host lengths."""
-    return Ragged(len(q_lens), q_offsets.data_ptr(), kv_offsets.data_ptr(),
-                  int(max(q_lens)) if len(q_lens) else 0,
-                  int(max(kv_lens)) if len(kv_lens) else 0, int(sum(q_lens)), int(sum(kv_lens)))
+def ragged(q_offsets, kv_offsets, q_lens: Sequence[int], kv_lens: Sequence[int],
+           block_table=None, page_size: int = 0, cache_rows: Optional[int] = None) -> Ragged:
+    """Build a dsa_ragged from device int32 offset tensors and host lengths; with a device
+    int32 block table [batch, max_pages] the cache arrays are paged (cache_rows rows).
+    The descriptor holds only the tensors' addresses: keep them alive while it is used."""
+    rg = Ragged(len(q_lens), q_offsets.data_ptr(), kv_offsets.data_ptr(),
+                int(max(q_lens)) if len(q_lens) else 0,
+                int(max(kv_lens)) if len(kv_lens) else 0, int(sum(q_lens)), int(sum(kv_lens)),
+                None, 0, 0)
+    if block_table is not None:
+        rg.block_table = block_table.data_ptr()
+        rg.max_pages = int(block_table.shape[1])
+        rg.page_size = int(page_size)
+        rg.total_kv = int(cache_rows)
+    return rg
 
 
 def dsa_index_scores(shape: LayerShape, rg: Ragged, q_idx, k_idx, w, q_begin: int, q_count: int,

@@ -279,6 +279,23 @@ DSA_DEV float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
 // ------------------------------------------------------------------ cp.async
 
 // 16-byte async copy global -> shared; src_bytes = 0 zero-fills the destination.
+// Row of the cache arrays that holds position j of sequence b: contiguous (kv_offsets[b] + j)
+// without a block table, else page table[b * max_pages + (j >> shift)] of 2^shift rows.  A
+// page id outside [0, n_pages) is clamped into it (bad device data reads a wrong page, never
+// outside the arrays).
+struct CachePages {
+  const int32_t* table;  // nullptr: contiguous
+  int max_pages;
+  int shift;             // log2(page size)
+  int n_pages;           // pages in the cache arrays
+};
+DSA_DEV int64_t cache_row(const int32_t* kv_offsets, const CachePages& pg, int b, int64_t j) {
+  if (!pg.table) return (int64_t)__ldg(kv_offsets + b) + j;
+  int page = __ldg(pg.table + (int64_t)b * pg.max_pages + (j >> pg.shift));
+  page = page < 0 ? 0 : page >= pg.n_pages ? pg.n_pages - 1 : page;
+  return ((int64_t)page << pg.shift) + (j & ((int64_t(1) << pg.shift) - 1));
+}
+
 DSA_DEV void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
                "r"(src_bytes)

@@ -147,7 +147,26 @@ dsa_status check_common(const dsa_params* P, const dsa_ragged* R) {
     return DSA_ERR_INVALID_ARG;
   if (R->total_q > INT32_MAX || R->total_kv > INT32_MAX) return DSA_ERR_UNSUPPORTED;
   if (P->top_k < 1 || P->top_k > kMaxTopK) return DSA_ERR_UNSUPPORTED;
+  if (R->block_table) {
+    const int ps = R->page_size;
+    if (ps < 128 || ps > (1 << 24) || (ps & (ps - 1)) != 0) return DSA_ERR_INVALID_ARG;
+    if (R->max_pages < 1 || (int64_t)R->max_pages * ps < R->max_kv_len) return DSA_ERR_INVALID_ARG;
+    if (R->total_kv % ps != 0) return DSA_ERR_INVALID_ARG;
+  }
   return DSA_OK;
+}
+
+CachePages cache_pages(const dsa_ragged* R) {
+  CachePages pg;
+  pg.table = R->block_table;
+  pg.max_pages = R->block_table ? R->max_pages : 0;
+  pg.shift = 0;
+  pg.n_pages = 0;
+  if (R->block_table) {
+    while ((1 << pg.shift) < R->page_size) ++pg.shift;
+    pg.n_pages = (int)(R->total_kv >> pg.shift);
+  }
+  return pg;
 }
 
 dsa_status check_indexer(const dsa_params* P) {
@@ -252,6 +271,7 @@ dsa_status launch_index_scores(const DeviceState& dev, const dsa_params* P, cons
   a.ld = ld;
   a.status = dev.status;
   a.shift = var.shift;
+  a.pages = var.shift ? CachePages{nullptr, 0, 0, 0} : cache_pages(R);  // samples are contiguous
   a.thr = var.thr;
   a.cand = var.cand;
   a.cap = var.cap;
@@ -336,7 +356,10 @@ bool fused_geom(const dsa_params* P, const dsa_ragged* R, FusedGeom* g) {
   const int64_t max_n = std::max(R->max_kv_len, 1);
   g->ld_s = round_up(((max_n - 1) >> kSampleShift) + 1, 32);
   g->ld_fb = round_up(max_n, 4);
-  g->samp_rows = (R->total_kv >> kSampleShift) + R->batch + 1;
+  // sampled rows are laid out by the logical offsets: sum_b L_b <= total_kv when contiguous,
+  // <= batch * max_kv_len when paged (pages may be shared)
+  const int64_t logical = R->block_table ? (int64_t)R->batch * R->max_kv_len : R->total_kv;
+  g->samp_rows = (logical >> kSampleShift) + R->batch + 1;
   g->key_row = (int64_t)P->n_idx_heads * 64 * (P->idx_dtype == DSA_FP8_E4M3 ? 1 : 2);
   g->fixed_bytes = round_up(g->samp_rows * g->key_row, 256) +
                    round_up((int64_t)kFallbackCtas * g->ld_fb * 4, 256) + 256 * 4;
@@ -395,7 +418,7 @@ dsa_status fused_prepare(const DeviceState& dev, const dsa_ragged* R, const void
   StageScope scope(0, stream);
   idx_sample_keys_kernel<<<(unsigned)std::max<int64_t>(blocks, 1), 256, 0, stream>>>(
       R->kv_offsets, R->batch, kSampleShift, static_cast<const uint4*>(k_idx), f.k_samp, vec,
-      g.samp_rows);
+      g.samp_rows, cache_pages(R));
   ++t_launches;
   return launch_status("idx_sample_keys_kernel");
 }
@@ -468,6 +491,7 @@ dsa_status fused_pass(const DeviceState& dev, const dsa_params* P, const dsa_rag
   a.idx_scale = P->idx_scale_q * P->idx_scale_k;
   a.fb_scores = f.fb_scores;
   a.ld_fb = g.ld_fb;
+  a.pages = cache_pages(R);
   const size_t smem = topk_smem_bytes(R->max_kv_len);
   a.bm_words = topk_fused_bm_words(std::max(R->max_kv_len, 1));
   {  // (4) exact selection over the candidates
@@ -515,6 +539,7 @@ dsa_status launch_attn(const DeviceState& dev, const dsa_params* P, const dsa_ra
   a.G = P->n_q_heads / P->n_kv_heads;
   const float scale = P->attn_scale > 0.f ? P->attn_scale : 1.0f / std::sqrt((float)P->head_dim);
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.pages = cache_pages(R);
   const int hkv_cta = std::min(P->n_kv_heads, 8);
   const int nt = a.G > 8 ? 2 : 1;
   dim3 grid((unsigned)q_count, (unsigned)(P->n_kv_heads / hkv_cta));
@@ -650,7 +675,7 @@ const char* dsa_status_string(dsa_status s) {
   return "unknown status";
 }
 
-int32_t dsa_version(void) { return 100; }
+int32_t dsa_version(void) { return 101; }
 
 dsa_status dsa_index_scores(const dsa_params* P, const dsa_ragged* R, const void* q_idx,
                             const void* k_idx, const float* w, int64_t q_begin, int64_t q_count,

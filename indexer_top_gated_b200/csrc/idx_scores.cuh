@@ -61,6 +61,7 @@ struct IdxArgs {
   float2* cand;        // [q_count, cap]: 4 segments of cap/4 (position as int bits, score)
   int cap;             // a multiple of 4
   int32_t* cand_cnt;   // [q_count, 4] candidates found per segment (may exceed cap/4)
+  CachePages pages;    // paged k_idx (not with sampled keys, which are always contiguous)
 };
 
 // first key-tensor row of sequence b
@@ -226,6 +227,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         if (!seq_range(b, rs, re, kh, pb)) continue;
         const int64_t kbase = idx_key_base(a, b);
         for (int kt = kt_lo; kt < kh; ++kt, ++i) {
+          // a key tile never straddles a page (pages are multiples of 128 positions)
+          const int64_t krow = a.pages.table ? cache_row(a.kv_offsets, a.pages, b, (int64_t)kt * kIdxKeyTile)
+                                             : kbase + (int64_t)kt * kIdxKeyTile;
           const int s = i % ST;
           if (!mbar_wait_bounded(smem_u32(&empty[s]), ((i / ST) & 1) ^ 1, a.status, &s_abort)) {
             ok = false;
@@ -234,7 +238,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           mbar_arrive_expect_tx(smem_u32(&full[s]), H * k_head_bytes);
           for (int h = 0; h < H; ++h)
             tma_load_2d(smem_u32(sK + ((size_t)s * H + h) * k_head_bytes), &tmap_k,
-                        smem_u32(&full[s]), h * 64, (int)(kbase + (int64_t)kt * kIdxKeyTile));
+                        smem_u32(&full[s]), h * 64, (int)krow);
         }
       }
       if (!ok) {
@@ -451,13 +455,15 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       if (r0 + c / 4 <= r_last) a.cand_cnt[(r0 - a.q_begin) * 4 + c] = (int32_t)s_cnt[c % 4][c / 4];
 }
 
-// Sampled key tensor of the fused path: row (kv_offsets[b] >> shift) + b + m is row
-// kv_offsets[b] + (m << shift) of k_idx, for every sequence b and m < ceil(L_b / 2^shift);
-// rows between sequences are zero.  One warp per row, `vec` 16-byte words per row.
+// Sampled key tensor of the fused path: row (kv_offsets[b] >> shift) + b + m holds position
+// m << shift of sequence b (cache row kv_offsets[b] + (m << shift), or its page), for every
+// sequence b and m < ceil(L_b / 2^shift); rows between sequences are zero.  One warp per
+// row, `vec` 16-byte words per row.
 __global__ void __launch_bounds__(256) idx_sample_keys_kernel(const int32_t* kv_offsets,
                                                               int batch, int shift,
                                                               const uint4* k, uint4* ks,
-                                                              int vec, int64_t rows) {
+                                                              int vec, int64_t rows,
+                                                              CachePages pages) {
   const int lane = lane_id();
   const int64_t n_warps = (int64_t)gridDim.x * (blockDim.x >> 5);
   for (int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); g < rows;
@@ -470,8 +476,8 @@ __global__ void __launch_bounds__(256) idx_sample_keys_kernel(const int32_t* kv_
     }
     const int64_t ko = __ldg(kv_offsets + lo), kn = __ldg(kv_offsets + lo + 1);
     const int64_t m = g - ((ko >> shift) + lo);
-    const int64_t src = ko + (m << shift);
-    const bool real = m >= 0 && src < kn;
+    const bool real = m >= 0 && ko + (m << shift) < kn;
+    const int64_t src = real ? cache_row(kv_offsets, pages, lo, m << shift) : 0;
     for (int v = lane; v < vec; v += 32)
       ks[g * vec + v] = real ? __ldg(k + src * vec + v) : make_uint4(0u, 0u, 0u, 0u);
   }

@@ -60,6 +60,7 @@ struct AttnArgs {
   int* status;
   int Hq, Hkv, G;
   float scale_log2;  // softmax scale * log2(e)
+  CachePages pages;  // paged k_cache / v_cache
 };
 
 template <int HKV_CTA>
@@ -140,14 +141,16 @@ __global__ void __launch_bounds__(AttnGeom<HKV_CTA>::kThreads, 1) sparse_attn_ke
   // and are masked in the softmax, so the copies need no per-piece predicate.
   const int lt = lane & 15, lhi = lane >> 4;
   const int64_t v_minus_k = a.v - a.k;  // V row = K row + this many elements
-  const __nv_bfloat16* kpiece = kh + kbase * row_stride + lt * 8;  // row 0, this lane's piece
+  const __nv_bfloat16* kpiece = kh + lt * 8;  // this lane's piece of cache row 0
   const uint32_t swz = (uint32_t)((lt ^ lhi) << 4);  // lt ^ ((2k + lhi) & 7) = (lt ^ lhi) ^ 2k&7
   auto load_chunk = [&](int c, int st) -> uint32_t {
     const int e = c * CH + sub * 16 + lt;
     const int j = e < K ? __ldg(irow + e) : -1;
     const bool valid = j >= 0 && (int64_t)j <= p;
     const uint32_t vmask = __ballot_sync(0xFFFFFFFFu, valid) & 0xFFFFu;
-    const int rowi = valid ? j : 0;
+    // the cache row of the position (or of position 0 for padding)
+    const int rowi = a.pages.table ? (int)cache_row(a.kv_offsets, a.pages, b, valid ? j : 0)
+                                   : (int)kbase + (valid ? j : 0);
     const uint32_t kdst = smem_u32(wsm + st * Geo::kWarpStage) + lhi * 256;
     const uint32_t vdst = kdst + Geo::kWarpHalf;
 #pragma unroll

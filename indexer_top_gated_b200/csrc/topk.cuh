@@ -100,6 +100,7 @@ struct TopkArgs {
   float idx_scale;
   float* fb_scores;         // [gridDim.x, ld_fb]
   int64_t ld_fb;
+  CachePages pages;         // paged k_idx
 };
 
 // Threshold estimate from sampled scores (fused path).
@@ -747,14 +748,14 @@ DSA_DEV void topk_recompute_scores(const TopkArgs& a, int64_t r, int b, int nn, 
   if (tid < H)
     s_w[tid] = a.w_row_stride ? __ldg(a.w + r * a.w_row_stride + tid) : __ldg(a.w + tid) * a.idx_scale;
   __syncthreads();
-  const int64_t ko = __ldg(a.kv_offsets + b);
   for (int j = tid; j < nn; j += kTopkThreads) {
+    const int64_t krow = cache_row(a.kv_offsets, a.pages, b, j);
     float acc = 0.f;
     for (int h = 0; h < H; ++h) {
       float dot = 0.f;
       if (a.idx_fp8) {
         const uint4* kr = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.k_idx) +
-                                                         (ko + j) * D + h * 64);
+                                                         krow * D + h * 64);
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           const uint4 u = __ldg(kr + v);
@@ -765,7 +766,7 @@ DSA_DEV void topk_recompute_scores(const TopkArgs& a, int64_t r, int b, int nn, 
         }
       } else {
         const uint4* kr = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.k_idx) +
-                                                         (ko + j) * D + h * 64);
+                                                         krow * D + h * 64);
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
           const uint4 u = __ldg(kr + v);

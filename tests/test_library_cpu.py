@@ -121,6 +121,28 @@ def test_host_validation_rejects_bad_arguments():
     assert L.dsa_topk(None, ctypes.byref(rg), A, 8, 0, 1, A, 4, null, null) == dsa.DSA_ERR_INVALID_ARG
 
 
+def test_paged_cache_descriptor_is_validated():
+    import indexer_top_gated_b200 as dsa
+    L = dsa.lib
+    P = dsa.LayerShape(top_k=4).params()
+    A = 0x10000
+    base = dict(block_table=A, max_pages=4, page_size=128)
+    bad = (dict(page_size=100), dict(page_size=64), dict(page_size=384), dict(max_pages=1),
+           dict(total_kv=1000))
+    for b in bad:
+        rg = dsa.Ragged(1, 0x1000, 0x2000, 8, 500, 8, 1024, None, 0, 0)
+        for k, v in dict(base, **b).items():
+            setattr(rg, k, v)
+        rc = L.dsa_sparse_attn_gated(ctypes.byref(P), ctypes.byref(rg), A, A, A, A, 4, 0, 1,
+                                     None, A, None, None, None)
+        assert rc == dsa.DSA_ERR_INVALID_ARG, (b, rc)
+    # a valid descriptor passes the host checks (workspace sizing is host-only)
+    rg = dsa.Ragged(1, 0x1000, 0x2000, 8, 500, 8, 1024, A, 4, 128)
+    mn, rec = dsa.dsa_workspace_size(dsa.LayerShape(top_k=4), rg)
+    assert 0 < mn <= rec
+    assert L.dsa_version() == 101
+
+
 def test_workspace_size_is_host_only():
     import indexer_top_gated_b200 as dsa
     shape = dsa.LayerShape(top_k=2048)
