@@ -65,6 +65,8 @@ def lib():
         L.oracle_layer_rows.argtypes = [ctypes.POINTER(Problem), vp, vp, vp, vp, vp, vp, vp, vp, i64,
                                         i32, vp, vp, vp]
         L.oracle_layer_rows.restype = None
+        L.oracle_block_topk_row.argtypes = [vp, i64, i32, i32, vp]
+        L.oracle_block_topk_row.restype = i32
         L.oracle_gate_mix.argtypes = [vp, vp, vp, i64, vp]
         L.oracle_gate_mix.restype = None
         L.oracle_hardware_threads.argtypes = []
@@ -148,6 +150,15 @@ class Oracle:
                                 _ptr(self.a["v"]), _ptr(self.a.get("gate")), rows.ctypes.data, nr,
                                 nthreads, idx.ctypes.data, out.ctypes.data, lse.ctypes.data)
         return idx, out, lse
+
+
+def block_topk_row(s: np.ndarray, B: int, Kb: int) -> np.ndarray:
+    """Oracle block-granular Top-K of one score row: positions of the Kb blocks (of B
+    positions) with the largest maxima, ascending, -1 up to Kb * B."""
+    s = np.ascontiguousarray(s, dtype=np.float64)
+    idx = np.empty(Kb * B, dtype=np.int32)
+    lib().oracle_block_topk_row(s.ctypes.data, len(s), B, Kb, idx.ctypes.data)
+    return idx
 
 
 def gate_mix(o: np.ndarray, gate_bits: np.ndarray, o2_bits: np.ndarray) -> np.ndarray:

@@ -25,6 +25,10 @@
  *   2. Top-K: the K largest scores of the row, ties to the lower position; all
  *      positions when the row has <= K ([HSA] same section, step 2; [ITK]
  *      "Introducing Indexed Top-K Sparse Attention", Top-K Selection Stage).
+ *      Block granularity ([HSA] same section, steps 1-2: positions "or blocks"): the
+ *      score of block m (positions mB .. mB+B-1 up to p) is the largest score of its
+ *      positions, the K blocks with the largest scores are kept (ties to the lower block;
+ *      all blocks when the row has <= K), and their positions are the selection.
  *   3. exact softmax attention over the selected rows only, scale 1/sqrt(d)
  *      ([HSA] same section, step 3 and its pseudocode; [SAE] "5. Abstract
  *       Implementation Sketch of Indexer + Top-K").
@@ -148,6 +152,35 @@ int32_t oracle_topk_row(const double* s, int64_t n, int32_t K, int32_t* idx) {
   std::sort(chosen.begin(), chosen.end());
   for (int32_t i = 0; i < K; ++i) idx[i] = i < take ? chosen[(size_t)i] : -1;
   return (int32_t)take;
+}
+
+/* Step 2 at block granularity: s[0..n) one row's scores, blocks of B positions (the last
+ * one partial), Kb blocks kept.  idx receives the selected positions in ascending order,
+ * then -1 up to Kb * B.  Returns the number of positions selected. */
+int32_t oracle_block_topk_row(const double* s, int64_t n, int32_t B, int32_t Kb, int32_t* idx) {
+  const int64_t nb = (n + B - 1) / B;
+  std::vector<std::pair<double, int64_t>> blocks((size_t)nb);
+  for (int64_t m = 0; m < nb; ++m) {
+    double best = s[m * B];
+    for (int64_t j = m * B + 1; j < n && j < (m + 1) * B; ++j)
+      if (s[j] > best) best = s[j];
+    blocks[(size_t)m] = {best == 0.0 ? 0.0 : best, m};  // -0.0 counts as +0.0
+  }
+  std::sort(blocks.begin(), blocks.end(), [](const std::pair<double, int64_t>& x,
+                                             const std::pair<double, int64_t>& y) {
+    if (x.first != y.first) return x.first > y.first;
+    return x.second < y.second;
+  });
+  const int64_t take = nb < (int64_t)Kb ? nb : (int64_t)Kb;
+  std::vector<int64_t> chosen((size_t)take);
+  for (int64_t i = 0; i < take; ++i) chosen[(size_t)i] = blocks[(size_t)i].second;
+  std::sort(chosen.begin(), chosen.end());
+  int32_t w = 0;
+  for (int64_t m : chosen)
+    for (int64_t j = m * B; j < n && j < (m + 1) * B; ++j) idx[w++] = (int32_t)j;
+  const int32_t total = w;
+  while (w < Kb * B) idx[w++] = -1;
+  return total;
 }
 
 /* Steps 3-4: gated exact softmax attention of packed query row r over the cache rows

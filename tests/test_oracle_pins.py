@@ -189,6 +189,35 @@ def test_topk_negative_zero_ties_with_zero():
     np.testing.assert_array_equal(O.topk_row(s, 1), [0])
 
 
+def test_block_topk_pins():
+    """Block granularity: B = 1 is the position Top-K; scores constant within blocks (and
+    distinct across them) give the position Top-K of K = Kb * B; a single planted maximum
+    selects its block; a partial last block is cut at the row's end; Kb covering every
+    block selects every position."""
+    rng = np.random.default_rng(21)
+    for n in (1, 7, 64, 257):
+        s = rng.integers(-3, 4, size=n).astype(np.float64)
+        for K in (1, 3, 50):
+            np.testing.assert_array_equal(O.block_topk_row(s, 1, K), O.topk_row(s, K))
+    for B, Kb, nb in ((4, 3, 10), (32, 2, 5), (8, 5, 5)):
+        vals = rng.permutation(nb).astype(np.float64) - 2.5
+        s = np.repeat(vals, B)
+        np.testing.assert_array_equal(O.block_topk_row(s, B, Kb), O.topk_row(s, Kb * B))
+    s = np.zeros(300)
+    s[137] = 5.0
+    got = O.block_topk_row(s, 32, 1)
+    np.testing.assert_array_equal(got, np.arange(128, 160))
+    # ties: the lower blocks win; the last block (positions 288..299) is partial
+    got = O.block_topk_row(np.zeros(300), 32, 10)
+    np.testing.assert_array_equal(got[:300], np.arange(300))
+    assert (got[300:] == -1).all()
+    s = rng.normal(size=100)
+    s[99] = 50.0
+    got = O.block_topk_row(s, 16, 1)
+    np.testing.assert_array_equal(got[:4], [96, 97, 98, 99])
+    assert (got[4:] == -1).all()
+
+
 def test_topk_short_row_takes_everything():
     idx = O.topk_row(np.array([3.0, 1.0, 2.0]), 5)
     np.testing.assert_array_equal(idx, [0, 1, 2, -1, -1])
