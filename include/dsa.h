@@ -189,6 +189,36 @@ dsa_status dsa_index_topk(const dsa_params* params, const dsa_ragged* ragged, co
                           size_t ws_bytes, void* stream);
 
 /*
+ * Steps 1-2 at block granularity ([HSA] "Indexer + Top-K: How Fine-Grained Sparse
+ * Attention Works", steps 1-2: score and keep positions "or blocks").  The pages define no
+ * block score; here a block of `block` consecutive positions scores as the largest indexer
+ * score among its positions (up to p), the top_k blocks with the largest scores are kept
+ * (ties to the lower block; all blocks when the row has no more than top_k), and the row's
+ * selection is their positions.
+ *   params->top_k  number of blocks kept per row (Kb)
+ *   block          positions per block: a power of two, 32 .. 4096
+ *   idx    int32 [q_count, ld_idx], ld_idx >= Kb * block: the selected positions of row i
+ *          ascending, then -1 up to Kb * block.  Pass it to dsa_sparse_attn_gated with a
+ *          params copy whose top_k is Kb * block.
+ *   cnt    int32 [q_count] or NULL: positions selected per row.
+ *   workspace device, 256-byte aligned, ws_bytes >= the minimum of
+ *          dsa_index_topk_blocks_workspace_size (one row's 32-position maxima, block scores
+ *          and block list); rows are processed in passes of as many as it holds.
+ * The indexer stores one value per 32 positions (the maximum) instead of 32 scores, so the
+ * Top-K works on n / block entries per row.  Every other argument as dsa_index_scores.
+ * Returns DSA_ERR_INVALID_ARG for a block size outside the range or ld_idx < Kb * block.
+ */
+dsa_status dsa_index_topk_blocks_workspace_size(const dsa_params* params,
+                                                const dsa_ragged* ragged, int32_t block,
+                                                int64_t q_count, size_t* min_bytes,
+                                                size_t* rec_bytes);
+dsa_status dsa_index_topk_blocks(const dsa_params* params, const dsa_ragged* ragged,
+                                 const void* q_idx, const void* k_idx, const float* w,
+                                 int32_t block, int64_t q_begin, int64_t q_count, int32_t* idx,
+                                 int64_t ld_idx, int32_t* cnt, void* workspace, size_t ws_bytes,
+                                 void* stream);
+
+/*
  * Steps 3-4 - exact softmax attention over the selected rows with the sigmoid output
  * gate fused in ([HSA] steps 3-4 and pseudocode; [SAE] section 5; [GSA] section 2).
  *   q        bf16 [total_q, Hq, d]

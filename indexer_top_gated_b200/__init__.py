@@ -55,7 +55,7 @@ EXPORTS = [
     "dsa_sparse_attn_gated", "dsa_workspace_size", "dsa_prefill", "dsa_decode",
     "dsa_device_status", "dsa_launch_count", "dsa_stage_timing", "dsa_stage_times",
     "dsa_decode_noalloc", "dsa_index_topk", "dsa_index_topk_workspace_size",
-    "dsa_sparse_attn_gated_mix",
+    "dsa_sparse_attn_gated_mix", "dsa_index_topk_blocks", "dsa_index_topk_blocks_workspace_size",
 ]
 
 
@@ -71,6 +71,9 @@ def _load():
     L.dsa_index_scores.argtypes = [PP, RP, vp, vp, vp, i64, i64, vp, i64, vp]
     L.dsa_topk.argtypes = [PP, RP, vp, i64, i64, i64, vp, i64, vp, vp]
     L.dsa_sparse_attn_gated.argtypes = [PP, RP, vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, vp, vp]
+    L.dsa_index_topk_blocks_workspace_size.argtypes = [PP, RP, i32, i64, ctypes.POINTER(sz),
+                                                       ctypes.POINTER(sz)]
+    L.dsa_index_topk_blocks.argtypes = [PP, RP, vp, vp, vp, i32, i64, i64, vp, i64, vp, vp, sz, vp]
     L.dsa_sparse_attn_gated_mix.argtypes = [PP, RP, vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, vp,
                                             vp, vp]
     L.dsa_workspace_size.argtypes = [PP, RP, ctypes.c_int, ctypes.POINTER(sz), ctypes.POINTER(sz)]
@@ -176,6 +179,29 @@ def dsa_sparse_attn_gated(shape: LayerShape, rg: Ragged, q, k_cache, v_cache, id
                                      _ptr(v_cache), _ptr(idx), ld_idx, q_begin, q_count,
                                      _ptr(gate), _ptr(out), _ptr(lse), _ptr(err_count),
                                      _stream(stream)), "dsa_sparse_attn_gated")
+
+
+def dsa_index_topk_blocks_workspace_size(shape: LayerShape, rg: Ragged, block: int,
+                                         q_count: int):
+    p = shape.params()
+    mn, rec = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check(lib.dsa_index_topk_blocks_workspace_size(ctypes.byref(p), ctypes.byref(rg), block,
+                                                    q_count, ctypes.byref(mn), ctypes.byref(rec)),
+           "dsa_index_topk_blocks_workspace_size")
+    return mn.value, rec.value
+
+
+def dsa_index_topk_blocks(shape: LayerShape, rg: Ragged, q_idx, k_idx, w, block: int, q_begin: int,
+                          q_count: int, idx, ld_idx: int, cnt=None, workspace=None, ws_bytes=None,
+                          stream=None):
+    """top_k of `shape` counts blocks; idx receives positions (ld_idx >= top_k * block)."""
+    p = shape.params()
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.dsa_index_topk_blocks(ctypes.byref(p), ctypes.byref(rg), _ptr(q_idx), _ptr(k_idx),
+                                     _ptr(w), block, q_begin, q_count, _ptr(idx), ld_idx,
+                                     _ptr(cnt), _ptr(workspace), ws_bytes, _stream(stream)),
+           "dsa_index_topk_blocks")
 
 
 def dsa_sparse_attn_gated_mix(shape: LayerShape, rg: Ragged, q, k_cache, v_cache, idx, ld_idx: int,

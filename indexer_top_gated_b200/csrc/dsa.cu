@@ -101,15 +101,19 @@ dsa_status device_setup(DeviceState** out) {
     d.max_smem = (size_t)smem_optin;
     const size_t idx_max = idx_smem_bytes(4, 64, false);
     cudaError_t e = cudaSuccess;
-    e = e ? e : allow_smem(idx_scores_kernel<64, false, false>, idx_max);
-    e = e ? e : allow_smem(idx_scores_kernel<16, false, false>, idx_max);
-    e = e ? e : allow_smem(idx_scores_kernel<64, true, false>, idx_max);
-    e = e ? e : allow_smem(idx_scores_kernel<16, true, false>, idx_max);
+    e = e ? e : allow_smem(idx_scores_kernel<64, false, kIdxScores>, idx_max);
+    e = e ? e : allow_smem(idx_scores_kernel<16, false, kIdxScores>, idx_max);
+    e = e ? e : allow_smem(idx_scores_kernel<64, true, kIdxScores>, idx_max);
+    e = e ? e : allow_smem(idx_scores_kernel<16, true, kIdxScores>, idx_max);
     const size_t cand_max = idx_smem_bytes(4, 64, false, true);
-    e = e ? e : allow_smem(idx_scores_kernel<64, false, true>, cand_max);
-    e = e ? e : allow_smem(idx_scores_kernel<16, false, true>, cand_max);
-    e = e ? e : allow_smem(idx_scores_kernel<64, true, true>, cand_max);
-    e = e ? e : allow_smem(idx_scores_kernel<16, true, true>, cand_max);
+    e = e ? e : allow_smem(idx_scores_kernel<64, false, kIdxCand>, cand_max);
+    e = e ? e : allow_smem(idx_scores_kernel<16, false, kIdxCand>, cand_max);
+    e = e ? e : allow_smem(idx_scores_kernel<64, true, kIdxCand>, cand_max);
+    e = e ? e : allow_smem(idx_scores_kernel<16, true, kIdxCand>, cand_max);
+    e = e ? e : allow_smem(idx_scores_kernel<64, false, kIdxBlockMax>, cand_max);
+    e = e ? e : allow_smem(idx_scores_kernel<16, false, kIdxBlockMax>, cand_max);
+    e = e ? e : allow_smem(idx_scores_kernel<64, true, kIdxBlockMax>, cand_max);
+    e = e ? e : allow_smem(idx_scores_kernel<16, true, kIdxBlockMax>, cand_max);
     e = e ? e : allow_smem(topk_kernel<kTopkScores>, topk_smem_bytes(0));
     e = e ? e : allow_smem(topk_fused_kernel, topk_fused_smem_bytes(kTopkFastCap, kTopkFusedMaxN));
     e = e ? e : allow_smem(topk_kernel<kTopkFallback>, topk_smem_bytes(0));
@@ -231,6 +235,7 @@ struct IdxVariant {
   float2* cand = nullptr;
   int cap = 0;
   int32_t* cand_cnt = nullptr;
+  bool bmax = false;               // 32-key maxima instead of scores (scores = ld-strided rows)
 };
 
 dsa_status launch_index_scores(const DeviceState& dev, const dsa_params* P, const dsa_ragged* R,
@@ -240,6 +245,7 @@ dsa_status launch_index_scores(const DeviceState& dev, const dsa_params* P, cons
   if (q_count == 0 || R->total_kv == 0) return DSA_OK;
   const bool fp8 = P->idx_dtype == DSA_FP8_E4M3;
   const bool cand = var.thr != nullptr;
+  const int mode = cand ? kIdxCand : var.bmax ? kIdxBlockMax : kIdxScores;
   CUtensorMap mq, mk;
   DSA_TRY(make_idx_map(&mq, q_idx, R->total_q, P->n_idx_heads, fp8, bq));
   if (var.shift)
@@ -276,20 +282,24 @@ dsa_status launch_index_scores(const DeviceState& dev, const dsa_params* P, cons
   a.cand = var.cand;
   a.cap = var.cap;
   a.cand_cnt = var.cand_cnt;
-  const size_t smem = idx_smem_bytes(P->n_idx_heads, bq, fp8, cand);
+  const size_t smem = idx_smem_bytes(P->n_idx_heads, bq, fp8, mode != kIdxScores);
   dim3 grid((unsigned)a.n_tiles, (unsigned)ysplit);
   StageScope scope(0, stream);
-#define DSA_IDX_CASE(BQ, F8, C)                                                      \
-  if (bq == BQ && fp8 == F8 && cand == C)                                            \
-    idx_scores_kernel<BQ, F8, C><<<grid, kIdxThreads, smem, stream>>>(mq, mk, a);
-  DSA_IDX_CASE(64, false, false)
-  DSA_IDX_CASE(64, true, false)
-  DSA_IDX_CASE(16, false, false)
-  DSA_IDX_CASE(16, true, false)
-  DSA_IDX_CASE(64, false, true)
-  DSA_IDX_CASE(64, true, true)
-  DSA_IDX_CASE(16, false, true)
-  DSA_IDX_CASE(16, true, true)
+#define DSA_IDX_CASE(BQ, F8, M)                                                      \
+  if (bq == BQ && fp8 == F8 && mode == M)                                            \
+    idx_scores_kernel<BQ, F8, M><<<grid, kIdxThreads, smem, stream>>>(mq, mk, a);
+  DSA_IDX_CASE(64, false, kIdxScores)
+  DSA_IDX_CASE(64, true, kIdxScores)
+  DSA_IDX_CASE(16, false, kIdxScores)
+  DSA_IDX_CASE(16, true, kIdxScores)
+  DSA_IDX_CASE(64, false, kIdxCand)
+  DSA_IDX_CASE(64, true, kIdxCand)
+  DSA_IDX_CASE(16, false, kIdxCand)
+  DSA_IDX_CASE(16, true, kIdxCand)
+  DSA_IDX_CASE(64, false, kIdxBlockMax)
+  DSA_IDX_CASE(64, true, kIdxBlockMax)
+  DSA_IDX_CASE(16, false, kIdxBlockMax)
+  DSA_IDX_CASE(16, true, kIdxBlockMax)
 #undef DSA_IDX_CASE
   ++t_launches;
   return launch_status("idx_scores_kernel");
@@ -297,7 +307,7 @@ dsa_status launch_index_scores(const DeviceState& dev, const dsa_params* P, cons
 
 dsa_status launch_topk(const dsa_params* P, const dsa_ragged* R, const float* scores, int64_t ld,
                        int64_t q_begin, int64_t q_count, int32_t* idx, int64_t ld_idx,
-                       int32_t* cnt, cudaStream_t stream) {
+                       int32_t* cnt, cudaStream_t stream, int blk_shift = 0) {
   if (q_count == 0) return DSA_OK;
   TopkArgs a;
   std::memset(&a, 0, sizeof(a));
@@ -312,6 +322,7 @@ dsa_status launch_topk(const dsa_params* P, const dsa_ragged* R, const float* sc
   a.idx = idx;
   a.ld_idx = ld_idx;
   a.cnt = cnt;
+  a.blk_shift = blk_shift;
   const size_t smem = topk_smem_bytes(R->max_kv_len);
   StageScope scope(1, stream);
   topk_kernel<kTopkScores><<<(unsigned)q_count, kTopkThreads, smem, stream>>>(a);
@@ -810,6 +821,105 @@ dsa_status dsa_index_topk(const dsa_params* P, const dsa_ragged* R, const void* 
     const int64_t n = std::min<int64_t>(rows, q_begin + q_count - s0);
     DSA_TRY(fused_pass(*dev, P, R, q_idx, k_idx, w, s0, n, idx + (s0 - q_begin) * ld_idx, ld_idx,
                        cnt ? cnt + (s0 - q_begin) : nullptr, g, f, st));
+  }
+  return DSA_OK;
+}
+
+// ---------------------------------------------------------------- block granularity
+namespace dsa {
+namespace {
+struct BlockGeom {
+  int bshift;
+  int64_t ld32, ldb, row_bytes;
+};
+bool block_geom(const dsa_params* P, const dsa_ragged* R, int block, BlockGeom* g) {
+  if (block < 32 || block > 4096 || (block & (block - 1)) != 0) return false;
+  g->bshift = 0;
+  while ((1 << g->bshift) < block) ++g->bshift;
+  const int64_t n = std::max(R->max_kv_len, 1);
+  g->ld32 = round_up((n + 31) / 32, 32);
+  g->ldb = block > 32 ? round_up((n + block - 1) / block, 32) : 0;
+  g->row_bytes = (g->ld32 + g->ldb) * 4 + round_up(P->top_k, 4) * 4;
+  return true;
+}
+}  // namespace
+}  // namespace dsa
+
+dsa_status dsa_index_topk_blocks_workspace_size(const dsa_params* P, const dsa_ragged* R,
+                                                int32_t block, int64_t q_count, size_t* min_bytes,
+                                                size_t* rec_bytes) {
+  DSA_TRY(check_common(P, R));
+  DSA_TRY(check_indexer(P));
+  if (q_count < 0) return DSA_ERR_INVALID_ARG;
+  BlockGeom g;
+  if (!block_geom(P, R, block, &g)) return DSA_ERR_INVALID_ARG;
+  if (min_bytes) *min_bytes = (size_t)(g.row_bytes + 3 * 256);
+  if (rec_bytes) *rec_bytes = (size_t)(std::max<int64_t>(1, q_count) * g.row_bytes + 3 * 256);
+  return DSA_OK;
+}
+
+dsa_status dsa_index_topk_blocks(const dsa_params* P, const dsa_ragged* R, const void* q_idx,
+                                 const void* k_idx, const float* w, int32_t block,
+                                 int64_t q_begin, int64_t q_count, int32_t* idx, int64_t ld_idx,
+                                 int32_t* cnt, void* workspace, size_t ws_bytes, void* stream) {
+  DSA_TRY(check_common(P, R));
+  DSA_TRY(check_indexer(P));
+  BlockGeom g;
+  if (!block_geom(P, R, block, &g)) return DSA_ERR_INVALID_ARG;
+  if (!q_idx || !k_idx || !w || !idx) return DSA_ERR_INVALID_ARG;
+  if (q_begin < 0 || q_count < 0 || q_begin + q_count > R->total_q) return DSA_ERR_INVALID_ARG;
+  if (ld_idx < (int64_t)P->top_k * block) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx)) return DSA_ERR_INVALID_ARG;
+  if (q_count > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255)) return DSA_ERR_WORKSPACE;
+  const int64_t rows = std::min<int64_t>(q_count, ((int64_t)ws_bytes - 3 * 256) / g.row_bytes);
+  if (((int64_t)ws_bytes - 3 * 256) / g.row_bytes < 1) return DSA_ERR_WORKSPACE;
+  if (q_count == 0) return DSA_OK;
+  DeviceState* dev = nullptr;
+  DSA_TRY(device_setup(&dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* p = static_cast<char*>(workspace);
+  float* s32 = reinterpret_cast<float*>(p);
+  p += round_up(rows * g.ld32 * 4, 256);
+  float* sb = reinterpret_cast<float*>(p);
+  p += round_up(rows * g.ldb * 4, 256);
+  int32_t* blk = reinterpret_cast<int32_t*>(p);
+  const int bq = R->max_q_len <= 16 ? 16 : 64;
+  for (int64_t s0 = q_begin; s0 < q_begin + q_count; s0 += rows) {
+    const int64_t n = std::min<int64_t>(rows, q_begin + q_count - s0);
+    IdxVariant v;
+    v.bmax = true;
+    DSA_TRY(launch_index_scores(*dev, P, R, q_idx, k_idx, w, s0, n, s32, g.ld32, bq, st, v));
+    BlockArgs ba;
+    std::memset(&ba, 0, sizeof(ba));
+    ba.q_offsets = R->q_offsets;
+    ba.kv_offsets = R->kv_offsets;
+    ba.batch = R->batch;
+    ba.q_begin = s0;
+    ba.bshift = g.bshift;
+    if (block > 32) {
+      ba.in = s32;
+      ba.ld_in = g.ld32;
+      ba.out = sb;
+      ba.ld_out = g.ldb;
+      StageScope scope(1, st);
+      block_max_kernel<<<(unsigned)n, 256, 0, st>>>(ba);
+      ++t_launches;
+      DSA_TRY(launch_status("block_max_kernel"));
+    }
+    DSA_TRY(launch_topk(P, R, block > 32 ? sb : s32, block > 32 ? g.ldb : g.ld32, s0, n, blk,
+                        P->top_k, nullptr, st, g.bshift));
+    ba.blk = blk;
+    ba.Kb = P->top_k;
+    ba.idx = idx + (s0 - q_begin) * ld_idx;
+    ba.ld_idx = ld_idx;
+    ba.cnt = cnt ? cnt + (s0 - q_begin) : nullptr;
+    {
+      StageScope scope(1, st);
+      block_expand_kernel<<<(unsigned)n, 256, 0, st>>>(ba);
+      ++t_launches;
+      DSA_TRY(launch_status("block_expand_kernel"));
+    }
   }
   return DSA_OK;
 }

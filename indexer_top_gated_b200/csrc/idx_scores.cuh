@@ -34,6 +34,9 @@
 //    in shared memory and reads it back transposed: each lane then compares 16 keys of
 //    one row, counts its hits with one popcount and stores them in a short loop.  The
 //    2 KiB per warp come out of the key ring, which has 2 stages in this variant.
+//  - 32-key maxima (BMAX), for block-granular selection: through the same transposed
+//    block, each row gets the maximum of its scores over every 32 keys it may see (one
+//    value per 32 positions instead of 32).
 #pragma once
 
 #include "common.cuh"
@@ -99,6 +102,7 @@ __host__ __device__ inline int idx_tmem_cols(int n_heads, int bq) {
 // the 512 columns asks for enough shared memory that CTAs sharing an SM can never
 // oversubscribe TMEM (an allocation that cannot be met would block).
 __host__ inline size_t idx_smem_bytes(int n_heads, int bq, bool fp8, bool cand = false) {
+  // cand: the variants with the shared score block (candidates, 32-key maxima)
   size_t row = fp8 ? 64 : 128;
   size_t q = (size_t)n_heads * bq * row;
   size_t k = (size_t)(cand ? kIdxCandStages : kIdxStages) * n_heads * kIdxKeyTile * row;
@@ -111,12 +115,18 @@ __host__ inline size_t idx_smem_bytes(int n_heads, int bq, bool fp8, bool cand =
   return bytes;
 }
 
-template <int BQ, bool FP8, bool CAND>
+// Variants of the epilogue: every score, candidates only, or the maximum of each 32 keys.
+enum IdxMode { kIdxScores = 0, kIdxCand = 1, kIdxBlockMax = 2 };
+
+template <int BQ, bool FP8, int MODE>
 __global__ void __launch_bounds__(kIdxThreads, 1)
     idx_scores_kernel(const __grid_constant__ CUtensorMap tmap_q,
                       const __grid_constant__ CUtensorMap tmap_k, IdxArgs a) {
   using Geo = IdxGeom<FP8>;
-  constexpr int ST = CAND ? kIdxCandStages : kIdxStages;
+  constexpr bool CAND = MODE == kIdxCand;
+  constexpr bool BMAX = MODE == kIdxBlockMax;
+  constexpr bool TILE = CAND || BMAX;  // the epilogue goes through the shared score block
+  constexpr int ST = TILE ? kIdxCandStages : kIdxStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -131,7 +141,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   uint64_t* tfull = bars + 2 * ST;  // [2]
   uint64_t* tempty = tfull + 2;     // [2]
   uint64_t* qfull = tempty + 2;     // [1]
-  float* tiles = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);  // CAND
+  float* tiles = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);  // TILE
   __shared__ uint32_t s_tmem;
   __shared__ int s_bfirst, s_blast;
   __shared__ volatile int s_abort;
@@ -334,7 +344,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           // heads in groups of HPB (two, or one in the candidate variant, which needs the
           // registers): HPB TMEM loads in flight, then their ReLU-weighted sum (the
           // accumulation order over heads is 0, 1, 2, 3 either way)
-          constexpr int HPB = CAND ? 1 : 2;
+          constexpr int HPB = TILE ? 1 : 2;
           float acc[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) acc[c] = 0.f;
@@ -378,6 +388,36 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           // sequence and sees the whole key tile, so no per-element predicate is needed.
           const bool inside = c0 >= c_lo && c0 + 16 <= c_hi &&
                               kt * kIdxKeyTile + (kIdxKeyTile - 1) <= ((p0 + c0) >> a.shift);
+          if (BMAX) {
+            // the maximum of each row over this warp's 32 keys (those the row may see)
+#pragma unroll
+            for (int c = 0; c < 16; ++c) tile[c * kIdxTileStride + lane] = acc[c];
+            __syncwarp();
+            const int rr = lane & 15, kh = (lane >> 4) * 16;
+            const float* trow = tile + rr * kIdxTileStride + kh;
+            const int cc = c0 + rr;
+            int k_lim = 16;
+            if (!inside) {
+              const int pr = (p0 + cc) >> a.shift;
+              const int lim = pr - (kt * kIdxKeyTile + quad * 32 + kh) + 1;
+              k_lim = (cc < c_lo || cc >= c_hi || lim <= 0) ? 0 : lim >= 16 ? 16 : lim;
+            }
+            float mx = -INFINITY;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float4 x = *reinterpret_cast<const float4*>(trow + 4 * q);
+              if (4 * q < k_lim) mx = fmaxf(mx, x.x);
+              if (4 * q + 1 < k_lim) mx = fmaxf(mx, x.y);
+              if (4 * q + 2 < k_lim) mx = fmaxf(mx, x.z);
+              if (4 * q + 3 < k_lim) mx = fmaxf(mx, x.w);
+            }
+            mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 16));
+            const int seen = __shfl_xor_sync(0xFFFFFFFFu, k_lim, 16) + k_lim;
+            if (lane < 16 && seen > 0)
+              a.scores[(int64_t)(row0 + cc) * a.ld + kt * 4 + quad] = mx;
+            __syncwarp();  // the block is read before the next chunk overwrites it
+            continue;
+          }
           if (CAND) {
             // keep the scores >= the row's threshold (float order; -0.0 == +0.0)
 #pragma unroll

@@ -89,6 +89,7 @@ struct TopkArgs {
   int cap;
   const int32_t* cand_cnt;  // [q_count, 4] per segment
   int32_t* fb_list;         // [1 + q_count]: count, then rows (within the launch) to redo
+  int blk_shift;            // rows of block scores: n = (p >> blk_shift) + 1 entries
   int bm_words;             // words of each position bitmap (topk_fused_bm_words)
   // fallback: recompute a row's scores on CUDA cores (same formula as the indexer)
   const void* q_idx;
@@ -792,7 +793,7 @@ DSA_DEV int64_t topk_row_len(const TopkArgs& a, int64_t r, int* b_out) {
   const int64_t L = (int64_t)__ldg(a.kv_offsets + b + 1) - __ldg(a.kv_offsets + b);
   const int64_t p = L - (qn - qo) + (r - qo);
   *b_out = b;
-  return p + 1 > 0 ? p + 1 : 0;
+  return p >= 0 ? (p >> a.blk_shift) + 1 : 0;
 }
 
 template <int MODE>
@@ -865,6 +866,79 @@ __global__ void __launch_bounds__(kTopkThreads, 3) topk_fused_kernel(TopkArgs a)
     return;
   }
   if (tid == 0 && a.cnt) a.cnt[i] = K;
+}
+
+// ---------------------------------------------------------------- block granularity
+// Scores of blocks of 2^bshift positions from the indexer's 32-key maxima: out[row][m] =
+// max of in[row][m G .. m G + G - 1] (G = 2^bshift / 32) over the row's n32 = p/32 + 1
+// entries.  One CTA of 256 threads per row.
+struct BlockArgs {
+  const int32_t* q_offsets;
+  const int32_t* kv_offsets;
+  int batch;
+  int64_t q_begin;
+  const float* in;
+  int64_t ld_in;
+  float* out;
+  int64_t ld_out;
+  int bshift;
+  // expansion
+  const int32_t* blk;  // [rows, Kb] selected blocks, ascending, -1 padded
+  int Kb;
+  int32_t* idx;        // [rows, ld_idx] positions
+  int64_t ld_idx;
+  int32_t* cnt;        // [rows] positions selected, or nullptr
+};
+
+DSA_DEV int64_t block_row_p(const BlockArgs& a, int64_t r) {
+  const int b = seq_of_row(a.q_offsets, a.batch, r);
+  const int64_t qo = __ldg(a.q_offsets + b), qn = __ldg(a.q_offsets + b + 1);
+  const int64_t L = (int64_t)__ldg(a.kv_offsets + b + 1) - __ldg(a.kv_offsets + b);
+  return L - (qn - qo) + (r - qo);
+}
+
+__global__ void __launch_bounds__(256) block_max_kernel(BlockArgs a) {
+  const int64_t i = blockIdx.x;
+  const int64_t p = block_row_p(a, a.q_begin + i);
+  if (p < 0) return;
+  const int64_t n32 = (p >> 5) + 1, nb = (p >> a.bshift) + 1;
+  const int G = 1 << (a.bshift - 5);
+  const float* in = a.in + i * a.ld_in;
+  float* out = a.out + i * a.ld_out;
+  for (int64_t m = threadIdx.x; m < nb; m += blockDim.x) {
+    float mx = -INFINITY;
+    for (int g = 0; g < G; ++g) {
+      const int64_t e = m * G + g;
+      if (e < n32) mx = fmaxf(mx, __ldg(in + e));
+    }
+    out[m] = mx;
+  }
+}
+
+// Positions of the selected blocks, ascending (only the block holding p can be partial and
+// it is the last one selected), then -1 up to Kb << bshift.
+__global__ void __launch_bounds__(256) block_expand_kernel(BlockArgs a) {
+  const int64_t i = blockIdx.x;
+  const int64_t p = block_row_p(a, a.q_begin + i);
+  const int B = 1 << a.bshift;
+  const int32_t* blk = a.blk + i * (int64_t)a.Kb;
+  int32_t* out = a.idx + i * a.ld_idx;
+  __shared__ int s_cnt;
+  if (threadIdx.x == 0) s_cnt = 0;
+  __syncthreads();
+  int mine = 0;
+  for (int e = threadIdx.x; e < a.Kb * B; e += blockDim.x) {
+    const int m = __ldg(blk + e / B);
+    const int64_t j = (int64_t)m * B + (e % B);
+    const bool ok = m >= 0 && j <= p;
+    out[e] = ok ? (int32_t)j : -1;
+    mine += ok;
+  }
+  if (a.cnt) {
+    atomicAdd(&s_cnt, mine);
+    __syncthreads();
+    if (threadIdx.x == 0) a.cnt[i] = s_cnt;
+  }
 }
 
 // One warp per row: a lower bound of the R-th largest of the row's S samples, R = S K / n

@@ -235,3 +235,69 @@ def test_prefill_layer_takes_the_fused_path():
                               w.total_q, dev["gate"], out2)
     torch.cuda.synchronize()
     assert torch.equal(out, out2)
+
+
+# ----------------------------------------------------------------------------- block granularity
+
+BLOCK_CASES = {
+    "b32_k16": dict(q_lens=[1500], kv_lens=[1500], K=16, B=32),
+    "b64_ragged": dict(q_lens=[700, 1, 300, 5], kv_lens=[3000, 4097, 300, 70], K=12, B=64),
+    "b128_k40": dict(q_lens=[2000], kv_lens=[6000], K=40, B=128),
+    "b32_fp8": dict(q_lens=[900], kv_lens=[2000], K=20, B=32, dtype="fp8"),
+}
+
+
+@pytest.mark.parametrize("case", sorted(BLOCK_CASES))
+def test_index_topk_blocks_matches_oracle(case):
+    cfg = dict(BLOCK_CASES[case])
+    B = cfg.pop("B")
+    w = _workload(**cfg)
+    host = S.make_host_inputs(w)
+    dev = _dev(host)
+    shape = dsa.workload_shape(w)
+    rg = _rg(w, dev)
+    Kb = w.top_k
+    ld = Kb * B + 3
+    mn, rec = dsa.dsa_index_topk_blocks_workspace_size(shape, rg, B, w.total_q)
+    idx = torch.full((w.total_q, ld), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(w.total_q, dtype=torch.int32, device="cuda")
+    for ws_bytes in (rec, mn + 5 * (rec - mn) // max(1, w.total_q)):  # one pass, then many
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+        idx.fill_(-7)
+        dsa.dsa_index_topk_blocks(shape, rg, dev["q_idx"], dev["k_idx"], dev["w"], B, 0, w.total_q,
+                                  idx, ld, cnt, ws)
+        torch.cuda.synchronize()
+        got = idx.cpu().numpy()
+        orc = O.Oracle.for_workload(w, host)
+        for r in PT.sample_rows(w, 24, seed=9):
+            ref = O.block_topk_row(orc.index_scores_row(r), B, Kb)
+            np.testing.assert_array_equal(got[r, : Kb * B], ref, err_msg=f"{case} row {r}")
+            assert int(cnt[r]) == int((ref >= 0).sum())
+        assert (got[:, Kb * B:] == -7).all()
+
+
+def test_block_selection_feeds_attention():
+    """Attention over a block selection (top_k = Kb * B positions) matches the oracle."""
+    B, Kb = 64, 6
+    w = _workload([300], [2000], K=Kb)
+    host = S.make_host_inputs(w)
+    dev = _dev(host)
+    shape = dsa.workload_shape(w)
+    rg = _rg(w, dev)
+    _, rec = dsa.dsa_index_topk_blocks_workspace_size(shape, rg, B, w.total_q)
+    ws = torch.empty(rec, dtype=torch.uint8, device="cuda")
+    idx = torch.empty((w.total_q, Kb * B), dtype=torch.int32, device="cuda")
+    dsa.dsa_index_topk_blocks(shape, rg, dev["q_idx"], dev["k_idx"], dev["w"], B, 0, w.total_q,
+                              idx, Kb * B, None, ws)
+    shape_a = dsa.workload_shape(w)
+    shape_a.top_k = Kb * B
+    out = torch.zeros((w.total_q, w.n_q_heads, 128), dtype=torch.bfloat16, device="cuda")
+    dsa.dsa_sparse_attn_gated(shape_a, rg, dev["q"], dev["k"], dev["v"], idx, Kb * B, 0,
+                              w.total_q, dev["gate"], out)
+    torch.cuda.synchronize()
+    got_idx = idx.cpu().numpy()
+    w_a = _workload([300], [2000], K=Kb * B)
+    orc = O.Oracle.for_workload(w_a, host)
+    rows = list(range(0, 300, 37))
+    ref = np.stack([orc.sparse_attn_row(r, got_idx[r])[0] for r in rows])
+    PT.assert_close(PT.bf16_tensor_to_f64(out)[rows], ref, "block attention")

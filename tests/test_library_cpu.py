@@ -143,6 +143,25 @@ def test_paged_cache_descriptor_is_validated():
     assert L.dsa_version() == 101
 
 
+def test_block_selection_arguments():
+    import indexer_top_gated_b200 as dsa
+    L = dsa.lib
+    rg = dsa.Ragged(1, 0x1000, 0x2000, 64, 4096, 64, 4096, None, 0, 0)
+    shape = dsa.LayerShape(top_k=8)
+    mn, rec = dsa.dsa_index_topk_blocks_workspace_size(shape, rg, 64, 64)
+    assert 0 < mn < rec
+    for bad_block in (16, 48, 8192):
+        with pytest.raises(RuntimeError, match="invalid"):
+            dsa.dsa_index_topk_blocks_workspace_size(shape, rg, bad_block, 64)
+    P = shape.params()
+    A = 0x10000
+    # ld_idx must hold Kb * block positions
+    assert L.dsa_index_topk_blocks(ctypes.byref(P), ctypes.byref(rg), A, A, A, 64, 0, 1, A,
+                                   8 * 64 - 1, None, A, rec, None) == dsa.DSA_ERR_INVALID_ARG
+    assert L.dsa_index_topk_blocks(ctypes.byref(P), ctypes.byref(rg), A, A, A, 64, 0, 1, A,
+                                   8 * 64, None, A, mn - 1, None) == dsa.DSA_ERR_WORKSPACE
+
+
 def test_workspace_size_is_host_only():
     import indexer_top_gated_b200 as dsa
     shape = dsa.LayerShape(top_k=2048)
