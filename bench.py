@@ -265,11 +265,20 @@ def run_ours(args, rank, world, local_rank):
         h2d = sum(host[k].numel() * host[k].element_size() for k in names)
         d2h = out.numel() * out.element_size()
 
-        def e2e_step():
-            for k in names:
-                inputs[k].copy_(host[k], non_blocking=True)
-            step()
-            out_host.copy_(out, non_blocking=True)
+        host_io = dict(host, out=out_host)
+        dev_io = dict(inputs, out=out)
+
+        if decode:
+            def e2e_step():
+                for k in names:
+                    inputs[k].copy_(host[k], non_blocking=True)
+                step()
+                out_host.copy_(out, non_blocking=True)
+        else:
+            def e2e_step():
+                # one C-ABI call: uploads overlapped with the computation of earlier row ranges,
+                # output rows copied back as they are done
+                dsa.dsa_prefill_from_host(shape, rg, host_io, dev_io, 0, ws, ws_bytes)
 
         for _ in range(2):
             e2e_step()

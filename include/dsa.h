@@ -284,6 +284,50 @@ dsa_status dsa_prefill(const dsa_params* params, const dsa_ragged* ragged, const
                        const void* v_cache, const void* gate, void* out, int32_t* idx_out,
                        int32_t* err_count, void* workspace, size_t ws_bytes, void* stream);
 
+/* Buffers of one layer call: the ragged offsets and the layer's inputs and output. */
+typedef struct {
+  const int32_t* q_offsets;   /* [batch+1] */
+  const int32_t* kv_offsets;  /* [batch+1] */
+  const void* q_idx;
+  const void* k_idx;
+  const float* w;
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  const void* gate;           /* NULL: no gate */
+  void* out;
+} dsa_layer_buffers;
+
+/*
+ * dsa_prefill from host memory, with the transfers overlapped with the computation: the
+ * packed query rows are split into n_chunks ranges (n_chunks <= 0: up to 16, one per 2048
+ * rows); for each range one copy stream uploads its query-side rows (q_idx, q, gate) and
+ * the cache rows its queries see that are not on the device yet, the caller's stream runs
+ * the layer on the range as soon as they have landed, and a second copy stream brings its
+ * output rows back.
+ *   order  1: ranges in row order (the cache arrives progressively); 2: last range first;
+ *          0: 2 when the batch has at least 256 query rows per sequence on average, else 1.
+ *          (Used when the layer runs per range, see below.)
+ * When the workspace also holds the index rows of every row (K int32 each) next to one pass
+ * of steps 1-2 over all rows (the dsa_workspace_size recommendation does for a prefill whose
+ * steps 1-2 run fused), steps 1-2 run once as soon as q_idx and k_idx have landed, and only
+ * the attention runs per range (in row order); otherwise the whole layer runs per range.
+ *   host  every input and the output in host memory (page-locked memory lets the copies
+ *         run asynchronously and overlap); host->q_offsets / kv_offsets are also read by
+ *         the host to plan the ranges.
+ *   dev   device buffers of the same sizes and layouts (caller-owned; overwritten with the
+ *         inputs, dev->out with the output).  R gives the sizes; its offset pointers are
+ *         replaced by dev's.
+ *   workspace as dsa_prefill.
+ * The call returns once everything is enqueued; `stream` completes after the last output
+ * row is back in host memory.  The device buffers must not be touched by other streams
+ * until then.  Contiguous caches only (DSA_ERR_UNSUPPORTED with a block table).
+ */
+dsa_status dsa_prefill_from_host(const dsa_params* params, const dsa_ragged* ragged,
+                                 const dsa_layer_buffers* host, const dsa_layer_buffers* dev,
+                                 int32_t n_chunks, int32_t order, void* workspace,
+                                 size_t ws_bytes, void* stream);
+
 /*
  * Whole layer for one new token per sequence (every Q_b = 1, so max_q_len must be 1 and
  * total_q = batch).  Same arguments and outputs as dsa_prefill; tiles are sized for a

@@ -50,12 +50,27 @@ class Ragged(ctypes.Structure):
     ]
 
 
+class LayerBuffers(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "q_offsets", "kv_offsets", "q_idx", "k_idx", "w", "q", "k_cache", "v_cache", "gate", "out")]
+
+
+LAYER_BUFFER_KEYS = ("q_offsets", "kv_offsets", "q_idx", "k_idx", "w", "q", "k", "v", "gate", "out")
+
+
+def layer_buffers(t: dict) -> LayerBuffers:
+    """dsa_layer_buffers from a dict of tensors keyed q_offsets, kv_offsets, q_idx, k_idx, w,
+    q, k, v, gate (optional), out."""
+    return LayerBuffers(*[_ptr(t.get(k)) for k in LAYER_BUFFER_KEYS])
+
+
 EXPORTS = [
     "dsa_status_string", "dsa_version", "dsa_index_scores", "dsa_topk",
     "dsa_sparse_attn_gated", "dsa_workspace_size", "dsa_prefill", "dsa_decode",
     "dsa_device_status", "dsa_launch_count", "dsa_stage_timing", "dsa_stage_times",
     "dsa_decode_noalloc", "dsa_index_topk", "dsa_index_topk_workspace_size",
     "dsa_sparse_attn_gated_mix", "dsa_index_topk_blocks", "dsa_index_topk_blocks_workspace_size",
+    "dsa_prefill_from_host",
 ]
 
 
@@ -71,6 +86,8 @@ def _load():
     L.dsa_index_scores.argtypes = [PP, RP, vp, vp, vp, i64, i64, vp, i64, vp]
     L.dsa_topk.argtypes = [PP, RP, vp, i64, i64, i64, vp, i64, vp, vp]
     L.dsa_sparse_attn_gated.argtypes = [PP, RP, vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, vp, vp]
+    LB = ctypes.POINTER(LayerBuffers)
+    L.dsa_prefill_from_host.argtypes = [PP, RP, LB, LB, i32, i32, vp, sz, vp]
     L.dsa_index_topk_blocks_workspace_size.argtypes = [PP, RP, i32, i64, ctypes.POINTER(sz),
                                                        ctypes.POINTER(sz)]
     L.dsa_index_topk_blocks.argtypes = [PP, RP, vp, vp, vp, i32, i64, i64, vp, i64, vp, vp, sz, vp]
@@ -179,6 +196,19 @@ def dsa_sparse_attn_gated(shape: LayerShape, rg: Ragged, q, k_cache, v_cache, id
                                      _ptr(v_cache), _ptr(idx), ld_idx, q_begin, q_count,
                                      _ptr(gate), _ptr(out), _ptr(lse), _ptr(err_count),
                                      _stream(stream)), "dsa_sparse_attn_gated")
+
+
+def dsa_prefill_from_host(shape: LayerShape, rg: Ragged, host: dict, dev: dict, n_chunks: int = 0,
+                          workspace=None, ws_bytes=None, stream=None, order: int = 0):
+    """dsa_prefill with inputs and output in (page-locked) host tensors, copies overlapped
+    with the computation; dev holds the device buffers of the same shapes."""
+    p = shape.params()
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    hb, db = layer_buffers(host), layer_buffers(dev)
+    _check(lib.dsa_prefill_from_host(ctypes.byref(p), ctypes.byref(rg), ctypes.byref(hb),
+                                     ctypes.byref(db), n_chunks, order, _ptr(workspace), ws_bytes,
+                                     _stream(stream)), "dsa_prefill_from_host")
 
 
 def dsa_index_topk_blocks_workspace_size(shape: LayerShape, rg: Ragged, block: int,

@@ -77,6 +77,9 @@ struct DeviceState {
   int* status = nullptr;  // device address of g_status
   int num_sms = 148;
   size_t max_smem = 0;
+  // copy streams of dsa_prefill_from_host (created on first use) and its events
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  std::vector<cudaEvent_t> events;
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -605,7 +608,7 @@ dsa_status run_layer(const dsa_params* P, const dsa_ragged* R, const void* q_idx
                      const void* k_idx, const float* w, const void* q, const void* k,
                      const void* v, const void* gate, void* out, int32_t* idx_out,
                      int32_t* err_count, void* ws, size_t ws_bytes, void* stream_v,
-                     bool decode) {
+                     bool decode, int64_t row0 = 0, int64_t row1 = -1) {
   DSA_TRY(check_common(P, R));
   DSA_TRY(check_indexer(P));
   DSA_TRY(check_attn(P));
@@ -615,7 +618,10 @@ dsa_status run_layer(const dsa_params* P, const dsa_ragged* R, const void* q_idx
     return DSA_ERR_INVALID_ARG;
   if (decode && (R->max_q_len != 1 || R->total_q != R->batch)) return DSA_ERR_INVALID_ARG;
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return DSA_ERR_WORKSPACE;
-  if (R->total_q == 0) return DSA_OK;
+  if (row1 < 0) row1 = R->total_q;
+  if (row0 < 0 || row1 > R->total_q || row0 > row1) return DSA_ERR_INVALID_ARG;
+  if (row0 == row1) return DSA_OK;
+  const int64_t n_rows = row1 - row0;
   const int64_t ld = scores_ld(R);
   const int64_t K = P->top_k;
   const int64_t irow = idx_out ? 0 : round_up(K * 4, 16);
@@ -623,7 +629,7 @@ dsa_status run_layer(const dsa_params* P, const dsa_ragged* R, const void* q_idx
   DeviceState* dev = nullptr;
   DSA_TRY(device_setup(&dev));
   PassPlan plan;
-  if (!plan_passes(R->total_q, ld * 4, irow, (int64_t)ws_bytes, dev->num_sms, &plan))
+  if (!plan_passes(n_rows, ld * 4, irow, (int64_t)ws_bytes, dev->num_sms, &plan))
     return DSA_ERR_WORKSPACE;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
   FusedGeom fg;
@@ -631,15 +637,15 @@ dsa_status run_layer(const dsa_params* P, const dsa_ragged* R, const void* q_idx
     // fused indexer -> Top-K, in passes of as many rows as the workspace holds (with their
     // index rows when the caller keeps none)
     const int64_t rows = std::min<int64_t>(
-        R->total_q, std::max<int64_t>(0, ((int64_t)ws_bytes - fg.fixed_bytes - 256) /
-                                             (fg.row_bytes + irow)));
-    if (rows >= std::min<int64_t>(R->total_q, kFusedMinRows)) {
+        n_rows, std::max<int64_t>(0, ((int64_t)ws_bytes - fg.fixed_bytes - 256) /
+                                          (fg.row_bytes + irow)));
+    if (rows >= std::min<int64_t>(n_rows, kFusedMinRows)) {
       const FusedWs f = fused_carve(fg, ws, rows);
       int32_t* idx_ws = reinterpret_cast<int32_t*>(
           static_cast<char*>(ws) + round_up(fg.fixed_bytes + rows * fg.row_bytes, 256));
       DSA_TRY(fused_prepare(*dev, R, k_idx, fg, f, stream));
-      for (int64_t a0 = 0; a0 < R->total_q; a0 += rows) {
-        const int64_t cnt_a = std::min<int64_t>(rows, R->total_q - a0);
+      for (int64_t a0 = row0; a0 < row1; a0 += rows) {
+        const int64_t cnt_a = std::min<int64_t>(rows, row1 - a0);
         int32_t* idx = idx_out ? idx_out + a0 * K : idx_ws;
         DSA_TRY(fused_pass(*dev, P, R, q_idx, k_idx, w, a0, cnt_a, idx, K, nullptr, fg, f, stream));
         DSA_TRY(launch_attn(*dev, P, R, q, k, v, idx, K, a0, cnt_a, gate, out, nullptr, err_count,
@@ -653,8 +659,8 @@ dsa_status run_layer(const dsa_params* P, const dsa_ragged* R, const void* q_idx
                             : reinterpret_cast<int32_t*>(static_cast<char*>(ws) +
                                                          plan.rows_s * ld * 4);
   const int bq = (decode || R->max_q_len <= 16) ? 16 : 64;
-  for (int64_t a0 = 0; a0 < R->total_q; a0 += plan.rows_a) {
-    const int64_t cnt_a = std::min<int64_t>(plan.rows_a, R->total_q - a0);
+  for (int64_t a0 = row0; a0 < row1; a0 += plan.rows_a) {
+    const int64_t cnt_a = std::min<int64_t>(plan.rows_a, row1 - a0);
     int32_t* idx = idx_out ? idx_out + a0 * K : idx_ws;
     for (int64_t s0 = a0; s0 < a0 + cnt_a; s0 += plan.rows_s) {
       const int64_t cnt_s = std::min<int64_t>(plan.rows_s, a0 + cnt_a - s0);
@@ -663,6 +669,42 @@ dsa_status run_layer(const dsa_params* P, const dsa_ragged* R, const void* q_idx
     }
     DSA_TRY(launch_attn(*dev, P, R, q, k, v, idx, K, a0, cnt_a, gate, out, nullptr, err_count,
                         stream));
+  }
+  return DSA_OK;
+}
+
+// Steps 1-2 alone for rows [a0, a1): index rows into idx (row r at idx + (r - a0) * K), in
+// passes sized to the workspace (fused indexer -> Top-K when dsa_prefill would take it).
+dsa_status run_index(const DeviceState& dev, const dsa_params* P, const dsa_ragged* R,
+                     const void* q_idx, const void* k_idx, const float* w, int64_t a0, int64_t a1,
+                     int32_t* idx, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  const int64_t n_rows = a1 - a0;
+  if (n_rows <= 0) return DSA_OK;
+  const int64_t K = P->top_k;
+  FusedGeom fg;
+  if (fused_wanted(P, R, &fg)) {
+    const int64_t rows = std::min<int64_t>(n_rows, fused_rows(fg, (int64_t)ws_bytes));
+    if (rows >= std::min<int64_t>(n_rows, kFusedMinRows)) {
+      const FusedWs f = fused_carve(fg, ws, rows);
+      DSA_TRY(fused_prepare(dev, R, k_idx, fg, f, stream));
+      for (int64_t s0 = a0; s0 < a1; s0 += rows) {
+        const int64_t n = std::min<int64_t>(rows, a1 - s0);
+        DSA_TRY(fused_pass(dev, P, R, q_idx, k_idx, w, s0, n, idx + (s0 - a0) * K, K, nullptr,
+                           fg, f, stream));
+      }
+      return DSA_OK;
+    }
+  }
+  const int64_t ld = scores_ld(R);
+  int64_t rows_s = std::min<int64_t>((int64_t)ws_bytes / (ld * 4),
+                                     std::max<int64_t>(kScorePassBytes / (ld * 4), 1));
+  if (rows_s < 1) return DSA_ERR_WORKSPACE;
+  float* scores = static_cast<float*>(ws);
+  const int bq = R->max_q_len <= 16 ? 16 : 64;
+  for (int64_t s0 = a0; s0 < a1; s0 += rows_s) {
+    const int64_t n = std::min<int64_t>(rows_s, a1 - s0);
+    DSA_TRY(launch_index_scores(dev, P, R, q_idx, k_idx, w, s0, n, scores, ld, bq, stream));
+    DSA_TRY(launch_topk(P, R, scores, ld, s0, n, idx + (s0 - a0) * K, K, nullptr, stream));
   }
   return DSA_OK;
 }
@@ -921,6 +963,184 @@ dsa_status dsa_index_topk_blocks(const dsa_params* P, const dsa_ragged* R, const
       DSA_TRY(launch_status("block_expand_kernel"));
     }
   }
+  return DSA_OK;
+}
+
+// ---------------------------------------------------------------- host buffers, pipelined
+namespace dsa {
+namespace {
+std::mutex g_copy_mu;
+
+dsa_status copy_streams(DeviceState* d, int n_events) {
+  std::lock_guard<std::mutex> lock(g_copy_mu);
+  if (!d->s_in && cudaStreamCreateWithFlags(&d->s_in, cudaStreamNonBlocking) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  if (!d->s_out && cudaStreamCreateWithFlags(&d->s_out, cudaStreamNonBlocking) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  while ((int)d->events.size() < n_events) {
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return DSA_ERR_CUDA;
+    d->events.push_back(e);
+  }
+  return DSA_OK;
+}
+
+dsa_status h2d(void* dst, const void* src, size_t bytes, cudaStream_t st) {
+  if (!bytes) return DSA_OK;
+  return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, st) == cudaSuccess ? DSA_OK
+                                                                                     : DSA_ERR_CUDA;
+}
+}  // namespace
+}  // namespace dsa
+
+dsa_status dsa_prefill_from_host(const dsa_params* P, const dsa_ragged* R,
+                                 const dsa_layer_buffers* host, const dsa_layer_buffers* dev,
+                                 int32_t n_chunks, int32_t order, void* workspace,
+                                 size_t ws_bytes, void* stream) {
+  DSA_TRY(check_common(P, R));
+  if (!host || !dev) return DSA_ERR_INVALID_ARG;
+  if (R->block_table) return DSA_ERR_UNSUPPORTED;
+  if (!host->q_offsets || !host->kv_offsets || !dev->q_offsets || !dev->kv_offsets ||
+      !host->q_idx || !host->k_idx || !host->w || !host->q || !host->k_cache ||
+      !host->v_cache || !host->out || (dev->gate != nullptr) != (host->gate != nullptr))
+    return DSA_ERR_INVALID_ARG;
+  const int B = R->batch;
+  const int32_t* qo = host->q_offsets;
+  const int32_t* ko = host->kv_offsets;
+  if (qo[0] != 0 || ko[0] != 0 || qo[B] != R->total_q || ko[B] != R->total_kv)
+    return DSA_ERR_INVALID_ARG;
+  for (int b = 0; b < B; ++b)
+    if (qo[b + 1] < qo[b] || ko[b + 1] < ko[b] || qo[b + 1] - qo[b] > ko[b + 1] - ko[b])
+      return DSA_ERR_INVALID_ARG;
+  dsa_ragged Rd = *R;  // the device offsets are the copies made below
+  Rd.q_offsets = dev->q_offsets;
+  Rd.kv_offsets = dev->kv_offsets;
+  const int64_t TQ = R->total_q;
+  if (order < 0 || order > 2) return DSA_ERR_INVALID_ARG;
+  if (n_chunks <= 0) n_chunks = (int32_t)std::max<int64_t>(1, std::min<int64_t>(16, TQ / 2048));
+  // heaviest ranges first for a few long sequences (causal cost grows along the rows; their
+  // cache is small next to the query side); in order otherwise, so that the cache arrives
+  // progressively
+  const bool reverse = order == 2 || (order == 0 && (int64_t)R->batch * 256 <= TQ);
+  n_chunks = (int32_t)std::max<int64_t>(1, std::min<int64_t>(n_chunks, std::max<int64_t>(TQ, 1)));
+  DeviceState* d = nullptr;
+  DSA_TRY(device_setup(&d));
+  DSA_TRY(copy_streams(d, 2 * n_chunks + 3));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaEvent_t ev_start = d->events[0], ev_end = d->events[1];
+  const size_t e_idx = P->idx_dtype == DSA_FP8_E4M3 ? 1 : 2;
+  const size_t idx_row = (size_t)P->n_idx_heads * P->idx_dim * e_idx;
+  const size_t q_row = (size_t)P->n_q_heads * P->head_dim * 2;
+  const size_t kv_row = (size_t)P->n_kv_heads * P->head_dim * 2;
+  const size_t w_bytes = (P->w_row_stride ? (size_t)TQ * P->w_row_stride : P->n_idx_heads) * 4;
+  auto at = [](const void* base, size_t off) {
+    return const_cast<char*>(static_cast<const char*>(base)) + off;
+  };
+  // the device buffers may still be in use by earlier work on the caller's stream
+  if (cudaEventRecord(ev_start, st) != cudaSuccess ||
+      cudaStreamWaitEvent(d->s_in, ev_start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(d->s_out, ev_start, 0) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  DSA_TRY(h2d(at(dev->q_offsets, 0), qo, (size_t)(B + 1) * 4, d->s_in));
+  DSA_TRY(h2d(at(dev->kv_offsets, 0), ko, (size_t)(B + 1) * 4, d->s_in));
+  DSA_TRY(h2d(at(dev->w, 0), host->w, w_bytes, d->s_in));
+  // cache rows the queries of rows [a0, a1) see: for every sequence the range touches, up
+  // to its last query's position (sequences are packed in order, so this grows with a1)
+  auto kv_need_of = [&](int64_t a0, int64_t a1) {
+    int b_lo = (int)(std::upper_bound(qo, qo + B + 1, (int32_t)a0) - qo) - 1;
+    b_lo = std::max(0, std::min(b_lo, B - 1));
+    int64_t need = 0;
+    for (int b = b_lo; b < B && qo[b] < a1; ++b) {
+      const int64_t last = std::min<int64_t>(a1, qo[b + 1]) - 1;
+      if (last < qo[b]) continue;
+      const int64_t p = (ko[b + 1] - ko[b]) - (qo[b + 1] - qo[b]) + (last - qo[b]);
+      need = std::max<int64_t>(need, ko[b] + p + 1);
+    }
+    return need;
+  };
+  // Index rows for every row at the start of the workspace, if it holds them and a pass of
+  // steps 1-2 over all rows: then steps 1-2 run once, as soon as the (small) indexer tensors
+  // have landed, and only the attention runs per range.
+  const int64_t K = P->top_k;
+  const int64_t idx_bytes = round_up(TQ * K * 4, 256);
+  FusedGeom fg;
+  const bool fused = fused_wanted(P, &Rd, &fg);
+  const bool split = (int64_t)ws_bytes > idx_bytes &&
+                     (fused ? fused_rows(fg, (int64_t)ws_bytes - idx_bytes) >= TQ
+                            : ((int64_t)ws_bytes - idx_bytes) / (scores_ld(R) * 4) >= 1);
+  int64_t kv_done = 0;
+  if (split) {
+    DSA_TRY(check_indexer(P));
+    DSA_TRY(check_attn(P));
+    int32_t* idx_all = static_cast<int32_t*>(workspace);
+    void* scratch = static_cast<char*>(workspace) + idx_bytes;
+    DSA_TRY(h2d(at(dev->q_idx, 0), host->q_idx, (size_t)TQ * idx_row, d->s_in));
+    DSA_TRY(h2d(at(dev->k_idx, 0), host->k_idx, (size_t)R->total_kv * idx_row, d->s_in));
+    cudaEvent_t ev_idx = d->events[2 + 2 * n_chunks];
+    if (cudaEventRecord(ev_idx, d->s_in) != cudaSuccess ||
+        cudaStreamWaitEvent(st, ev_idx, 0) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    DSA_TRY(run_index(*d, P, &Rd, dev->q_idx, dev->k_idx, dev->w, 0, TQ, idx_all, scratch,
+                      (size_t)((int64_t)ws_bytes - idx_bytes), st));
+    for (int c = 0; c < n_chunks; ++c) {
+      const int64_t a0 = TQ * c / n_chunks, a1 = TQ * (c + 1) / n_chunks;
+      if (a0 == a1) continue;
+      const int64_t kv_need = std::max(kv_done, kv_need_of(a0, a1));
+      cudaEvent_t ev_in = d->events[2 + 2 * c], ev_done = d->events[3 + 2 * c];
+      const size_t r0 = (size_t)kv_done, rn = (size_t)(kv_need - kv_done);
+      DSA_TRY(h2d(at(dev->k_cache, r0 * kv_row), at(host->k_cache, r0 * kv_row), rn * kv_row, d->s_in));
+      DSA_TRY(h2d(at(dev->v_cache, r0 * kv_row), at(host->v_cache, r0 * kv_row), rn * kv_row, d->s_in));
+      kv_done = kv_need;
+      const size_t q0 = (size_t)a0, qn = (size_t)(a1 - a0);
+      DSA_TRY(h2d(at(dev->q, q0 * q_row), at(host->q, q0 * q_row), qn * q_row, d->s_in));
+      if (host->gate)
+        DSA_TRY(h2d(at(dev->gate, q0 * q_row), at(host->gate, q0 * q_row), qn * q_row, d->s_in));
+      if (cudaEventRecord(ev_in, d->s_in) != cudaSuccess ||
+          cudaStreamWaitEvent(st, ev_in, 0) != cudaSuccess)
+        return DSA_ERR_CUDA;
+      DSA_TRY(launch_attn(*d, P, &Rd, dev->q, dev->k_cache, dev->v_cache, idx_all + a0 * K, K, a0,
+                          a1 - a0, dev->gate, dev->out, nullptr, nullptr, st));
+      if (cudaEventRecord(ev_done, st) != cudaSuccess ||
+          cudaStreamWaitEvent(d->s_out, ev_done, 0) != cudaSuccess ||
+          cudaMemcpyAsync(at(host->out, q0 * q_row), at(dev->out, q0 * q_row), qn * q_row,
+                          cudaMemcpyDeviceToHost, d->s_out) != cudaSuccess)
+        return DSA_ERR_CUDA;
+    }
+  } else {
+    // the layer per range, each range's inputs uploaded just before it
+    for (int ci = 0; ci < n_chunks; ++ci) {
+      const int c = reverse ? n_chunks - 1 - ci : ci;
+      const int64_t a0 = TQ * c / n_chunks, a1 = TQ * (c + 1) / n_chunks;
+      if (a0 == a1) continue;
+      const int64_t kv_need = std::max(kv_done, kv_need_of(a0, a1));
+      cudaEvent_t ev_in = d->events[2 + 2 * ci], ev_done = d->events[3 + 2 * ci];
+      const size_t r0 = (size_t)kv_done, rn = (size_t)(kv_need - kv_done);
+      DSA_TRY(h2d(at(dev->k_idx, r0 * idx_row), at(host->k_idx, r0 * idx_row), rn * idx_row, d->s_in));
+      DSA_TRY(h2d(at(dev->k_cache, r0 * kv_row), at(host->k_cache, r0 * kv_row), rn * kv_row, d->s_in));
+      DSA_TRY(h2d(at(dev->v_cache, r0 * kv_row), at(host->v_cache, r0 * kv_row), rn * kv_row, d->s_in));
+      kv_done = kv_need;
+      const size_t q0 = (size_t)a0, qn = (size_t)(a1 - a0);
+      DSA_TRY(h2d(at(dev->q_idx, q0 * idx_row), at(host->q_idx, q0 * idx_row), qn * idx_row, d->s_in));
+      DSA_TRY(h2d(at(dev->q, q0 * q_row), at(host->q, q0 * q_row), qn * q_row, d->s_in));
+      if (host->gate)
+        DSA_TRY(h2d(at(dev->gate, q0 * q_row), at(host->gate, q0 * q_row), qn * q_row, d->s_in));
+      if (cudaEventRecord(ev_in, d->s_in) != cudaSuccess ||
+          cudaStreamWaitEvent(st, ev_in, 0) != cudaSuccess)
+        return DSA_ERR_CUDA;
+      DSA_TRY(run_layer(P, &Rd, dev->q_idx, dev->k_idx, dev->w, dev->q, dev->k_cache,
+                        dev->v_cache, dev->gate, dev->out, nullptr, nullptr, workspace, ws_bytes,
+                        stream, false, a0, a1));
+      if (cudaEventRecord(ev_done, st) != cudaSuccess ||
+          cudaStreamWaitEvent(d->s_out, ev_done, 0) != cudaSuccess ||
+          cudaMemcpyAsync(at(host->out, q0 * q_row), at(dev->out, q0 * q_row), qn * q_row,
+                          cudaMemcpyDeviceToHost, d->s_out) != cudaSuccess)
+        return DSA_ERR_CUDA;
+    }
+  }
+  // the caller's stream completes after the last copy back
+  if (cudaEventRecord(ev_end, d->s_out) != cudaSuccess ||
+      cudaStreamWaitEvent(st, ev_end, 0) != cudaSuccess)
+    return DSA_ERR_CUDA;
   return DSA_OK;
 }
 
