@@ -321,7 +321,9 @@ typedef struct {
  *   workspace as dsa_prefill.
  * The call returns once everything is enqueued; `stream` completes after the last output
  * row is back in host memory.  The device buffers must not be touched by other streams
- * until then.  Contiguous caches only (DSA_ERR_UNSUPPORTED with a block table).
+ * until then.  The library's two copy streams per device are shared by all such calls
+ * (calls from several host threads enqueue one at a time and their copies queue behind each
+ * other).  Contiguous caches only (DSA_ERR_UNSUPPORTED with a block table).
  */
 dsa_status dsa_prefill_from_host(const dsa_params* params, const dsa_ragged* ragged,
                                  const dsa_layer_buffers* host, const dsa_layer_buffers* dev,

@@ -80,6 +80,7 @@ struct DeviceState {
   // copy streams of dsa_prefill_from_host (created on first use) and its events
   cudaStream_t s_in = nullptr, s_out = nullptr;
   std::vector<cudaEvent_t> events;
+  std::mutex enqueue_mu;
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -508,6 +509,7 @@ dsa_status fused_pass(const DeviceState& dev, const dsa_params* P, const dsa_rag
   a.pages = cache_pages(R);
   const size_t smem = topk_smem_bytes(R->max_kv_len);
   a.bm_words = topk_fused_bm_words(std::max(R->max_kv_len, 1));
+  a.prefetch_ahead = 3 * dev.num_sms;  // three selection CTAs share an SM
   {  // (4) exact selection over the candidates
     StageScope scope(1, stream);
     topk_fused_kernel<<<(unsigned)q_count, kTopkThreads,
@@ -554,7 +556,12 @@ dsa_status launch_attn(const DeviceState& dev, const dsa_params* P, const dsa_ra
   const float scale = P->attn_scale > 0.f ? P->attn_scale : 1.0f / std::sqrt((float)P->head_dim);
   a.scale_log2 = scale * 1.4426950408889634f;
   a.pages = cache_pages(R);
-  const int hkv_cta = std::min(P->n_kv_heads, 8);
+  // KV heads per CTA: up to 8, fewer when there are too few query rows to fill the GPU
+  // twice over (decode batches), down to one KV head per CTA (halving keeps dividing Hkv:
+  // 1, 2, 4 or a multiple of 8)
+  int hkv_cta = std::min(P->n_kv_heads, 8);
+  while (hkv_cta > 1 && q_count * (P->n_kv_heads / hkv_cta) < 2 * (int64_t)dev.num_sms)
+    hkv_cta /= 2;
   const int nt = a.G > 8 ? 2 : 1;
   dim3 grid((unsigned)q_count, (unsigned)(P->n_kv_heads / hkv_cta));
   const size_t smem = attn_smem_bytes();
@@ -1026,6 +1033,9 @@ dsa_status dsa_prefill_from_host(const dsa_params* P, const dsa_ragged* R,
   DeviceState* d = nullptr;
   DSA_TRY(device_setup(&d));
   DSA_TRY(copy_streams(d, 2 * n_chunks + 3));
+  // the copy streams and events are shared by the device's calls: one enqueue at a time
+  // (a later call's records do not disturb the waits an earlier call already enqueued)
+  std::lock_guard<std::mutex> enqueue_lock(d->enqueue_mu);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaEvent_t ev_start = d->events[0], ev_end = d->events[1];
   const size_t e_idx = P->idx_dtype == DSA_FP8_E4M3 ? 1 : 2;

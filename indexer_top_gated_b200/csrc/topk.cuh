@@ -90,6 +90,8 @@ struct TopkArgs {
   const int32_t* cand_cnt;  // [q_count, 4] per segment
   int32_t* fb_list;         // [1 + q_count]: count, then rows (within the launch) to redo
   int blk_shift;            // rows of block scores: n = (p >> blk_shift) + 1 entries
+  int prefetch_ahead;       // fused selection: warm L2 with the candidates of the row this
+                            // many rows later in launch order (about one wave of CTAs)
   int bm_words;             // words of each position bitmap (topk_fused_bm_words)
   // fallback: recompute a row's scores on CUDA cores (same formula as the indexer)
   const void* q_idx;
@@ -855,6 +857,20 @@ __global__ void __launch_bounds__(kTopkThreads, 3) topk_fused_kernel(TopkArgs a)
     return;
   }
   const int seg = a.cap >> 2;
+  if (tid == 0 && a.prefetch_ahead > 0 && i >= a.prefetch_ahead) {
+    // the CTA that will take row i2 starts about when this one ends: pull its candidate
+    // segments towards L2 now (a hint only; nothing waits for it)
+    const int64_t i2 = i - a.prefetch_ahead;
+    const int4 n4 = __ldg(reinterpret_cast<const int4*>(a.cand_cnt) + i2);
+    const int nseg[4] = {n4.x, n4.y, n4.z, n4.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int n = nseg[q] < seg ? nseg[q] : seg;
+      if (n > 0)
+        bulk_prefetch_l2(a.cand + i2 * (int64_t)a.cap + (int64_t)q * seg,
+                         (uint32_t)(((int64_t)n * 8 + 15) & ~int64_t(15)));
+    }
+  }
   const int4 c4 = __ldg(reinterpret_cast<const int4*>(a.cand_cnt) + i);
   const uint32_t cnt[4] = {(uint32_t)c4.x, (uint32_t)c4.y, (uint32_t)c4.z, (uint32_t)c4.w};
   const uint32_t C = cnt[0] + cnt[1] + cnt[2] + cnt[3];
