@@ -556,12 +556,10 @@ dsa_status launch_attn(const DeviceState& dev, const dsa_params* P, const dsa_ra
   const float scale = P->attn_scale > 0.f ? P->attn_scale : 1.0f / std::sqrt((float)P->head_dim);
   a.scale_log2 = scale * 1.4426950408889634f;
   a.pages = cache_pages(R);
-  // KV heads per CTA: up to 8, fewer when there are too few query rows to fill the GPU
-  // twice over (decode batches), down to one KV head per CTA (halving keeps dividing Hkv:
-  // 1, 2, 4 or a multiple of 8)
-  int hkv_cta = std::min(P->n_kv_heads, 8);
-  while (hkv_cta > 1 && q_count * (P->n_kv_heads / hkv_cta) < 2 * (int64_t)dev.num_sms)
-    hkv_cta /= 2;
+  // KV heads per CTA: up to 8.  Fixed by the shape alone, so that a row's result does not
+  // depend on how the rows are split into launches (the warps' partial softmax states are
+  // merged in an order set by the CTA shape).
+  const int hkv_cta = std::min(P->n_kv_heads, 8);
   const int nt = a.G > 8 ? 2 : 1;
   dim3 grid((unsigned)q_count, (unsigned)(P->n_kv_heads / hkv_cta));
   const size_t smem = attn_smem_bytes();

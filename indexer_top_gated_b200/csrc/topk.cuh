@@ -688,7 +688,9 @@ DSA_DEV bool topk_candidates_row(const TopkArgs& a, int nn, const float2* cl, in
     }
 #pragma unroll
     for (int u = 0; u < kTopkCandBatch; ++u) {
-      if (pp[u] == 0xFFFFFFFFu) continue;
+      // (also skips positions outside the row, which only a corrupted workspace can hold:
+      // they never index the bitmap)
+      if (pp[u] >= (uint32_t)nn) continue;
       const uint32_t bin = kk[u] >> 20, pos = pp[u];
       if (bin > b || (whole && bin == b)) {
         atomicOr(&bm[pos >> 5], 1u << (pos & 31u));
@@ -700,12 +702,13 @@ DSA_DEV bool topk_candidates_row(const TopkArgs& a, int nn, const float2* cl, in
     }
   }
   __syncthreads();
-  if (!whole && tid < (int)n_bin) {
+  const uint32_t n_set = sh.ncand;  // the bin's candidates set aside (n_bin unless skipped)
+  if (!whole && tid < (int)n_set) {
     // rank among the bin: larger keys first, then lower positions
     const uint32_t k0 = bk[tid], p0 = bp[tid];
     uint32_t rank = 0;
 #pragma unroll 4
-    for (uint32_t x = 0; x < n_bin; ++x) {
+    for (uint32_t x = 0; x < n_set; ++x) {
       const uint32_t k1 = bk[x];
       rank += (k1 > k0) || (k1 == k0 && bp[x] < p0);
     }
