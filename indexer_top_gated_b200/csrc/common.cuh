@@ -272,10 +272,6 @@ DSA_DEV float ex2_approx(float x) {
   return y;
 }
 
-// The two bf16 halves of a packed pair, as fp32 (exact).
-DSA_DEV float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
-DSA_DEV float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
-
 // ------------------------------------------------------------------ cp.async
 
 // 16-byte async copy global -> shared; src_bytes = 0 zero-fills the destination.

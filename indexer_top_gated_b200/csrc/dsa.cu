@@ -123,12 +123,8 @@ dsa_status device_setup(DeviceState** out) {
     e = e ? e : allow_smem(topk_kernel<kTopkFallback>, topk_smem_bytes(0));
     e = e ? e : allow_smem(sparse_attn_kernel<1, 1>, attn_smem_bytes());
     e = e ? e : allow_smem(sparse_attn_kernel<2, 1>, attn_smem_bytes());
-    e = e ? e : allow_smem(sparse_attn_kernel<4, 1>, attn_smem_bytes());
-    e = e ? e : allow_smem(sparse_attn_kernel<8, 1>, attn_smem_bytes());
     e = e ? e : allow_smem(sparse_attn_kernel<1, 2>, attn_smem_bytes());
     e = e ? e : allow_smem(sparse_attn_kernel<2, 2>, attn_smem_bytes());
-    e = e ? e : allow_smem(sparse_attn_kernel<4, 2>, attn_smem_bytes());
-    e = e ? e : allow_smem(sparse_attn_kernel<8, 2>, attn_smem_bytes());
     if (e != cudaSuccess) return DSA_ERR_CUDA;
     if (!g_encode) {
       void* fn = nullptr;
@@ -556,10 +552,10 @@ dsa_status launch_attn(const DeviceState& dev, const dsa_params* P, const dsa_ra
   const float scale = P->attn_scale > 0.f ? P->attn_scale : 1.0f / std::sqrt((float)P->head_dim);
   a.scale_log2 = scale * 1.4426950408889634f;
   a.pages = cache_pages(R);
-  // KV heads per CTA: up to 8.  Fixed by the shape alone, so that a row's result does not
-  // depend on how the rows are split into launches (the warps' partial softmax states are
-  // merged in an order set by the CTA shape).
-  const int hkv_cta = std::min(P->n_kv_heads, 8);
+  // KV heads per CTA: two (one for a single-KV-head layer).  Fixed by the shape alone, so
+  // that a row's result does not depend on how the rows are split into launches (the
+  // warps' partial softmax states are merged in an order set by the CTA shape).
+  const int hkv_cta = P->n_kv_heads == 1 ? 1 : 2;
   const int nt = a.G > 8 ? 2 : 1;
   dim3 grid((unsigned)q_count, (unsigned)(P->n_kv_heads / hkv_cta));
   const size_t smem = attn_smem_bytes();
@@ -569,12 +565,8 @@ dsa_status launch_attn(const DeviceState& dev, const dsa_params* P, const dsa_ra
     sparse_attn_kernel<H, N><<<grid, AttnGeom<H>::kThreads, smem, stream>>>(a);
   DSA_ATTN_CASE(1, 1)
   DSA_ATTN_CASE(2, 1)
-  DSA_ATTN_CASE(4, 1)
-  DSA_ATTN_CASE(8, 1)
   DSA_ATTN_CASE(1, 2)
   DSA_ATTN_CASE(2, 2)
-  DSA_ATTN_CASE(4, 2)
-  DSA_ATTN_CASE(8, 2)
 #undef DSA_ATTN_CASE
   ++t_launches;
   return launch_status("sparse_attn_kernel");

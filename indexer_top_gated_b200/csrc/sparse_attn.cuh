@@ -1,12 +1,12 @@
 // sparse_attn.cuh - steps 3-4 of the layer: exact softmax attention over the selected
 // cache rows, with the sigmoid output gate fused into the epilogue.
 //
-// One CTA per (query row, block of up to 8 KV heads), 8 warps.  Each warp owns one KV
-// head and 16 positions of every chunk of selected positions, and gathers exactly the
-// bytes it consumes, so warps never synchronise with each other inside the main loop:
+// One CTA per (query row, pair of KV heads), 4 warps, three CTAs per SM.  Each warp owns
+// one KV head and 16 positions of every chunk of selected positions, and gathers exactly
+// the bytes it consumes, so warps never synchronise with each other inside the main loop:
 //  - gather: the warp's 16 positions x (K and V slices of its head, 256 B each) arrive
 //    through 16-byte cp.async (32 lanes = 512 contiguous bytes per instruction) into the
-//    warp's own 3-stage ring (XOR-swizzled 16-byte chunks, conflict-free for ldmatrix).
+//    warp's own 2-stage ring (XOR-swizzled 16-byte chunks, conflict-free for ldmatrix).
 //    Index entries are read once per position and shared across the warp by shuffles;
 //    padding / out-of-range entries are zero-filled and masked (a ballot mask).
 //  - logits are computed transposed, S^T = K_sel Q^T (mma.sync m16n8k16, keys on M, the
@@ -14,9 +14,10 @@
 //    heads needs no padding and the query heads of a GQA group share the gather.
 //  - online softmax in registers (log2 domain); P^T becomes the B operand of
 //    O^T += V_sel^T P^T through movmatrix (8x8 transposes in registers) and V^T comes
-//    from ldmatrix.trans.  P enters as two bf16 terms (P_hi + P_lo), so rounding P costs
-//    ~2^-17 relative instead of 2^-9: the error no longer scales with sum_j p_j |v_j|
-//    (which dominates outputs that nearly cancel).
+//    from ldmatrix.trans.  P enters rounded to bf16 (2^-9 relative per weight; the row sum
+//    l is taken from the fp32 weights).  Carrying P as P_hi + P_lo (two bf16 terms, ~2^-17)
+//    was measured at 8 % more time for the whole kernel: the output is bf16 itself, so the
+//    single rounding costs no more than the output's own.
 //  - warps of the same KV head merge (m, l, O) through shared memory; the epilogue
 //    divides by l, multiplies by sigmoid(gate) (and adds the second branch weighted by
 //    1 - sigmoid(gate) when one is given) and stores bf16 (and the LSE).
@@ -31,13 +32,18 @@ namespace dsa {
 constexpr int kHeadDim = 128;
 constexpr float kLazyMax = 8.f;  // log2 units the running maximum may lag behind
 
-// Warps per CTA and ring depth per warp: 12 warps x 2 stages when a CTA holds at most 4
-// KV heads (more warps hide more latency), 8 warps x 3 stages for 8 KV heads.  Either
-// way the rings take 192 KiB.
+// CTA shape: 4 warps with 2-stage rings (64 KiB), three CTAs per SM (12 warps, the most
+// that the ~150-170 registers per thread and the rings allow).  A CTA holds two KV heads
+// (two warps each, 32 positions per chunk) or, for a layer with a single KV head, one
+// head (four warps, 64 positions per chunk).  Several small CTAs per SM overlap one row's
+// set-up (index scan, query loads, first gathers) and merge / epilogue with the main
+// loops of the others, which one large CTA per SM left exposed.
 template <int HKV_CTA>
 struct AttnShape {
-  static constexpr int kWarps = HKV_CTA == 8 ? 8 : 12;
-  static constexpr int kStages = HKV_CTA == 8 ? 3 : 2;
+  static_assert(HKV_CTA == 1 || HKV_CTA == 2, "one or two KV heads per CTA");
+  static constexpr int kWarps = 4;
+  static constexpr int kStages = 2;
+  static constexpr int kCtasPerSm = 3;
 };
 
 struct AttnArgs {
@@ -80,7 +86,8 @@ __host__ inline size_t attn_smem_bytes() {
 }
 
 template <int HKV_CTA, int NT>
-__global__ void __launch_bounds__(AttnGeom<HKV_CTA>::kThreads, 1) sparse_attn_kernel(AttnArgs a) {
+__global__ void __launch_bounds__(AttnGeom<HKV_CTA>::kThreads, AttnShape<HKV_CTA>::kCtasPerSm)
+    sparse_attn_kernel(AttnArgs a) {
   using Geo = AttnGeom<HKV_CTA>;
   constexpr int CH = Geo::kChunk;
   constexpr int kAttnThreads = Geo::kThreads;
@@ -236,7 +243,7 @@ __global__ void __launch_bounds__(AttnGeom<HKV_CTA>::kThreads, 1) sparse_attn_ke
     }
     const bool v_lo = (vm >> (lane >> 2)) & 1u;
     const bool v_hi = (vm >> ((lane >> 2) + 8)) & 1u;
-    uint32_t pb[NT][4];
+    uint32_t pb[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       s[nt][0] = v_lo ? (s[nt][0] + s2[nt][0]) * a.scale_log2 : -INFINITY;
@@ -285,14 +292,8 @@ __global__ void __launch_bounds__(AttnGeom<HKV_CTA>::kThreads, 1) sparse_attn_ke
           l_run[nt][cc] += pr[cc] + pr[cc + 2];
         }
       }
-      // P = P_hi + P_lo, both bf16: the P.V product keeps ~16 significant bits of P
-      const uint32_t h01 = pack_bf16x2(pr[0], pr[1]), h23 = pack_bf16x2(pr[2], pr[3]);
-      const uint32_t l01 = pack_bf16x2(pr[0] - bf16_lo(h01), pr[1] - bf16_hi(h01));
-      const uint32_t l23 = pack_bf16x2(pr[2] - bf16_lo(h23), pr[3] - bf16_hi(h23));
-      pb[nt][0] = movmatrix_trans(h01);  // positions 0-7
-      pb[nt][1] = movmatrix_trans(h23);  // positions 8-15
-      pb[nt][2] = movmatrix_trans(l01);
-      pb[nt][3] = movmatrix_trans(l23);
+      pb[nt][0] = movmatrix_trans(pack_bf16x2(pr[0], pr[1]));  // positions 0-7
+      pb[nt][1] = movmatrix_trans(pack_bf16x2(pr[2], pr[3]));  // positions 8-15
     }
     // O^T[128 dims x 8 heads] += V_sel^T[128 x 16] * P^T[16 x 8]
 #pragma unroll
@@ -301,10 +302,7 @@ __global__ void __launch_bounds__(AttnGeom<HKV_CTA>::kThreads, 1) sparse_attn_ke
       const int chv = mt * 2 + vch;
       ldmatrix_x4_trans(vst + vt * 256 + ((chv ^ (vt & 7)) << 4), vf);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        mma_bf16_16816(o[nt][mt], vf, pb[nt][0], pb[nt][1]);
-        mma_bf16_16816(o[nt][mt], vf, pb[nt][2], pb[nt][3]);
-      }
+      for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[nt][mt], vf, pb[nt][0], pb[nt][1]);
     }
     __syncwarp();  // the slot is refilled by the next iteration's loads
   }
@@ -314,9 +312,9 @@ __global__ void __launch_bounds__(AttnGeom<HKV_CTA>::kThreads, 1) sparse_attn_ke
 
   // ---- merge the warps of each KV head through shared memory
   constexpr int HPW = NT * 8;  // head slots per warp
-  float* red_o = reinterpret_cast<float*>(smem);       // [8 warps][HPW][128]
-  float* red_m = red_o + kAttnWarps * HPW * kHeadDim;  // [8][HPW]
-  float* red_l = red_m + kAttnWarps * HPW;             // [8][HPW]
+  float* red_o = reinterpret_cast<float*>(smem);       // [warps][HPW][128]
+  float* red_m = red_o + kAttnWarps * HPW * kHeadDim;  // [warps][HPW]
+  float* red_l = red_m + kAttnWarps * HPW;             // [warps][HPW]
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll

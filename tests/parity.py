@@ -4,12 +4,16 @@ Tolerance (gated bf16 outputs vs the fp64 oracle):
   max |err| <= 1e-2 and mean |err| <= 1e-3 (the stated bar), plus two checks that keep
   the bar meaningful at these magnitudes (|out| is ~1e-3 for near-uniform softmax, so
   an all-zero output would pass the absolute bar):
-  ||err||_2 / ||ref||_2 <= 1e-2, and per element |err| <= 2^-7 |ref| + 1e-5.
+  ||err||_2 / ||ref||_2 <= 1e-2, and per element |err| <= 2^-7 |ref| + 2^-6 rms_h, with
+  rms_h the root mean square of the reference over the element's (row, head).
 Derivation of the per-element bound: the output is rounded to bf16 (relative 2^-9);
-the softmax weights enter the P.V product as a sum of two bf16 terms (relative error
-~2^-17 of sum_j p_j |v_j|, far below 1e-5 at these magnitudes); logits, exponentials
-and sums are fp32 (relative ~1e-6).  2^-7 leaves a factor 4 over the output rounding,
-and 1e-5 covers outputs that cancel to near zero.
+the softmax weights enter the P.V product rounded to bf16 (relative 2^-9 each), so an
+element's error is sum_j (p^_j - p_j) v_j / l: with the rounding errors of ~2048 weights
+independent, its standard deviation is ~2^-9 / sqrt(3) times the spread of sum_j p_j v_j / l
+over the head's elements, i.e. ~1.1e-3 rms_h for random V; logits, exponentials and sums
+are fp32 (relative ~1e-6).  2^-7 leaves a factor 4 over the output rounding, and 2^-6 rms_h
+is ~14 standard deviations of the weight rounding, while one wrong index among K or a
+dropped gate moves many elements by far more.
 """
 from __future__ import annotations
 
@@ -22,7 +26,7 @@ MAX_ABS = 1e-2
 MEAN_ABS = 1e-3
 REL_L2 = 1e-2
 ELEM_REL = 2.0 ** -7
-ELEM_ABS = 1e-5
+ELEM_RMS = 2.0 ** -6
 
 
 def close_report(got: np.ndarray, ref: np.ndarray) -> dict:
@@ -30,11 +34,13 @@ def close_report(got: np.ndarray, ref: np.ndarray) -> dict:
     ref = np.asarray(ref, dtype=np.float64)
     err = np.abs(got - ref)
     nref = np.linalg.norm(ref)
+    # (row, head) scale: the last axis is the head dimension
+    rms_h = np.sqrt(np.mean(ref * ref, axis=-1, keepdims=True)) if ref.ndim else np.abs(ref)
     rep = {
         "max_abs": float(err.max()) if err.size else 0.0,
         "mean_abs": float(err.mean()) if err.size else 0.0,
         "rel_l2": float(np.linalg.norm(got - ref) / nref) if nref > 0 else float(np.linalg.norm(got)),
-        "elem_viol": int(np.sum(err > ELEM_REL * np.abs(ref) + ELEM_ABS)),
+        "elem_viol": int(np.sum(err > ELEM_REL * np.abs(ref) + ELEM_RMS * rms_h)),
     }
     rep["ok"] = (rep["max_abs"] <= MAX_ABS and rep["mean_abs"] <= MEAN_ABS
                  and rep["rel_l2"] <= REL_L2 and rep["elem_viol"] == 0)
