@@ -526,7 +526,8 @@ dsa_status launch_attn(const DeviceState& dev, const dsa_params* P, const dsa_ra
                        const void* q, const void* k,
                        const void* v, const int32_t* idx, int64_t ld_idx, int64_t q_begin,
                        int64_t q_count, const void* gate, void* out, float* lse,
-                       int32_t* err_count, cudaStream_t stream, const void* other = nullptr) {
+                       int32_t* err_count, cudaStream_t stream, const void* other = nullptr,
+                       bool decode = false) {
   if (q_count == 0) return DSA_OK;
   AttnArgs a;
   a.q_offsets = R->q_offsets;
@@ -552,10 +553,12 @@ dsa_status launch_attn(const DeviceState& dev, const dsa_params* P, const dsa_ra
   const float scale = P->attn_scale > 0.f ? P->attn_scale : 1.0f / std::sqrt((float)P->head_dim);
   a.scale_log2 = scale * 1.4426950408889634f;
   a.pages = cache_pages(R);
-  // KV heads per CTA: two (one for a single-KV-head layer).  Fixed by the shape alone, so
-  // that a row's result does not depend on how the rows are split into launches (the
-  // warps' partial softmax states are merged in an order set by the CTA shape).
-  const int hkv_cta = P->n_kv_heads == 1 ? 1 : 2;
+  // KV heads per CTA: two, or one for a single-KV-head layer and for decode (one query per
+  // sequence gives too few rows to fill the GPU with two-head CTAs; one-head CTAs put four
+  // warps on a head and halve each warp's chunks).  Fixed by the call type and the shape
+  // alone, so that a row's result does not depend on how the rows are split into launches
+  // (the warps' partial softmax states are merged in an order set by the CTA shape).
+  const int hkv_cta = (decode || P->n_kv_heads == 1) ? 1 : 2;
   const int nt = a.G > 8 ? 2 : 1;
   dim3 grid((unsigned)q_count, (unsigned)(P->n_kv_heads / hkv_cta));
   const size_t smem = attn_smem_bytes();
@@ -665,7 +668,7 @@ dsa_status run_layer(const dsa_params* P, const dsa_ragged* R, const void* q_idx
       DSA_TRY(launch_topk(P, R, scores, ld, s0, cnt_s, idx + (s0 - a0) * K, K, nullptr, stream));
     }
     DSA_TRY(launch_attn(*dev, P, R, q, k, v, idx, K, a0, cnt_a, gate, out, nullptr, err_count,
-                        stream));
+                        stream, nullptr, decode));
   }
   return DSA_OK;
 }
