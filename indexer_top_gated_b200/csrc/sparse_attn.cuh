@@ -1,7 +1,7 @@
 // sparse_attn.cuh - steps 3-4 of the layer: exact softmax attention over the selected
 // cache rows, with the sigmoid output gate fused into the epilogue.
 //
-// One CTA per (query row, pair of KV heads), 4 warps, three CTAs per SM.  Each warp owns
+// One CTA per (query row, pair of KV heads or one KV head), 4 warps, three CTAs per SM.  Each warp owns
 // one KV head and 16 positions of every chunk of selected positions, and gathers exactly
 // the bytes it consumes, so warps never synchronise with each other inside the main loop:
 //  - gather: the warp's 16 positions x (K and V slices of its head, 256 B each) arrive
@@ -34,8 +34,9 @@ constexpr float kLazyMax = 8.f;  // log2 units the running maximum may lag behin
 
 // CTA shape: 4 warps with 2-stage rings (64 KiB), three CTAs per SM (12 warps, the most
 // that the ~150-170 registers per thread and the rings allow).  A CTA holds two KV heads
-// (two warps each, 32 positions per chunk) or, for a layer with a single KV head, one
-// head (four warps, 64 positions per chunk).  Several small CTAs per SM overlap one row's
+// (two warps each, 32 positions per chunk) or one head (four warps, 64 positions per
+// chunk): for a layer with a single KV head, and in decode, where one query per sequence
+// gives too few rows to fill the GPU with two-head CTAs.  Several small CTAs per SM overlap one row's
 // set-up (index scan, query loads, first gathers) and merge / epilogue with the main
 // loops of the others, which one large CTA per SM left exposed.
 template <int HKV_CTA>
