@@ -232,6 +232,10 @@ dsa_status dsa_index_topk_blocks(const dsa_params* params, const dsa_ragged* rag
  *   err_count int32 [1] or NULL: incremented once per index entry > p (skipped)
  * A row with nothing selected gets out = 0.  All rows read the same index set for all
  * heads; the gather of a KV head is shared by the query heads of its group.
+ * Precision: logits, the running maximum and the softmax sums are fp32, the softmax
+ * weights enter the P.V product rounded to bf16 (fp32 accumulation), and out is rounded
+ * to bf16 (nearest even).  A row's result does not depend on q_begin / q_count (how the
+ * rows are split into calls).
  * Requirements: q, k_cache, v_cache, gate, out 16-byte aligned.
  */
 dsa_status dsa_sparse_attn_gated(const dsa_params* params, const dsa_ragged* ragged,
