@@ -17,6 +17,8 @@ dropped gate moves many elements by far more.
 """
 from __future__ import annotations
 
+import math
+
 import numpy as np
 
 import dsa_synth as S
@@ -115,19 +117,45 @@ def oracle_row(w: S.Workload, r: int):
     return idx, out, lse, scores
 
 
+def fused_cap(K: int) -> int:
+    """Candidate slots per row of the library's fused indexer -> Top-K path (a planning
+    constant of that path, restated here to aim rows at its regimes): rows with n <= K
+    select everything, rows with n <= cap keep every score as a candidate, longer rows
+    use the sampled threshold."""
+    e = K / 16.0 + 1.0
+    R = math.ceil(e + 5.0 * math.sqrt(e) + 16.0)
+    return int(math.ceil(16.0 * (R + 6.0 * math.sqrt(R)) / 256.0) * 256)
+
+
 def sample_rows(w: S.Workload, count: int, seed: int = 1):
-    """Rows to check: first, last, sequence boundaries, needle rows, seeded random rest."""
+    """Rows to check: the first and last row of every sequence (of the first 16 and the last
+    one when there are more), the needle rows, the decode row with the longest history, rows
+    on both sides of n = K and n = cap (the fused path's regimes: select all, keep every
+    score, sampled threshold), then seeded random rows up to `count`."""
     total = w.total_q
     rows = {0, total - 1}
     qo = w.q_offsets
-    for b in range(min(w.batch, 4)):
-        rows.add(int(qo[b]))
-        rows.add(int(qo[b + 1]) - 1)
-    if w.batch > 4:
-        rows.add(int(qo[w.batch - 1]))
+    seqs = list(range(min(w.batch, 16))) + [w.batch - 1]
+    for b in seqs:
+        if w.q_lens[b] > 0:
+            rows.add(int(qo[b]))
+            rows.add(int(qo[b + 1]) - 1)
     if w.needle_rows:
         rows.add(w.needle_rows[0])
         rows.add(w.needle_rows[-1])
+    dec = [b for b in range(w.batch) if w.q_lens[b] == 1]
+    if dec:
+        rows.add(int(qo[max(dec, key=lambda b: w.kv_lens[b])]))
+        rows.add(int(qo[min(dec, key=lambda b: w.kv_lens[b])]))
+    K, cap = w.top_k, fused_cap(w.top_k)
+    for b in range(w.batch):
+        if w.q_lens[b] < 2:
+            continue
+        p0 = w.kv_lens[b] - w.q_lens[b]
+        for n in (K, K + 1, cap, cap + 1):
+            i = n - 1 - p0  # query index whose position is n - 1
+            if 0 <= i < w.q_lens[b]:
+                rows.add(int(qo[b]) + i)
     rng = np.random.default_rng(seed)
     while len(rows) < count:
         rows.add(int(rng.integers(0, total)))

@@ -3,7 +3,9 @@
 The same problem is run twice: with contiguous cache rows, and with every sequence's
 positions spread over pages in a random physical order (unused pages hold junk).  Paging
 only changes where rows are read, so every output (index rows, attention output, LSE)
-must be bit-identical; the contiguous results are pinned to the oracle elsewhere.
+must be bit-identical to the contiguous run; the paged results are also compared directly
+with the oracle run on the logical (contiguous) sequences: index rows bit for bit, outputs
+within the parity tolerance.
 Covered: the materialised layer (prefill and decode), the fused indexer -> Top-K path
 (sampled keys, candidate indexer and the CUDA-core recompute of rows whose threshold
 missed), and two sequences sharing the pages of a common prefix.
@@ -13,6 +15,8 @@ import pytest
 import torch
 
 import dsa_synth as S
+import oracle as O
+from tests import parity as PT
 
 pytestmark = pytest.mark.gpu
 
@@ -148,6 +152,12 @@ def test_paged_index_topk_with_recomputed_rows():
     idx_p = run(rgp, _to_dev(phys["k_idx"]))
     assert torch.equal(idx_c, idx_p)
     assert (idx_p[::3][: -1, :10].cpu().numpy() == np.arange(10)).all()
+    # and against the oracle's selection on the logical sequence (recomputed and regular rows)
+    orc = O.Oracle.for_workload(w, host)
+    got = idx_p.cpu().numpy()
+    for r in list(range(0, w.total_q, 41)) + [w.total_q - 1]:
+        np.testing.assert_array_equal(got[r], O.topk_row(orc.index_scores_row(r), w.top_k),
+                                      err_msg=f"row {r}")
 
 
 def test_shared_prefix_pages():
@@ -181,3 +191,43 @@ def test_shared_prefix_pages():
     out_p, idx_p = _layer(dsa.dsa_prefill, w, dev, cache, rgp)
     assert torch.equal(idx_c, idx_p)
     assert torch.equal(out_c, out_p)
+    _check_oracle(w, host, idx_p, out_p, range(w.total_q), "shared prefix")
+
+
+def _check_oracle(w, host, idx, out, rows, what):
+    """Paged results against the oracle on the logical sequences (host arrays)."""
+    rows = list(rows)
+    idx_ref, out_ref, _ = O.Oracle.for_workload(w, host).layer_rows(rows)
+    got_idx = idx.cpu().numpy()[rows]
+    np.testing.assert_array_equal(got_idx, idx_ref, err_msg=what)
+    PT.assert_close(PT.bf16_tensor_to_f64(out)[rows], out_ref, what)
+
+
+PAGED_ORACLE_CASES = {
+    "materialised": (dict(q_lens=[300, 1, 700], kv_lens=[900, 513, 700], K=64), 128, "prefill"),
+    "fused": (dict(q_lens=[12288], kv_lens=[12288], K=512), 256, "prefill"),
+    "decode": (dict(q_lens=[1] * 12, kv_lens=[1, 127, 128, 129, 1000, 4097, 300, 2500, 640, 768,
+                                               5000, 33], K=256), 256, "decode"),
+}
+
+
+@pytest.mark.parametrize("case", sorted(PAGED_ORACLE_CASES))
+def test_paged_matches_oracle(case):
+    """Shuffled, non-identity page assignments (unused pages hold junk), checked row by row
+    against the oracle on the logical sequences, not only against the contiguous GPU run."""
+    cfg, ps, kind = PAGED_ORACLE_CASES[case]
+    w = _wl(cfg["q_lens"], cfg["kv_lens"], K=cfg["K"])
+    fn = dsa.dsa_decode if kind == "decode" else dsa.dsa_prefill
+    _, (op, ip), (host, _, _, _, _, bt) = _both(w, ps, fn=fn, seed=11)
+    table = bt.cpu().numpy()
+    # the mapping is not the identity: some logical page lives elsewhere
+    ident = np.arange(table.shape[1])[None, :] + np.concatenate(
+        [[0], np.cumsum([(L + ps - 1) // ps for L in w.kv_lens])[:-1]])[:, None]
+    used = np.arange(table.shape[1])[None, :] < np.array(
+        [(L + ps - 1) // ps for L in w.kv_lens])[:, None]
+    assert np.any(table[used] != ident[used])
+    if w.total_q > 2000:
+        rows = sorted(set(range(0, w.total_q, 97)) | {w.total_q - 2, w.total_q - 1})
+    else:
+        rows = range(w.total_q)
+    _check_oracle(w, host, ip, op, rows, f"paged {case}")

@@ -360,11 +360,42 @@ def test_full_size_sampled_rows(name):
         pytest.skip(f"needs {w.device_bytes() / 2**30:.1f} GiB")
     dev = S.make_device_inputs(w)
     idx, out = _run_layer(w, dev)
-    for r in PT.sample_rows(w, 10):
+    rows = PT.sample_rows(w, 40)
+    assert len(rows) >= 40
+    for r in rows:
         idx_ref, out_ref, _, _ = PT.oracle_row(w, r)
         np.testing.assert_array_equal(idx[r].cpu().numpy(), idx_ref, err_msg=f"row {r}")
         PT.assert_close(PT.bf16_tensor_to_f64(out[r]), out_ref, f"{name} row {r}")
     for r in w.needle_rows:
         assert set(w.needle_pos) <= set(idx[r].cpu().numpy().tolist())
+    del dev, idx, out
+    torch.cuda.empty_cache()
+
+
+def test_full_size_discrimination():
+    """At the benchmark's size (T = 32768, K = 2048): one swapped index, or a dropped gate,
+    fails the parity check on every sampled row, while the layer's own output passes."""
+    w = S.workload("prefill_t32768_k2048")
+    dev = S.make_device_inputs(w)
+    idx, out = _run_layer(w, dev)
+    shape = dsa.workload_shape(w)
+    rg = _rg(w, dev)
+    rows = [2048, 5000, 17000, 32767]
+    for r in rows:
+        idx_ref, out_ref, _, _ = PT.oracle_row(w, r)
+        np.testing.assert_array_equal(idx[r].cpu().numpy(), idx_ref)
+        assert PT.close_report(PT.bf16_tensor_to_f64(out[r]), out_ref)["ok"]
+        bad = idx[r: r + 1].clone()
+        sel = set(bad[0].cpu().numpy().tolist())
+        bad[0, 0] = next(j for j in range(w.row_position(r) + 1) if j not in sel)
+        one = torch.zeros_like(out)
+        dsa.dsa_sparse_attn_gated(shape, rg, dev["q"], dev["k"], dev["v"], bad, w.top_k, r, 1,
+                                  dev["gate"], one)
+        nogate = torch.zeros_like(out)
+        dsa.dsa_sparse_attn_gated(shape, rg, dev["q"], dev["k"], dev["v"], idx[r: r + 1],
+                                  w.top_k, r, 1, None, nogate)
+        torch.cuda.synchronize()
+        assert not PT.close_report(PT.bf16_tensor_to_f64(one[r]), out_ref)["ok"], r
+        assert not PT.close_report(PT.bf16_tensor_to_f64(nogate[r]), out_ref)["ok"], r
     del dev, idx, out
     torch.cuda.empty_cache()

@@ -127,6 +127,59 @@ def test_indexer_fp8_e4m3_decoding_matches_torch():
         np.testing.assert_array_equal(s, np.maximum(0.0, sign * ref))
 
 
+def _e4m3(vals):
+    """OCP e4m3 codes (uint8) of values exactly representable in it (torch's conversion)."""
+    t = torch.tensor(np.asarray(vals, dtype=np.float32)).to(torch.float8_e4m3fn)
+    return t.view(torch.uint8).numpy()
+
+
+def test_indexer_dequant_scales_reduce_to_one_scaled_matmul():
+    """e4m3 indexer tensors with dequantisation scales 0.375 (q) and 2^-3 (k), the indexer
+    at lower precision of [GSA] "4. The Role of Gating and Engineering Considerations".
+    With q, k >= 0 ReLU is the identity and s = (scale_q q w) (scale_k k)^T is one matmul
+    (torch, fp64).  Every product is exact, so the match is bit for bit; a dropped, squared
+    or doubled scale fails."""
+    rng = np.random.default_rng(31)
+    Hi, Di, Q, L = 3, 16, 4, 11
+    qv = rng.integers(0, 5, size=(Q, Hi, Di)) / 8.0
+    kv = rng.integers(0, 5, size=(L, Hi, Di)) / 8.0
+    w = np.array([0.25, 0.5, 1.0], dtype=np.float32)
+    sq, sk = 0.375, 2.0 ** -3
+    a = {"q_idx": _e4m3(qv), "k_idx": _e4m3(kv), "w": w,
+         "q_offsets": np.array([0, Q]), "kv_offsets": np.array([0, L])}
+    orc = _problem(a, n_idx_heads=Hi, idx_dim=Di, idx_fp8=True, idx_scale_q=sq, idx_scale_k=sk)
+    qt = torch.tensor(qv) * sq * torch.tensor(w, dtype=torch.float64)[None, :, None]
+    lib = torch.matmul(qt.reshape(Q, -1), (torch.tensor(kv) * sk).reshape(L, -1).T).numpy()
+    for i in range(Q):
+        p = L - Q + i
+        np.testing.assert_array_equal(orc.index_scores_row(i), lib[i, : p + 1])
+    # the same problem unscaled is sq * sk times larger in every score: the scale is applied
+    unscaled = _problem(a, n_idx_heads=Hi, idx_dim=Di, idx_fp8=True)
+    s1 = unscaled.index_scores_row(Q - 1)
+    assert np.any(s1 > 0)
+    np.testing.assert_array_equal(orc.index_scores_row(Q - 1), s1 * (sq * sk))
+
+
+def test_indexer_scale_enters_once_as_a_product():
+    """Signed inputs: s(scale_q, scale_k) = scale_q * scale_k * s(1, 1), since a positive
+    factor commutes with the ReLU.  0.3 is not a power of two, so the match is to fp64
+    rounding; the splits (0.3, 1), (1, 0.3), (0.6, 0.5) pin c q.k with c = scale_q * scale_k
+    and fail for c^2, for scale_q applied to both operands, or for a dropped scale.
+    Positions whose unscaled score is 0 (every head's dot <= 0) stay 0 up to the fp64
+    rounding of a dot whose exact value is 0 (a few 1e-18)."""
+    a = _rand_layer(32, [5], [40], Hi=4, Di=8)
+    a["w"] = np.array([0.25, 0.5, 1.0, 2.0], dtype=np.float32)
+    base = _problem(a, n_idx_heads=4, idx_dim=8)
+    for r in range(5):
+        s1 = base.index_scores_row(r)
+        assert np.any(s1 == 0) and np.any(s1 > 0)
+        for sq, sk in ((0.3, 1.0), (1.0, 0.3), (0.6, 0.5), (0.375, 0.8)):
+            s = _problem(a, n_idx_heads=4, idx_dim=8, idx_scale_q=sq,
+                         idx_scale_k=sk).index_scores_row(r)
+            np.testing.assert_allclose(s, (sq * sk) * s1, rtol=1e-14, atol=1e-16)
+            assert np.all(np.abs(s[s1 == 0]) <= 1e-16)
+
+
 # ----------------------------------------------------------------------------- top-k
 
 def _is_valid_topk(s, K, idx):
@@ -225,8 +278,10 @@ def test_topk_short_row_takes_everything():
 
 # ----------------------------------------------------------------------------- attention
 
-def _dense_causal_reference(a, q_lens, kv_lens, Hq, Hkv, d, mask_rows=None, gate=True):
-    """torch SDPA (fp64, CPU) per sequence, GQA by repeating KV heads, times sigmoid(gate)."""
+def _dense_causal_reference(a, q_lens, kv_lens, Hq, Hkv, d, mask_rows=None, gate=True,
+                            scale=None):
+    """torch SDPA (fp64, CPU) per sequence, GQA by repeating KV heads, times sigmoid(gate);
+    scale None is SDPA's default 1/sqrt(d)."""
     G = Hq // Hkv
     outs = []
     qo, ko = a["q_offsets"], a["kv_offsets"]
@@ -244,7 +299,7 @@ def _dense_causal_reference(a, q_lens, kv_lens, Hq, Hkv, d, mask_rows=None, gate
             for i in range(Q):
                 sel = mask_rows[int(qo[b]) + i]
                 mask[i, sel[sel >= 0]] = True
-        o = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=mask)
+        o = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=mask, scale=scale)
         o = o.permute(1, 0, 2)
         if gate:
             g = torch.tensor(_val(a["gate"][qo[b]:qo[b + 1]]))
@@ -267,6 +322,28 @@ def test_full_history_reduces_to_dense_causal_attention():
     for r in rows:
         p = orc.position(r)
         np.testing.assert_array_equal(idx[r, : p + 1], np.arange(p + 1))
+
+
+def test_attention_scale_override_matches_sdpa():
+    """attn_scale = 0.2 instead of 1/sqrt(d): with K >= history the layer is dense causal
+    attention, i.e. torch SDPA with scale=0.2, times the sigmoid gate; the LSE is
+    torch.logsumexp of the 0.2-scaled logits.  The default-scale output must differ."""
+    q_lens, kv_lens = [5, 3], [9, 14]
+    Hq, Hkv, d = 4, 2, 8
+    a = _rand_layer(33, q_lens, kv_lens, Hq=Hq, Hkv=Hkv, d=d, scale=1.0)
+    kw = dict(top_k=16, n_idx_heads=3, idx_dim=8, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d)
+    orc = _problem(a, attn_scale=0.2, **kw)
+    rows = list(range(sum(q_lens)))
+    idx, out, lse = orc.layer_rows(rows, nthreads=2)
+    ref = _dense_causal_reference(a, q_lens, kv_lens, Hq, Hkv, d, scale=0.2)
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-14)
+    _, out_default, _ = _problem(a, **kw).layer_rows(rows, nthreads=2)
+    assert np.max(np.abs(out_default - out)) > 1e-3
+    # LSE of the last row of sequence 1 (position 13) and query head 3 (KV head 1)
+    r, h = rows[-1], 3
+    qv = torch.tensor(_val(a["q"][r, h]))
+    kv = torch.tensor(_val(a["k"][a["kv_offsets"][1]:a["kv_offsets"][2], h // 2]))
+    np.testing.assert_allclose(lse[r, h], torch.logsumexp(0.2 * (kv @ qv), 0).item(), rtol=1e-14)
 
 
 def test_sparse_selection_matches_masked_dense_attention():
