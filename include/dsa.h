@@ -359,7 +359,9 @@ dsa_status dsa_decode(const dsa_params* params, const dsa_ragged* ragged, const 
  *   before anything is launched (max_kv_len up to about 8.3 million at K = 2048).
  *   This entry point calls no cudaMalloc, cudaFree or other allocating routine.
  *   The first call on a device looks up the scratch's device address
- *   (cudaGetSymbolAddress), so make that first call before any stream capture.
+ *   (cudaGetSymbolAddress), so make that first call before any stream capture.  The
+ *   address is tied to the device's CUDA context; a call made in a new context (after
+ *   cudaDeviceReset, say) looks it up again, so that call too should precede any capture.
  *   All calls on a device share the one scratch array: calls that can overlap on the
  *   GPU (different streams, or different host threads) race and must be serialised by
  *   the caller.  No part of the scratch needs to be zeroed between calls.

@@ -72,8 +72,42 @@ struct StageScope {
 };
 
 // ---------------------------------------------------------------- per-device setup
+//
+// What the setup caches (the device address of the status word, the kernels' shared-memory
+// limits) belongs to the device's CUDA context: a context created anew (after
+// cudaDeviceReset, for instance) reloads the library's module at possibly other addresses.
+// The cache is therefore keyed by the context's unique id and redone when it changes.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+std::once_flag g_ctx_fns_once;
+
+// Unique id of the calling thread's current context, 0 if there is none (or it cannot be
+// read; callers then redo their setup, which is correct, only slower).
+uint64_t current_context_id() {
+  std::call_once(g_ctx_fns_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(fn);
+  });
+  if (!g_ctx_get_current || !g_ctx_get_id) return 0;
+  CUcontext c = nullptr;
+  if (g_ctx_get_current(&c) != CUDA_SUCCESS || !c) return 0;
+  unsigned long long id = 0;
+  if (g_ctx_get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return (uint64_t)id;
+}
+
 struct DeviceState {
   bool ready = false;
+  uint64_t ctx = 0;       // id of the context the cached setup belongs to
   int* status = nullptr;  // device address of g_status
   int num_sms = 148;
   size_t max_smem = 0;
@@ -97,7 +131,10 @@ dsa_status device_setup(DeviceState** out) {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_dev_mu);
   DeviceState& d = g_dev[dev];
-  if (!d.ready) {
+  const uint64_t ctx = current_context_id();
+  if (!d.ready || ctx == 0 || ctx != d.ctx) {
+    d.ready = false;
+    // (this call also creates and binds the primary context if there is none yet)
     if (cudaGetSymbolAddress((void**)&d.status, g_status) != cudaSuccess) return DSA_ERR_CUDA;
     cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
     int smem_optin = 0;
@@ -135,6 +172,7 @@ dsa_status device_setup(DeviceState** out) {
         return DSA_ERR_CUDA;
       g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
+    d.ctx = current_context_id();
     d.ready = true;
   }
   *out = &d;
@@ -1169,23 +1207,28 @@ dsa_status dsa_decode(const dsa_params* P, const dsa_ragged* R, const void* q_id
 // so callers that cannot allocate never have to.  It is reserved on every GPU that
 // loads the library and kept until the process exits.  Host code must not pass the
 // symbol itself to a kernel (on the host it names a stand-in, not device memory): the
-// first call on each device looks up its device address with cudaGetSymbolAddress.
+// first call on each device looks up its device address with cudaGetSymbolAddress.  The
+// address belongs to the device's current CUDA context: it is looked up again when the
+// context changes (a context created after cudaDeviceReset loads the module anew).
 namespace dsa {
 namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB per device
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 void* g_noalloc_ptr[kMaxDevices] = {};
+uint64_t g_noalloc_ctx[kMaxDevices] = {};
 std::mutex g_noalloc_mu;
 
 dsa_status noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  const uint64_t ctx = current_context_id();
+  if (!g_noalloc_ptr[dev] || ctx == 0 || ctx != g_noalloc_ctx[dev]) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr)
       return DSA_ERR_CUDA;
     g_noalloc_ptr[dev] = ptr;
+    g_noalloc_ctx[dev] = current_context_id();
   }
   *out = g_noalloc_ptr[dev];
   return DSA_OK;
