@@ -7,8 +7,12 @@ indexer 4 heads x 64 (bf16), with inputs resident in HBM.  Prints one JSON line.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Under torchrun every rank runs its own copy of the workload (weak scaling, no
-collective on the data path); the reported time is the max over ranks.
+Under torchrun the global batch is `world` copies of the workload, split over ranks by the
+data-parallel partitioner (indexer_top_gated_b200.partition: whole sequences by cost); each
+rank runs its share with no collective on the data path (weak scaling), and the reported
+time is the max over ranks.  Beside the headline the same run measures the gather ceilings
+that bound the attention, the decode workload and the K = 2048 workloads whose cache does
+not fit in L2.
 `--impl reference` times the CPU oracle on bounded samples of the same workload.
 """
 from __future__ import annotations
@@ -33,6 +37,10 @@ if ROOT not in sys.path:
 METRIC = "sparse-attn layer tokens/sec (prefill) & µs/token (decode) at K=2048, % roofline"
 WORKLOAD = "prefill_t32768_k2048"
 DECODE_WORKLOAD = "decode_b64_l131072"
+# measured in the same run beside the headline: the K = 2048 configurations whose K/V cache
+# no longer fits in L2
+EXTRA_WORKLOADS = ["prefill_t131072_needles", "mixed_serving"]
+L2_BYTES = 126e6
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -51,10 +59,15 @@ def parse_args():
     ap.add_argument("--ws-rows", type=int, default=0,
                     help="cap the workspace at this many query rows per pass (profiling)")
     ap.add_argument("--lean", action="store_true",
-                    help="only the timed region: no e2e, decode or CPU-baseline legs")
+                    help="only the timed region: no e2e, decode, CPU-baseline, gather-peak or "
+                         "extra-workload legs")
+    ap.add_argument("--also", default=",".join(EXTRA_WORKLOADS),
+                    help="comma-separated workloads also measured (not the headline); '' for none")
+    ap.add_argument("--no-peaks", action="store_true", help="skip the live gather-ceiling probe")
     a = ap.parse_args()
     if a.lean:
-        a.no_e2e = a.no_decode = a.no_cpu_baseline = True
+        a.no_e2e = a.no_decode = a.no_cpu_baseline = a.no_peaks = True
+        a.also = ""
     return a
 
 
@@ -107,6 +120,24 @@ def aggregate_max(ms_local: float, tokens_per_rank: int, world: int, device="cud
     return ms_max, tokens_per_rank * world / (ms_max / 1e3)
 
 
+def rank_workload(w, world: int, rank: int):
+    """This rank's share of a global batch of `world` copies of workload w (weak scaling):
+    the data-parallel partitioner deals whole sequences to ranks by cost; the rank's
+    sequences are generated with seed = rank, so ranks hold different data."""
+    import copy
+
+    from indexer_top_gated_b200 import partition as PA
+    if world == 1:
+        return w
+    sh = PA.shard(list(w.q_lens) * world, list(w.kv_lens) * world, w.top_k, world, rank,
+                  by="sequences")
+    rw = copy.copy(w)
+    rw.q_lens, rw.kv_lens, rw.seed = list(sh.q_lens), list(sh.kv_lens), rank
+    if (rw.q_lens, rw.kv_lens) != (list(w.q_lens), list(w.kv_lens)):
+        rw.needle_pos, rw.needle_rows = [], []  # planted rows belong to the workload's own layout
+    return rw
+
+
 def source_sha(paths):
     h = hashlib.sha256()
     for p in paths:
@@ -123,8 +154,9 @@ def l2_note(w):
     return f"inputs fit in L2 (q + gate + out = {mib:.0f} MiB per step); no flush: L2-warm timing"
 
 
-def committed_traffic(kernel_file: str, summary: str):
-    """DRAM bytes per launch recorded by an ncu capture, if the kernel has not changed since."""
+def committed_traffic(kernel_file: str, summary: str, key: str = "traffic_bytes_per_full_launch"):
+    """DRAM bytes per launch recorded by an ncu capture (a `key: value` line of a summary in
+    profiles/), or None if there is none or the kernel's source has changed since."""
     path = os.path.join(ROOT, "profiles", summary)
     if not os.path.exists(path):
         return None
@@ -136,9 +168,72 @@ def committed_traffic(kernel_file: str, summary: str):
     try:
         if vals.get("source_sha256_16") != source_sha([kernel_file, "indexer_top_gated_b200/csrc/common.cuh"]):
             return None
-        return float(vals["traffic_bytes_per_full_launch"])
+        return float(vals[key])
     except Exception:
         return None
+
+
+ATTN_SRC = "indexer_top_gated_b200/csrc/sparse_attn.cuh"
+
+
+def attn_traffic(workload: str):
+    return committed_traffic(ATTN_SRC, f"sparse_attn_gated_{workload}.txt")
+
+
+def kv_cache_bytes(w) -> int:
+    return 2 * w.total_kv * w.n_kv_heads * w.head_dim * 2
+
+
+def stage_report(w, stage_ms, stage_n, peaks, gather):
+    """Per-stage achieved rates and roofline fractions of one step of workload w.
+
+    - indexer: algorithmic flops (512 per score) against the sustained dense bf16 peak;
+    - Top-K: two byte definitions against the HBM copy peak -- the scope table's
+      (4 B per score read + 4 B per index written, the bytes a materialised selection must
+      move; the >= 60 % target is stated against this one) and, on the fused path, the
+      floor of what that path moves (12 B per selected position);
+    - attention: algorithmic bytes (selected K/V rows, q, gate, out, indices) against the
+      measured gather ceiling of random 256-byte rows from L2 (every gathered byte crosses
+      L2 -> SM), plus the DRAM bytes of a committed ncu capture against the HBM copy peak.
+    """
+    alg = algorithmic(w)
+    fused = stage_n[1] > 1
+    idx_tf = alg["idx_flops"] / (stage_ms[0] / 1e3) / 1e12 if stage_ms[0] > 0 else None
+    tk_s = alg["topk_bytes"] / (stage_ms[1] / 1e3) / 1e9 if stage_ms[1] > 0 else None
+    tk_f = alg["topk_bytes_fused"] / (stage_ms[1] / 1e3) / 1e9 if stage_ms[1] > 0 else None
+    at = alg["attn_bytes"] / (stage_ms[2] / 1e3) / 1e9 if stage_ms[2] > 0 else None
+    traffic = attn_traffic(w.name)
+    l2p = gather.get("l2", {}).get("gbs") if gather else None
+    dram_gbs = traffic / stage_n[2] / (stage_ms[2] / stage_n[2] / 1e3) / 1e9 \
+        if traffic and stage_ms[2] > 0 else None
+    hbm = peaks["hbm_gbs"]
+    stages = [
+        {"kernel": "idx_scores", "ms_per_step": stage_ms[0], "launches_per_step": stage_n[0],
+         "bound": "tensor", "achieved": idx_tf, "unit": "TFLOP/s",
+         "peak": peaks["bf16_tflops_sustained"],
+         "frac": idx_tf / peaks["bf16_tflops_sustained"] if idx_tf else None,
+         "path": "fused: sampled threshold, candidates only" if fused else "materialised scores"},
+        {"kernel": "topk_select", "ms_per_step": stage_ms[1], "launches_per_step": stage_n[1],
+         "bound": "hbm", "unit": "GB/s", "peak": hbm,
+         "achieved": tk_s, "frac": tk_s / hbm if tk_s else None,
+         "bytes_definition": "4 B per causal score read + 4 B per index written (target)",
+         "achieved_floor": tk_f if fused else None,
+         "frac_floor": tk_f / hbm if (fused and tk_f) else None,
+         "floor_definition": ("12 B per selected position (read its (position, score) "
+                              "candidate, write its index): what the fused path must move")},
+        {"kernel": "sparse_attn_gated", "ms_per_step": stage_ms[2], "launches_per_step": stage_n[2],
+         "bound": "l2", "unit": "GB/s", "achieved": at, "peak": l2p,
+         "frac": at / l2p if (at and l2p) else None,
+         "peak_definition": "measured gather of random 256-byte rows from an L2-resident buffer",
+         "kv_cache_bytes": kv_cache_bytes(w),
+         "kv_fits_l2": kv_cache_bytes(w) <= L2_BYTES,
+         "dram_traffic_per_launch": traffic / stage_n[2] if traffic else None,
+         "dram_gbs": dram_gbs, "dram_frac": dram_gbs / hbm if dram_gbs else None},
+    ]
+    for st in stages:
+        if st["bound"] == "hbm" and st["frac"] is not None:
+            assert st["frac"] <= 1.0, f"{st['kernel']}: {st['frac']:.3f} of the HBM peak is not an HBM rate"
+    return stages
 
 
 class ClockSampler:
@@ -213,8 +308,7 @@ def run_ours(args, rank, world, local_rank):
 
     dev_id = local_rank
     torch.cuda.set_device(dev_id)
-    w = S.workload(args.workload)
-    w.seed = rank  # every rank its own sequence; same shapes
+    w = rank_workload(S.workload(args.workload), world, rank)
     inputs = S.make_device_inputs(w)
     shape = dsa.workload_shape(w)
     rg = dsa.ragged(inputs["q_offsets"], inputs["kv_offsets"], w.q_lens, w.kv_lens)
@@ -362,6 +456,63 @@ def run_decode_side(args):
                               (stage_ms[0] / n / 1e3) / 1e9}
 
 
+def run_extra_workload(name, gather, steps=3, warmup=2):
+    """One more workload in the same run (not the headline): tokens/s and the per-stage
+    roofline fractions of a few steps of dsa_prefill / dsa_decode, inputs resident."""
+    import torch
+
+    import dsa_synth as S
+    import indexer_top_gated_b200 as dsa
+
+    w = S.workload(name)
+    decode = max(w.q_lens) == 1
+    free, _ = torch.cuda.mem_get_info()
+    if w.device_bytes() * 1.1 > free:
+        return {"workload": name, "skipped": f"needs {w.device_bytes() / 2**30:.1f} GiB"}
+    inputs = S.make_device_inputs(w)
+    shape = dsa.workload_shape(w)
+    rg = dsa.ragged(inputs["q_offsets"], inputs["kv_offsets"], w.q_lens, w.kv_lens)
+    _, ws_bytes = dsa.dsa_workspace_size(shape, rg, decode)
+    free, _ = torch.cuda.mem_get_info()
+    ws_bytes = int(min(ws_bytes, max(free - (4 << 30), 0)))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    out = torch.empty((w.total_q, w.n_q_heads, w.head_dim), dtype=torch.bfloat16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    layer = dsa.dsa_decode if decode else dsa.dsa_prefill
+
+    def step():
+        layer(shape, rg, inputs["q_idx"], inputs["k_idx"], inputs["w"], inputs["q"], inputs["k"],
+              inputs["v"], inputs["gate"], out, err_count=err, workspace=ws, ws_bytes=ws_bytes)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    dsa.dsa_stage_times(reset=True)
+    dsa.dsa_stage_timing(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        e0.record()
+        for _ in range(steps):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+    dsa.dsa_stage_timing(False)
+    stage_ms, stage_launches = dsa.dsa_stage_times(reset=True)
+    ms = e0.elapsed_time(e1) / steps
+    assert dsa.dsa_device_status() == 0 and int(err.item()) == 0
+    peaks, _ = load_peaks()
+    sm = [x / steps for x in stage_ms]
+    sn = [max(1, n // steps) for n in stage_launches]
+    rep = {"workload": name, "batch": w.batch, "total_q": w.total_q, "total_kv": w.total_kv,
+           "max_kv_len": max(w.kv_lens), "top_k": w.top_k, "q_heads": w.n_q_heads,
+           "kv_heads": w.n_kv_heads, "steps": steps, "warmup": warmup, "ms_per_step": ms,
+           "tokens_per_s": w.total_q / (ms / 1e3), "workspace_bytes": ws_bytes,
+           "stages": stage_report(w, sm, sn, peaks, gather), "clocks": clocks.summary()}
+    del inputs, ws, out
+    torch.cuda.empty_cache()
+    return rep
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 
 def cpu_oracle_sample(w, target_seconds: float, rows_per_call=None, offset=0):
@@ -493,6 +644,14 @@ def main():
     decode = None
     if world == 1 and not args.no_decode:
         decode = run_decode_side(args)
+    gather = None
+    if rank == 0 and not args.no_peaks:
+        from indexer_top_gated_b200 import peaks as P
+        gather = P.gather_peaks(torch.cuda.get_device_properties(local_rank).multi_processor_count)
+    extra = []
+    if world == 1:
+        for name in [x for x in args.also.split(",") if x]:
+            extra.append(run_extra_workload(name, gather))
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -500,46 +659,27 @@ def main():
         return
 
     w = res["w"]
-    alg = algorithmic(w)
     peaks, peak_src = load_peaks()
     steps = args.steps
     stage_ms = [m / steps for m in res["stage_ms"]]          # per step
     stage_n = [max(1, n // steps) for n in res["stage_launches"]]
-    names = ["idx_scores", "topk_select", "sparse_attn_gated"]
-    attn_gbs = alg["attn_bytes"] / (stage_ms[2] / 1e3) / 1e9 if stage_ms[2] > 0 else None
-    idx_tflops = alg["idx_flops"] / (stage_ms[0] / 1e3) / 1e12 if stage_ms[0] > 0 else None
-    # steps 1-2 ran fused (sampled keys + samples + candidates | thresholds + selection +
-    # fallback rows: several launches per stage) or on a materialised score matrix
-    fused = stage_n[1] > 1
-    topk_alg = alg["topk_bytes_fused"] if fused else alg["topk_bytes"]
-    topk_gbs = topk_alg / (stage_ms[1] / 1e3) / 1e9 if stage_ms[1] > 0 else None
-    stages = [
-        {"kernel": names[0], "ms_per_step": stage_ms[0], "launches_per_step": stage_n[0],
-         "bound": "tensor", "achieved": idx_tflops, "unit": "TFLOP/s",
-         "peak": peaks["bf16_tflops_sustained"],
-         "frac": idx_tflops / peaks["bf16_tflops_sustained"] if idx_tflops else None,
-         "path": "fused: sampled threshold, candidates only" if fused else "materialised scores",
-         "score_write_gbs": (None if fused else
-                             4 * alg["scores"] / (stage_ms[0] / 1e3) / 1e9 if stage_ms[0] else None)},
-        {"kernel": names[1], "ms_per_step": stage_ms[1], "launches_per_step": stage_n[1],
-         "bound": "hbm", "achieved": topk_gbs, "unit": "GB/s", "peak": peaks["hbm_gbs"],
-         "frac": topk_gbs / peaks["hbm_gbs"] if topk_gbs else None},
-        {"kernel": names[2], "ms_per_step": stage_ms[2], "launches_per_step": stage_n[2],
-         "bound": "hbm", "achieved": attn_gbs, "unit": "GB/s", "peak": peaks["hbm_gbs"],
-         "frac": attn_gbs / peaks["hbm_gbs"] if attn_gbs else None},
-    ]
+    stages = stage_report(w, stage_ms, stage_n, peaks, gather)
     dom = int(np.argmax(stage_ms))
-    traffic = None
+    alg = algorithmic(w)
+    roof = {"kernel": stages[dom]["kernel"], "bound": stages[dom]["bound"],
+            "achieved": stages[dom]["achieved"], "peak": stages[dom]["peak"],
+            "unit": stages[dom]["unit"], "frac": stages[dom]["frac"],
+            "traffic": stages[dom].get("dram_traffic_per_launch"),
+            "algorithmic_per_launch": (alg["attn_bytes"] if dom == 2 else alg["topk_bytes"]
+                                       if dom == 1 else alg["idx_flops"]) / stage_n[dom]}
     if dom == 2:
-        # DRAM bytes per launch of this configuration, from the committed ncu capture (which
-        # covers this workload only)
-        traffic = committed_traffic("indexer_top_gated_b200/csrc/sparse_attn.cuh",
-                                    f"sparse_attn_gated_{w.name}.txt")
-    roof = {"kernel": names[dom], "bound": stages[dom]["bound"], "achieved": stages[dom]["achieved"],
-            "peak": stages[dom]["peak"], "unit": stages[dom]["unit"], "frac": stages[dom]["frac"],
-            "traffic": traffic, "peak_source": f"{peak_src} ({'hbm_gbs' if dom else 'bf16_tflops_sustained'})",
-            "algorithmic_per_launch": (alg["attn_bytes"] if dom == 2 else topk_alg if dom == 1
-                                       else alg["idx_flops"]) / stage_n[dom]}
+        roof["peak_source"] = ("measured live in this run: " + gather["l2"]["best"]
+                               if gather else "not measured (--no-peaks)")
+        roof["dram"] = {"achieved": stages[2]["dram_gbs"], "peak": peaks["hbm_gbs"],
+                        "frac": stages[2]["dram_frac"], "unit": "GB/s",
+                        "peak_source": f"{peak_src} (hbm_gbs)"}
+    else:
+        roof["peak_source"] = f"{peak_src} ({'hbm_gbs' if dom else 'bf16_tflops_sustained'})"
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         c = cpu_oracle_sample(w, args.cpu_seconds)
@@ -556,7 +696,10 @@ def main():
         "config": {"workload": w.name, "batch": w.batch, "seq_len": w.kv_lens[0],
                    "top_k": w.top_k, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
                    "head_dim": w.head_dim, "idx_heads": w.n_idx_heads, "idx_dim": w.idx_dim,
-                   "idx_dtype": w.idx_dtype, "parallelism": f"dp{world} (independent sequences)",
+                   "idx_dtype": w.idx_dtype,
+                   "parallelism": (f"dp{world} (a batch of {world} copies of the workload, "
+                                   f"whole sequences dealt to ranks by cost; no collective "
+                                   f"on the data path)" if world > 1 else "dp1"),
                    "l2": l2_note(w),
                    "workspace_bytes": res["ws_bytes"]},
         "roofline": roof,
@@ -566,6 +709,8 @@ def main():
         "gpu_launches": res["launches"],
         "clocks": res["clocks"],
         "decode": decode,
+        "gather_peaks": gather,
+        "workloads": extra,
     }
     print(json.dumps(line), flush=True)
 

@@ -1,4 +1,6 @@
-"""In-tree build of libdsa.so (the C-ABI library) for sm_100a with nvcc."""
+"""In-tree builds for sm_100a with nvcc: libdsa.so (the C-ABI library of the layer) and
+libdsaprobe.so (the gather-bandwidth measurement kernels the benchmark uses for its
+roofline; not part of the layer)."""
 from __future__ import annotations
 
 import os
@@ -9,6 +11,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libdsa.so")
+PROBE_SRC = os.path.join(PKG, "probe", "gather_peak.cu")
+PROBE_LIB = os.path.join(PKG, "libdsaprobe.so")
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
@@ -42,5 +46,19 @@ def build(force: bool = False, verbose: bool = False) -> str:
     return LIB
 
 
+def build_probe(force: bool = False, verbose: bool = False) -> str:
+    if (not force and os.path.exists(PROBE_LIB)
+            and os.path.getmtime(PROBE_LIB) >= os.path.getmtime(PROBE_SRC)):
+        return PROBE_LIB
+    nvcc = os.environ.get("NVCC", "nvcc")
+    cmd = [nvcc, *NVCC_FLAGS, "-o", PROBE_LIB + ".tmp", PROBE_SRC]
+    if verbose:
+        print(" ".join(cmd))
+    subprocess.check_call(cmd)
+    os.replace(PROBE_LIB + ".tmp", PROBE_LIB)
+    return PROBE_LIB
+
+
 if __name__ == "__main__":
     print(build(force=True, verbose=True))
+    print(build_probe(force=True, verbose=True))
