@@ -99,6 +99,17 @@ typedef struct {
   const int32_t* block_table; /* device [B, max_pages] or NULL                     */
   int32_t max_pages;
   int32_t page_size;
+  /* Host copies of q_offsets and kv_offsets (optional, NULL when not given; the same
+   * values as the device arrays).  With them dsa_prefill and dsa_workspace_size plan per
+   * sequence: in a batch that mixes long query groups (Q_b >= 128, prefill chunks) with
+   * short ones (Q_b < 128, e.g. one new token per sequence), steps 1-2 run over each stretch
+   * of consecutive sequences of one kind with the tiles that suit it -- the fused indexer ->
+   * Top-K over 128-row query tiles for the long groups, key-split score tiles of 16 queries
+   * for the short ones -- and the attention then runs once over all rows.  A serving
+   * scheduler has these lengths on the host already; without them such a batch takes the
+   * score-matrix path planned from the totals above. */
+  const int32_t* q_offsets_host;   /* host [B+1] or NULL */
+  const int32_t* kv_offsets_host;  /* host [B+1] or NULL */
 } dsa_ragged;
 
 /* Layer shape and numerics.  Supported by this build: idx_dim = 64,
@@ -121,7 +132,8 @@ typedef struct {
 /* Human-readable name of a status code (static string). */
 const char* dsa_status_string(dsa_status s);
 
-/* Library ABI version (major*10000 + minor*100 + patch). */
+/* Library ABI version (major*10000 + minor*100 + patch): 102 (dsa_ragged gained the
+ * optional host offsets). */
 int32_t dsa_version(void);
 
 /*
@@ -381,6 +393,12 @@ dsa_status dsa_device_status(void* stream, int32_t* status, int clear);
 
 /* Number of kernels this library has launched from the calling host thread. */
 int64_t dsa_launch_count(void);
+
+/* Number of query rows whose steps 1-2 the calling host thread ran through the fused
+ * indexer -> Top-K path (dsa_index_topk, and the rows dsa_prefill planned that way) since
+ * the last reset; reset != 0 clears the count after reading it.  Lets a caller see which
+ * path a layer call took. */
+int64_t dsa_fused_rows(int reset);
 
 /*
  * Per-stage device timing, for measurement.  While enabled, each stage launch made

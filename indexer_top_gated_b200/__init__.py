@@ -47,6 +47,7 @@ class Ragged(ctypes.Structure):
         ("max_kv_len", ctypes.c_int32), ("total_q", ctypes.c_int64),
         ("total_kv", ctypes.c_int64), ("block_table", ctypes.c_void_p),
         ("max_pages", ctypes.c_int32), ("page_size", ctypes.c_int32),
+        ("q_offsets_host", ctypes.c_void_p), ("kv_offsets_host", ctypes.c_void_p),
     ]
 
 
@@ -70,7 +71,7 @@ EXPORTS = [
     "dsa_device_status", "dsa_launch_count", "dsa_stage_timing", "dsa_stage_times",
     "dsa_decode_noalloc", "dsa_index_topk", "dsa_index_topk_workspace_size",
     "dsa_sparse_attn_gated_mix", "dsa_index_topk_blocks", "dsa_index_topk_blocks_workspace_size",
-    "dsa_prefill_from_host",
+    "dsa_prefill_from_host", "dsa_fused_rows",
 ]
 
 
@@ -102,6 +103,8 @@ def _load():
     L.dsa_device_status.argtypes = [vp, ctypes.POINTER(i32), ctypes.c_int]
     L.dsa_launch_count.argtypes = []
     L.dsa_launch_count.restype = i64
+    L.dsa_fused_rows.argtypes = [ctypes.c_int]
+    L.dsa_fused_rows.restype = i64
     L.dsa_stage_timing.argtypes = [ctypes.c_int]
     L.dsa_stage_times.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64), ctypes.c_int]
     for name in ("dsa_index_scores", "dsa_topk", "dsa_sparse_attn_gated", "dsa_workspace_size",
@@ -160,11 +163,17 @@ def ragged(q_offsets, kv_offsets, q_lens: Sequence[int], kv_lens: Sequence[int],
            block_table=None, page_size: int = 0, cache_rows: Optional[int] = None) -> Ragged:
     """Build a dsa_ragged from device int32 offset tensors and host lengths; with a device
     int32 block table [batch, max_pages] the cache arrays are paged (cache_rows rows).
-    The descriptor holds only the tensors' addresses: keep them alive while it is used."""
+    Host copies of the offsets are made from the lengths and attached (they let the layer
+    plan per sequence).  The descriptor holds only the tensors' addresses: keep them alive
+    while it is used."""
+    import numpy as np
+    qoh = np.concatenate([[0], np.cumsum(np.asarray(q_lens, dtype=np.int64))]).astype(np.int32)
+    koh = np.concatenate([[0], np.cumsum(np.asarray(kv_lens, dtype=np.int64))]).astype(np.int32)
     rg = Ragged(len(q_lens), q_offsets.data_ptr(), kv_offsets.data_ptr(),
                 int(max(q_lens)) if len(q_lens) else 0,
                 int(max(kv_lens)) if len(kv_lens) else 0, int(sum(q_lens)), int(sum(kv_lens)),
-                None, 0, 0)
+                None, 0, 0, qoh.ctypes.data, koh.ctypes.data)
+    rg.host_offsets = (qoh, koh)  # keeps the host copies alive with the descriptor
     if block_table is not None:
         rg.block_table = block_table.data_ptr()
         rg.max_pages = int(block_table.shape[1])
@@ -312,6 +321,10 @@ def dsa_device_status(clear: bool = True, stream=None) -> int:
 
 def dsa_launch_count() -> int:
     return int(lib.dsa_launch_count())
+
+
+def dsa_fused_rows(reset: bool = False) -> int:
+    return int(lib.dsa_fused_rows(int(reset)))
 
 
 def dsa_stage_timing(enable: bool):

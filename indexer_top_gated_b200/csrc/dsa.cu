@@ -13,6 +13,7 @@
 
 #include "dsa.h"
 #include "common.cuh"
+#include "idx_cand.cuh"
 #include "idx_scores.cuh"
 #include "sparse_attn.cuh"
 #include "topk.cuh"
@@ -28,6 +29,7 @@ constexpr int kMaxDevices = 64;
 constexpr int kMaxTopK = 16384;
 
 thread_local int64_t t_launches = 0;
+thread_local int64_t t_fused_rows = 0;  // query rows whose steps 1-2 ran fused
 
 // ---------------------------------------------------------------- stage timing
 struct StageRec {
@@ -151,6 +153,8 @@ dsa_status device_setup(DeviceState** out) {
     e = e ? e : allow_smem(idx_scores_kernel<16, false, kIdxCand>, cand_max);
     e = e ? e : allow_smem(idx_scores_kernel<64, true, kIdxCand>, cand_max);
     e = e ? e : allow_smem(idx_scores_kernel<16, true, kIdxCand>, cand_max);
+    e = e ? e : allow_smem(idx_cand_kernel<false>, idx_cand_smem_bytes(false));
+    e = e ? e : allow_smem(idx_cand_kernel<true>, idx_cand_smem_bytes(true));
     e = e ? e : allow_smem(idx_scores_kernel<64, false, kIdxBlockMax>, cand_max);
     e = e ? e : allow_smem(idx_scores_kernel<16, false, kIdxBlockMax>, cand_max);
     e = e ? e : allow_smem(idx_scores_kernel<64, true, kIdxBlockMax>, cand_max);
@@ -285,6 +289,36 @@ dsa_status launch_index_scores(const DeviceState& dev, const dsa_params* P, cons
   const bool cand = var.thr != nullptr;
   const int mode = cand ? kIdxCand : var.bmax ? kIdxBlockMax : kIdxScores;
   CUtensorMap mq, mk;
+  if (cand && bq > 16) {
+    // query-major candidate pass: 128 query rows per CTA, 64-key tiles, 2 segments per row
+    DSA_TRY(make_idx_map(&mq, q_idx, R->total_q, P->n_idx_heads, fp8, kCandBQ));
+    DSA_TRY(make_idx_map(&mk, k_idx, R->total_kv, P->n_idx_heads, fp8, kCandKT));
+    IdxArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.q_offsets = R->q_offsets;
+    a.kv_offsets = R->kv_offsets;
+    a.batch = R->batch;
+    a.n_heads = P->n_idx_heads;
+    a.q_begin = q_begin;
+    a.q_count = q_count;
+    a.n_tiles = (int)((q_count + kCandBQ - 1) / kCandBQ);
+    a.w = w;
+    a.w_row_stride = P->w_row_stride;
+    a.scale = P->idx_scale_q * P->idx_scale_k;
+    a.status = dev.status;
+    a.pages = cache_pages(R);
+    a.thr = var.thr;
+    a.cand = var.cand;
+    a.cap = var.cap;
+    a.cand_cnt = var.cand_cnt;
+    StageScope scope(0, stream);
+    if (fp8)
+      idx_cand_kernel<true><<<a.n_tiles, kCandThreads, idx_cand_smem_bytes(true), stream>>>(mq, mk, a);
+    else
+      idx_cand_kernel<false><<<a.n_tiles, kCandThreads, idx_cand_smem_bytes(false), stream>>>(mq, mk, a);
+    ++t_launches;
+    return launch_status("idx_cand_kernel");
+  }
   DSA_TRY(make_idx_map(&mq, q_idx, R->total_q, P->n_idx_heads, fp8, bq));
   if (var.shift)
     DSA_TRY(make_idx_map(&mk, var.k_rows, var.k_rows_n, P->n_idx_heads, fp8, kIdxKeyTile));
@@ -479,6 +513,7 @@ dsa_status fused_pass(const DeviceState& dev, const dsa_params* P, const dsa_rag
   if (q_count == 0) return DSA_OK;
   const int bq = R->max_q_len <= 16 ? 16 : 64;
   float* samp = reinterpret_cast<float*>(f.sc);
+  t_fused_rows += q_count;
   {  // (1) sampled scores
     IdxVariant v;
     v.shift = kSampleShift;
@@ -529,6 +564,7 @@ dsa_status fused_pass(const DeviceState& dev, const dsa_params* P, const dsa_rag
   a.cnt = cnt;
   a.cand = reinterpret_cast<const float2*>(f.sc);
   a.cap = g.cap;
+  a.cand_segs = bq > 16 ? kCandSegs : 4;  // query-major pass : row-major pass
   a.cand_cnt = f.ccnt;
   a.fb_list = f.list;
   a.q_idx = q_idx;
@@ -642,6 +678,56 @@ bool plan_passes(int64_t total_q, int64_t srow, int64_t irow, int64_t ws, int nu
   return true;
 }
 
+dsa_status run_index(const DeviceState& dev, const dsa_params* P, const dsa_ragged* R,
+                     const void* q_idx, const void* k_idx, const float* w, int64_t a0, int64_t a1,
+                     int32_t* idx, void* ws, size_t ws_bytes, cudaStream_t stream, int fused,
+                     int bq);
+
+// ---------------------------------------------------------------- per-sequence planning
+//
+// With host copies of the offsets the layer sees each sequence's shape.  A stretch of
+// consecutive sequences of one kind -- long query groups (prefill chunks, Q_b >= kLongQ) or
+// short ones (decode tokens) -- is one contiguous range of packed query rows.
+constexpr int kLongQ = 128;
+
+struct RowRun {
+  int64_t a0, a1;  // packed query rows
+  bool lng;        // sequences with Q_b >= kLongQ
+  int max_q;       // longest query group in the stretch
+};
+
+// Stretches of the batch within rows [row0, row1); empty without host offsets.
+std::vector<RowRun> row_runs(const dsa_ragged* R, int64_t row0, int64_t row1) {
+  std::vector<RowRun> runs;
+  const int32_t* qo = R->q_offsets_host;
+  if (!qo) return runs;
+  for (int b = 0; b < R->batch; ++b) {
+    const int64_t s0 = std::max<int64_t>(qo[b], row0), s1 = std::min<int64_t>(qo[b + 1], row1);
+    if (s1 <= s0) continue;
+    const int q = qo[b + 1] - qo[b];
+    const bool lng = q >= kLongQ;
+    if (!runs.empty() && runs.back().lng == lng && runs.back().a1 == s0) {
+      runs.back().a1 = s1;
+      runs.back().max_q = std::max(runs.back().max_q, q);
+    } else {
+      runs.push_back({s0, s1, lng, q});
+    }
+  }
+  return runs;
+}
+
+bool mixed_runs(const std::vector<RowRun>& runs) {
+  bool l = false, sh = false;
+  for (const RowRun& r : runs) (r.lng ? l : sh) = true;
+  return l && sh;
+}
+
+// Score rows of one materialised sub-pass over `rows` query rows (as plan_passes).
+int64_t score_pass_rows(int64_t rows, int64_t srow) {
+  return std::max<int64_t>(1, std::min(rows, std::max<int64_t>(kScorePassBytes / srow,
+                                                                 std::min<int64_t>(rows, 148))));
+}
+
 dsa_status run_layer(const dsa_params* P, const dsa_ragged* R, const void* q_idx,
                      const void* k_idx, const float* w, const void* q, const void* k,
                      const void* v, const void* gate, void* out, int32_t* idx_out,
@@ -670,6 +756,23 @@ dsa_status run_layer(const dsa_params* P, const dsa_ragged* R, const void* q_idx
   if (!plan_passes(n_rows, ld * 4, irow, (int64_t)ws_bytes, dev->num_sms, &plan))
     return DSA_ERR_WORKSPACE;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  if (!decode) {
+    // a batch mixing prefill chunks with short query groups: steps 1-2 per stretch with the
+    // tiles that suit it, then one attention launch over every row
+    const std::vector<RowRun> runs = row_runs(R, row0, row1);
+    const int64_t idx_bytes = idx_out ? 0 : round_up(n_rows * K * 4, 256);
+    if (mixed_runs(runs) && (int64_t)ws_bytes >= idx_bytes + ld * 4) {
+      int32_t* idx_all = idx_out ? idx_out + row0 * K : static_cast<int32_t*>(ws);
+      void* scratch = static_cast<char*>(ws) + idx_bytes;
+      const size_t sb = ws_bytes - (size_t)idx_bytes;
+      for (const RowRun& r : runs)
+        DSA_TRY(run_index(*dev, P, R, q_idx, k_idx, w, r.a0, r.a1, idx_all + (r.a0 - row0) * K,
+                          scratch, sb, stream, r.lng ? 1 : 0,
+                          r.lng ? 64 : (r.max_q <= 16 ? 16 : 64)));
+      return launch_attn(*dev, P, R, q, k, v, idx_all, K, row0, n_rows, gate, out, nullptr,
+                         err_count, stream);
+    }
+  }
   FusedGeom fg;
   if (!decode && fused_wanted(P, R, &fg)) {
     // fused indexer -> Top-K, in passes of as many rows as the workspace holds (with their
@@ -712,15 +815,18 @@ dsa_status run_layer(const dsa_params* P, const dsa_ragged* R, const void* q_idx
 }
 
 // Steps 1-2 alone for rows [a0, a1): index rows into idx (row r at idx + (r - a0) * K), in
-// passes sized to the workspace (fused indexer -> Top-K when dsa_prefill would take it).
+// passes sized to the workspace.  fused: -1 as dsa_prefill decides for the whole batch, 1 the
+// fused indexer -> Top-K whenever it supports the problem and the workspace holds enough
+// rows, 0 never.  bq: query rows per score tile (16 or 64; 0: from max_q_len).
 dsa_status run_index(const DeviceState& dev, const dsa_params* P, const dsa_ragged* R,
                      const void* q_idx, const void* k_idx, const float* w, int64_t a0, int64_t a1,
-                     int32_t* idx, void* ws, size_t ws_bytes, cudaStream_t stream) {
+                     int32_t* idx, void* ws, size_t ws_bytes, cudaStream_t stream, int fused = -1,
+                     int bq = 0) {
   const int64_t n_rows = a1 - a0;
   if (n_rows <= 0) return DSA_OK;
   const int64_t K = P->top_k;
   FusedGeom fg;
-  if (fused_wanted(P, R, &fg)) {
+  if (fused < 0 ? fused_wanted(P, R, &fg) : fused > 0 && fused_geom(P, R, &fg)) {
     const int64_t rows = std::min<int64_t>(n_rows, fused_rows(fg, (int64_t)ws_bytes));
     if (rows >= std::min<int64_t>(n_rows, kFusedMinRows)) {
       const FusedWs f = fused_carve(fg, ws, rows);
@@ -738,7 +844,7 @@ dsa_status run_index(const DeviceState& dev, const dsa_params* P, const dsa_ragg
                                      std::max<int64_t>(kScorePassBytes / (ld * 4), 1));
   if (rows_s < 1) return DSA_ERR_WORKSPACE;
   float* scores = static_cast<float*>(ws);
-  const int bq = R->max_q_len <= 16 ? 16 : 64;
+  if (bq == 0) bq = R->max_q_len <= 16 ? 16 : 64;
   for (int64_t s0 = a0; s0 < a1; s0 += rows_s) {
     const int64_t n = std::min<int64_t>(rows_s, a1 - s0);
     DSA_TRY(launch_index_scores(dev, P, R, q_idx, k_idx, w, s0, n, scores, ld, bq, stream));
@@ -766,7 +872,7 @@ const char* dsa_status_string(dsa_status s) {
   return "unknown status";
 }
 
-int32_t dsa_version(void) { return 101; }
+int32_t dsa_version(void) { return 102; }
 
 dsa_status dsa_index_scores(const dsa_params* P, const dsa_ragged* R, const void* q_idx,
                             const void* k_idx, const float* w, int64_t q_begin, int64_t q_count,
@@ -846,6 +952,19 @@ dsa_status dsa_workspace_size(const dsa_params* P, const dsa_ragged* R, int is_d
   const int64_t irow = round_up((int64_t)P->top_k * 4, 16);
   if (min_bytes) *min_bytes = (size_t)(srow + irow);
   FusedGeom fg;
+  const std::vector<RowRun> runs = is_decode ? std::vector<RowRun>() : row_runs(R, 0, R->total_q);
+  if (rec_bytes && mixed_runs(runs)) {
+    // index rows of every row, plus the largest stretch's steps 1-2 in one pass
+    int64_t need = 0;
+    const bool can_fuse = fused_geom(P, R, &fg);
+    for (const RowRun& r : runs) {
+      const int64_t n = r.a1 - r.a0;
+      need = std::max(need, r.lng && can_fuse ? fg.fixed_bytes + 256 + n * fg.row_bytes
+                                              : score_pass_rows(n, srow) * srow);
+    }
+    *rec_bytes = (size_t)(round_up(R->total_q * irow, 256) + need);
+    return DSA_OK;
+  }
   if (rec_bytes && !is_decode && fused_wanted(P, R, &fg)) {
     // one fused pass over every query row
     *rec_bytes = (size_t)(fg.fixed_bytes + 256 + std::max<int64_t>(1, R->total_q) * (fg.row_bytes + irow));
@@ -1122,7 +1241,7 @@ dsa_status dsa_prefill_from_host(const dsa_params* P, const dsa_ragged* R,
         cudaStreamWaitEvent(st, ev_idx, 0) != cudaSuccess)
       return DSA_ERR_CUDA;
     DSA_TRY(run_index(*d, P, &Rd, dev->q_idx, dev->k_idx, dev->w, 0, TQ, idx_all, scratch,
-                      (size_t)((int64_t)ws_bytes - idx_bytes), st));
+                      (size_t)((int64_t)ws_bytes - idx_bytes), st, -1, 0));
     for (int c = 0; c < n_chunks; ++c) {
       const int64_t a0 = TQ * c / n_chunks, a1 = TQ * (c + 1) / n_chunks;
       if (a0 == a1) continue;
@@ -1271,6 +1390,12 @@ dsa_status dsa_device_status(void* stream, int32_t* status, int clear) {
 }
 
 int64_t dsa_launch_count(void) { return t_launches; }
+
+int64_t dsa_fused_rows(int reset) {
+  const int64_t n = t_fused_rows;
+  if (reset) t_fused_rows = 0;
+  return n;
+}
 
 dsa_status dsa_stage_timing(int enable) {
   t_timing = enable != 0;

@@ -1,0 +1,384 @@
+// idx_cand.cuh - the candidate pass of the fused indexer -> Top-K path, query-major.
+//
+//   s[t, j] = sum_h w_h * max(0, c * q_idx[t,h,:] . k_idx[j,h,:]),   j = 0..p(t)
+//
+// keeping only the (position, score) pairs with s >= thr[t] (the row's sampled threshold).
+// Same scores as idx_scores_kernel, laid out the other way round on the tensor core:
+//  - One CTA owns 128 consecutive packed query rows and every key tile they can see (so it
+//    owns their candidate lists).  The query tile is the MMA's M side: TMEM lane = query
+//    row, columns = keys (64 per tile and head), so each epilogue thread owns one query row.
+//    The ReLU-weighted head sum, the threshold compare and the candidate emission are then
+//    private to the thread: no transposition, no shuffles, no shared counters.
+//  - Warp 0 issues TMA loads (128-byte swizzle, one box per indexer head; the query tile
+//    once, then a 3-stage ring of key tiles); warp 1 issues tcgen05.mma (A = query tile,
+//    B = key tile, one UMMA per head and K step) into one of two TMEM buffers of 4 x 64
+//    columns; warps 2-9 drain TMEM: the two warps of a lane quadrant take 32 key columns
+//    each (segment sub = 0 or 1 of the row's candidate list).
+//  - A thread appends its hits to a small staging area of its own in shared memory and
+//    writes them to its segment in whole 32-byte sectors (4 pairs), so the candidate stream
+//    leaves the SM in full sectors instead of one scattered 8-byte store per hit.
+//  - The TMEM buffer is released as soon as its four heads are in registers, before the
+//    emission, so the MMAs of the next tiles overlap it.
+// Tiles may straddle sequences of a ragged batch (one pass per sequence, other rows masked
+// by an infinite threshold).  Every wait is bounded; on a timeout the CTA records it, waits
+// (bounded) for its own copies and MMAs in flight, frees TMEM and returns.
+#pragma once
+
+#include "common.cuh"
+#include "idx_scores.cuh"
+
+namespace dsa {
+
+constexpr int kCandBQ = 128;       // query rows per CTA (MMA M, TMEM lanes)
+constexpr int kCandKT = 64;        // keys per tile (MMA N)
+constexpr int kCandStages = 3;     // key-tile ring depth
+constexpr int kCandEpiWarps = 8;   // two per TMEM lane quadrant
+constexpr int kCandThreads = 64 + 32 * kCandEpiWarps;
+constexpr int kCandSegs = 2;       // candidate segments per row (one per key half of a tile)
+constexpr int kCandSlots = 22;     // staging slots (8-byte pairs) per (row, segment)
+constexpr int kCandSlotStride = kCandSlots * 8;  // 176 B: 16-byte aligned, banks spread by row
+
+template <bool FP8>
+__host__ __device__ constexpr size_t cand_q_bytes() { return (size_t)4 * kCandBQ * (FP8 ? 64 : 128); }
+template <bool FP8>
+__host__ __device__ constexpr size_t cand_k_stage_bytes() { return (size_t)4 * kCandKT * (FP8 ? 64 : 128); }
+
+__host__ inline size_t idx_cand_smem_bytes(bool fp8) {
+  const size_t q = fp8 ? cand_q_bytes<true>() : cand_q_bytes<false>();
+  const size_t k = kCandStages * (fp8 ? cand_k_stage_bytes<true>() : cand_k_stage_bytes<false>());
+  size_t bytes = 1024 /*align*/ + q + k + 256 /*barriers*/ +
+                 (size_t)kCandSegs * kCandBQ * kCandSlotStride;
+  // the CTA takes all 512 TMEM columns: ask for enough shared memory that no second CTA
+  // can share the SM (an allocation that cannot be met would block)
+  if (bytes < 120 * 1024) bytes = 120 * 1024;
+  return bytes;
+}
+
+template <bool FP8>
+__global__ void __launch_bounds__(kCandThreads, 1)
+    idx_cand_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                    const __grid_constant__ CUtensorMap tmap_k, IdxArgs a) {
+  using Geo = IdxGeom<FP8>;
+  constexpr uint32_t kQHead = kCandBQ * Geo::kRowBytes;  // one head of the query tile
+  constexpr uint32_t kKHead = kCandKT * Geo::kRowBytes;  // one head of a key tile
+  constexpr int ST = kCandStages;
+  constexpr int kCols = 2 * 4 * kCandKT;                 // TMEM columns (2 buffers x 4 heads)
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + 4 * kQHead;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sK + (size_t)ST * 4 * kKHead);
+  uint64_t* full = bars;            // [ST]
+  uint64_t* empty = bars + ST;      // [ST]
+  uint64_t* tfull = bars + 2 * ST;  // [2]
+  uint64_t* tempty = tfull + 2;     // [2]
+  uint64_t* qfull = tempty + 2;     // [1]
+  uint8_t* stage_base = reinterpret_cast<uint8_t*>(bars) + 256;  // [segs][128 rows][slots]
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_bfirst, s_blast;
+  __shared__ volatile int s_abort;
+  __shared__ int s_consumed;
+
+  const int H = a.n_heads;
+  const int warp = threadIdx.x >> 5;
+  const int lane = lane_id();
+  const int tile = a.n_tiles - 1 - (int)blockIdx.x;  // largest first
+  const int64_t r0 = a.q_begin + (int64_t)tile * kCandBQ;
+  const int64_t q_end = a.q_begin + a.q_count;
+  const int64_t r_last = (r0 + kCandBQ < q_end ? r0 + kCandBQ : q_end) - 1;
+
+  if (threadIdx.x == 0) {
+    s_bfirst = seq_of_row(a.q_offsets, a.batch, r0);
+    s_blast = seq_of_row(a.q_offsets, a.batch, r_last);
+    s_abort = 0;
+    s_consumed = 0;
+  }
+  __syncthreads();
+  const int b_first = s_bfirst, b_last = s_blast;
+
+  // rows rs..re-1 of the tile belong to sequence b; its key tiles are 0..kt_hi-1
+  auto seq_range = [&](int b, int64_t& rs, int64_t& re, int& kt_hi, int64_t& pbase) -> bool {
+    const int64_t qo = __ldg(a.q_offsets + b), qn = __ldg(a.q_offsets + b + 1);
+    const int64_t ko = __ldg(a.kv_offsets + b), kn = __ldg(a.kv_offsets + b + 1);
+    rs = r0 > qo ? r0 : qo;
+    re = (r_last + 1) < qn ? (r_last + 1) : qn;
+    if (rs >= re) return false;
+    pbase = (kn - ko) - (qn - qo) - qo;  // p(r) = pbase + r
+    const int64_t pmax = pbase + re - 1;
+    if (pmax < 0) return false;
+    kt_hi = (int)(pmax / kCandKT) + 1;
+    return true;
+  };
+
+  int n_jobs = 0;
+  for (int b = b_first; b <= b_last; ++b) {
+    int64_t rs, re, pb;
+    int kh;
+    if (seq_range(b, rs, re, kh, pb)) n_jobs += kh;
+  }
+  if (n_jobs == 0) {  // uniform across the CTA
+    for (int c = threadIdx.x; c < 4 * kCandBQ; c += blockDim.x)
+      if (r0 + c / 4 <= r_last) a.cand_cnt[(r0 - a.q_begin) * 4 + c] = 0;
+    return;
+  }
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&tfull[i]), 1);
+      mbar_init(smem_u32(&tempty[i]), kCandEpiWarps);
+    }
+    mbar_init(smem_u32(qfull), 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&s_tmem), (uint32_t)kCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmap_q);
+      prefetch_tensormap(&tmap_k);
+      mbar_arrive_expect_tx(smem_u32(qfull), H * kQHead);
+      for (int h = 0; h < H; ++h)
+        tma_load_2d(smem_u32(sQ + h * kQHead), &tmap_q, smem_u32(qfull), h * 64, (int)r0);
+      int i = 0;
+      bool ok = true;
+      for (int b = b_first; b <= b_last && ok; ++b) {
+        int64_t rs, re, pb;
+        int kh;
+        if (!seq_range(b, rs, re, kh, pb)) continue;
+        const int64_t kbase = __ldg(a.kv_offsets + b);
+        for (int kt = 0; kt < kh; ++kt, ++i) {
+          // a 64-key tile never straddles a page (pages are multiples of 128 positions)
+          const int64_t krow = a.pages.table ? cache_row(a.kv_offsets, a.pages, b, (int64_t)kt * kCandKT)
+                                             : kbase + (int64_t)kt * kCandKT;
+          const int s = i % ST;
+          if (!mbar_wait_bounded(smem_u32(&empty[s]), ((i / ST) & 1) ^ 1, a.status, &s_abort)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(smem_u32(&full[s]), H * kKHead);
+          for (int h = 0; h < H; ++h)
+            tma_load_2d(smem_u32(sK + ((size_t)s * 4 + h) * kKHead), &tmap_k, smem_u32(&full[s]),
+                        h * 64, (int)krow);
+        }
+      }
+      if (!ok) {
+        mbar_wait_bounded(smem_u32(qfull), 0, nullptr, nullptr);
+        for (int j = s_consumed; j < i; ++j)
+          mbar_wait_bounded(smem_u32(&full[j % ST]), (j / ST) & 1, nullptr, nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t idesc = umma_idesc(kCandBQ, kCandKT, FP8 ? 0u : 1u);
+    int i = 0, issued = 0;
+    bool ok = mbar_wait_bounded(smem_u32(qfull), 0, a.status, &s_abort);
+    for (int b = b_first; b <= b_last && ok; ++b) {
+      int64_t rs, re, pb;
+      int kh;
+      if (!seq_range(b, rs, re, kh, pb)) continue;
+      for (int kt = 0; kt < kh; ++kt, ++i) {
+        const int s = i % ST, buf = i & 1;
+        if (!mbar_wait_bounded(smem_u32(&full[s]), (i / ST) & 1, a.status, &s_abort) ||
+            !mbar_wait_bounded(smem_u32(&tempty[buf]), ((i >> 1) & 1) ^ 1, a.status, &s_abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          for (int h = 0; h < H; ++h) {
+            const uint32_t a_base = smem_u32(sQ + h * kQHead);
+            const uint32_t b_base = smem_u32(sK + ((size_t)s * 4 + h) * kKHead);
+            const uint32_t d = tmem + (uint32_t)(buf * 4 * kCandKT + h * kCandKT);
+#pragma unroll
+            for (int kk = 0; kk < Geo::kKSteps; ++kk) {
+              const uint64_t ad = umma_smem_desc(a_base + kk * 32, Geo::kSbo, Geo::kLayout);
+              const uint64_t bd = umma_smem_desc(b_base + kk * 32, Geo::kSbo, Geo::kLayout);
+              if (FP8) umma_fp8(d, ad, bd, idesc, kk > 0);
+              else umma_bf16(d, ad, bd, idesc, kk > 0);
+            }
+          }
+          umma_commit(smem_u32(&empty[s]));
+          umma_commit(smem_u32(&tfull[buf]));
+        }
+        __syncwarp();
+        issued = i + 1;
+        if (lane == 0) s_consumed = i + 1;
+      }
+    }
+    if (!ok && issued > 0 && lane == 0) {
+      const int j = issued - 1;  // the last commit completes after every earlier MMA
+      mbar_wait_bounded(smem_u32(&tfull[j & 1]), (j >> 1) & 1, nullptr, nullptr);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2-9)
+    const int quad = warp & 3;          // TMEM lanes 32 quad .. 32 quad + 31
+    const int sub = (warp - 2) >> 2;    // key columns 32 sub .. 32 sub + 31 of each tile
+    const int rr = quad * 32 + lane;    // this thread's row within the tile
+    const int64_t row = r0 + rr;
+    const bool in_launch = row <= r_last;
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    // shared head weights with the (positive) dequantisation scale folded in:
+    // w * max(0, c * x) = (w * c) * max(0, x) for c > 0; per-row weights take c on the dot
+    float wsh[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      if (h >= H) wsh[h] = 0.f;
+      else if (a.w_row_stride == 0) wsh[h] = __ldg(a.w + h) * a.scale;
+      else wsh[h] = in_launch ? __ldg(a.w + row * a.w_row_stride + h) : 0.f;
+    }
+    const bool row_w = a.w_row_stride != 0;
+    const float thr_row = in_launch ? __ldg(a.thr + (row - a.q_begin)) : INFINITY;
+    const int seg = a.cap / kCandSegs;
+    float2* dst = a.cand + (in_launch ? (row - a.q_begin) : 0) * (int64_t)a.cap + sub * seg;
+    uint8_t* stg = stage_base + ((size_t)sub * kCandBQ + rr) * kCandSlotStride;
+    uint32_t cnt = 0;      // hits so far (may exceed seg: the selection then falls back)
+    uint32_t written = 0;  // pairs moved to global memory (multiple of 4 until the tail)
+    uint32_t pend = 0;     // pairs waiting in the staging slots 0 .. pend-1
+
+    // write every complete group of 4 pending pairs (whole 32-byte sectors) and move the
+    // rest (< 4) to the front of the staging area
+    auto flush = [&]() {
+      const uint32_t groups = pend >> 2;
+#pragma unroll
+      for (uint32_t g = 0; g < 5; ++g) {
+        if (g < groups) {
+          const float4 x0 = *reinterpret_cast<const float4*>(stg + g * 32);
+          const float4 x1 = *reinterpret_cast<const float4*>(stg + g * 32 + 16);
+          if (written + 4 * g + 4 <= (uint32_t)seg) {
+            float4* d4 = reinterpret_cast<float4*>(dst + written + 4 * g);
+            d4[0] = x0;
+            d4[1] = x1;
+          }
+        }
+      }
+      const uint32_t rest = pend & 3u;
+      if (groups > 0) {
+#pragma unroll
+        for (uint32_t t = 0; t < 3; ++t)
+          if (t < rest)
+            *reinterpret_cast<float2*>(stg + t * 8) =
+                *reinterpret_cast<const float2*>(stg + (groups * 4 + t) * 8);
+      }
+      written += groups * 4;
+      pend = rest;
+    };
+
+    int i = 0;
+    bool ok = true;
+    for (int b = b_first; b <= b_last && ok; ++b) {
+      int64_t rs, re, pbase;
+      int kh;
+      if (!seq_range(b, rs, re, kh, pbase)) continue;
+      const bool in_seq = row >= rs && row < re;
+      const float thr = in_seq ? thr_row : INFINITY;  // rows of other sequences keep nothing
+      const int prow = in_seq ? (int)(pbase + row) : -1;
+      // the warp's rows are all in this sequence and its first row sees every key of a
+      // chunk that ends at or below p_min: such chunks need no causal compare
+      const int p_min = (int)(pbase + r0 + quad * 32);
+      const bool warp_in_seq = r0 + quad * 32 >= rs && r0 + quad * 32 + 31 < re;
+      for (int kt = 0; kt < kh; ++kt, ++i) {
+        const int buf = i & 1;
+        if (!mbar_wait_bounded(smem_u32(&tfull[buf]), (i >> 1) & 1, a.status, &s_abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tbase = tmem + lane_base + (uint32_t)(buf * 4 * kCandKT + sub * 32);
+        float acc[32];
+        {
+          uint32_t v[2][32];
+#pragma unroll
+          for (int hp = 0; hp < 4; hp += 2) {
+            if (hp >= H) break;
+            tmem_ld32_async(tbase + (uint32_t)(hp * kCandKT), v[0]);
+            if (hp + 1 < H) tmem_ld32_async(tbase + (uint32_t)((hp + 1) * kCandKT), v[1]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const int h = hp + q;
+              if (h >= H) break;
+              reg_fence(v[q]);
+              if (!row_w) {
+                const float2 w2 = make_float2(wsh[h], wsh[h]);
+#pragma unroll
+                for (int c = 0; c < 32; c += 2) {
+                  const float2 x = make_float2(fmaxf(__uint_as_float(v[q][c]), 0.f),
+                                               fmaxf(__uint_as_float(v[q][c + 1]), 0.f));
+                  const float2 prev = h == 0 ? make_float2(0.f, 0.f) : make_float2(acc[c], acc[c + 1]);
+                  const float2 r2 = __ffma2_rn(w2, x, prev);
+                  acc[c] = r2.x;
+                  acc[c + 1] = r2.y;
+                }
+              } else {
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                  acc[c] = fmaf(wsh[h], fmaxf(__uint_as_float(v[q][c]) * a.scale, 0.f),
+                                h == 0 ? 0.f : acc[c]);
+              }
+            }
+          }
+        }
+        // the four heads are in registers: hand the TMEM buffer back to the MMA warp
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&tempty[buf]));
+
+        const int j0 = kt * kCandKT + sub * 32;  // position of key column 0
+        const bool interior = __all_sync(0xFFFFFFFFu, warp_in_seq && j0 + 31 <= p_min);
+        const int lim = prow - j0;               // keys k <= lim are visible to this row
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          float2* p = reinterpret_cast<float2*>(stg) + pend;
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int k = half * 16 + c;
+            const bool hit = acc[k] >= thr && (interior || k <= lim);
+            if (hit) {
+              *p = make_float2(__int_as_float(j0 + k), acc[k]);
+              ++p;
+            }
+          }
+          const uint32_t now = (uint32_t)(p - reinterpret_cast<float2*>(stg));
+          cnt += now - pend;
+          pend = now;
+          if (pend >= 4) flush();
+        }
+      }
+    }
+    // tail: the last (< 4) pending pairs, one by one
+    if (in_launch) {
+#pragma unroll
+      for (uint32_t t = 0; t < 3; ++t)
+        if (t < pend && written + t < (uint32_t)seg)
+          dst[written + t] = *reinterpret_cast<const float2*>(stg + t * 8);
+      int32_t* cc = a.cand_cnt + (row - a.q_begin) * 4;
+      cc[sub] = (int32_t)cnt;
+      if (sub == 0) {
+        cc[2] = 0;
+        cc[3] = 0;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, (uint32_t)kCols);
+  }
+}
+
+}  // namespace dsa

@@ -37,7 +37,8 @@ def gather_rate(buf_bytes: int, variant: int, blocks: int, chunks_per_warp: int 
     rows = buf_bytes // 256
     assert rows > 0 and rows & (rows - 1) == 0
     buf = torch.zeros(buf_bytes // 2, dtype=torch.int16, device="cuda")
-    n_idx = 1 << 22
+    # one index per row read, none reused within a launch (a reused row could hit in L2)
+    n_idx = 1 << max(22, (blocks * 8 * chunks_per_warp * 32 - 1).bit_length())
     idx = torch.empty(n_idx, dtype=torch.int32, device="cuda")
     sink = torch.empty(blocks * 256 * 4, dtype=torch.int32, device="cuda")
     torch.cuda.synchronize()

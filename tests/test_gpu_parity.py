@@ -399,3 +399,22 @@ def test_full_size_discrimination():
         assert not PT.close_report(PT.bf16_tensor_to_f64(nogate[r]), out_ref)["ok"], r
     del dev, idx, out
     torch.cuda.empty_cache()
+
+
+def test_mixed_batch_runs_prefill_chunks_fused_and_decode_rows_materialised():
+    """A batch of prefill chunks and single decode queries (the serving layout), with host
+    offsets: the chunks' rows take the fused indexer -> Top-K, the decode rows score tiles of
+    16 queries, one attention launch covers all; every row matches the oracle."""
+    q_lens = [300, 1, 1, 640, 1, 1, 1, 200] + [1] * 9
+    kv_lens = [2500, 3000, 5, 4000, 129, 6000, 4097, 900] + [700 + 311 * i for i in range(9)]
+    w = _workload(q_lens, kv_lens, K=256)
+    host = S.make_host_inputs(w)
+    dev = _dev(host)
+    dsa.dsa_fused_rows(reset=True)
+    idx, out = _run_layer(w, dev)
+    fused = dsa.dsa_fused_rows(reset=True)
+    assert fused == sum(q for q in q_lens if q >= 128)
+    rows = list(range(w.total_q))
+    idx_ref, out_ref, _ = O.Oracle.for_workload(w, host).layer_rows(rows)
+    np.testing.assert_array_equal(idx.cpu().numpy(), idx_ref)
+    PT.assert_close(PT.bf16_tensor_to_f64(out), out_ref, "mixed batch")

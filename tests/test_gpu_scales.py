@@ -114,7 +114,8 @@ def test_index_scores_power_of_two_scales_bitexact(dtype, stride, sq, sk):
 def test_index_scores_non_dyadic_scale_within_rounding(stride):
     """c = 0.3 * 1.7 rounds in fp32: every term w_h max(0, c x_h) is >= 0, so the score's
     own magnitude bounds the rounding of its few products and fused adds (5 roundings of
-    2^-24 relative each at most; 1e-6 relative is checked)."""
+    2^-24 relative each at most; 1e-6 relative is checked).  Where the exact score is 0 the
+    oracle's fp64 product of scaled operands leaves a residue of ~1e-17: 1e-12 absolute."""
     w = _wl([200, 77], [600, 900])
     host = S.make_host_inputs(w)
     if stride:
@@ -125,8 +126,10 @@ def test_index_scores_non_dyadic_scale_within_rounding(stride):
     for r in range(w.total_q):
         ref = orc.index_scores_row(r)
         err = np.abs(got[r, : len(ref)].astype(np.float64) - ref)
-        assert np.all(err <= 1e-6 * ref + 1e-30), f"row {r}: {err.max()}"
-        worst = max(worst, float(np.max(err / np.maximum(ref, 1e-30))))
+        bad = err > 1e-6 * ref + 1e-12
+        assert not np.any(bad), f"row {r}: {err[bad][:4]} at ref {ref[bad][:4]}"
+        big = ref > 1e-6
+        worst = max(worst, float(np.max(err[big] / ref[big], initial=0.0)))
     # a squared or dropped scale would be off by a factor 0.51 or 1/0.51
     assert worst < 1e-6
 
@@ -208,12 +211,15 @@ def test_topk_non_dyadic_scale_is_a_valid_selection():
 @pytest.mark.parametrize("decode", [False, True])
 def test_layer_with_scales_matches_oracle(decode):
     """Whole layer with idx scales (0.5, 4) and attn_scale 0.2 against the oracle with the
-    same parameters (q, k ~ N(0,1) so the logit scale shapes the softmax)."""
+    same parameters.  q and k ~ N(0,1) so that the logit scale shapes the softmax (logits
+    of standard deviation ~2.3); v and the gate keep the configurations' distributions."""
     if decode:
-        w = _wl([1] * 6, [1, 300, 129, 2048, 3000, 777], K=256, Hq=16, Hkv=2, scale=1.0)
+        w = _wl([1] * 6, [1, 300, 129, 2048, 3000, 777], K=256, Hq=16, Hkv=2)
     else:
-        w = _wl([400, 90], [400, 1000], K=128, Hq=16, Hkv=2, scale=1.0)
+        w = _wl([400, 90], [400, 1000], K=128, Hq=16, Hkv=2)
     host = S.make_host_inputs(w)
+    host["q"] = S.host_bf16(host["q"].size, S.NORMAL, 7, S.T_Q, 0, 1.0).reshape(host["q"].shape)
+    host["k"] = S.host_bf16(host["k"].size, S.NORMAL, 7, S.T_K, 0, 1.0).reshape(host["k"].shape)
     dev = _dev(host)
     shape = _shape(w, 0.5, 4.0, attn_scale=0.2)
     rg = dsa.ragged(dev["q_offsets"], dev["kv_offsets"], w.q_lens, w.kv_lens)

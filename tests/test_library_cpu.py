@@ -140,7 +140,7 @@ def test_paged_cache_descriptor_is_validated():
     rg = dsa.Ragged(1, 0x1000, 0x2000, 8, 500, 8, 1024, A, 4, 128)
     mn, rec = dsa.dsa_workspace_size(dsa.LayerShape(top_k=4), rg)
     assert 0 < mn <= rec
-    assert L.dsa_version() == 101
+    assert L.dsa_version() == 102
 
 
 def test_block_selection_arguments():
@@ -203,3 +203,33 @@ def test_fused_index_topk_workspace_and_limits():
     assert L.dsa_index_topk(*args(A, mn, ld=2047)) == dsa.DSA_ERR_INVALID_ARG
     assert L.dsa_index_topk(*args(A, mn, q0=32768)) == dsa.DSA_ERR_INVALID_ARG
     assert L.dsa_index_topk(*args(A, mn, qn=0)) == 0  # nothing to do
+
+
+def test_mixed_batch_workspace_plan_uses_host_offsets():
+    """With host copies of the offsets, a batch mixing prefill chunks and single queries is
+    planned per stretch of sequences: the recommended workspace holds every row's index row
+    plus the largest stretch's steps 1-2 (host-side sizing only, no device access)."""
+    import numpy as np
+
+    import dsa_synth as S
+    import indexer_top_gated_b200 as dsa
+
+    w = S.workload("mixed_serving")
+    shape = dsa.workload_shape(w)
+    qoh = w.q_offsets.astype(np.int32)
+    koh = w.kv_offsets.astype(np.int32)
+    base = (w.batch, 0x1000, 0x2000, max(w.q_lens), max(w.kv_lens), w.total_q, w.total_kv,
+            None, 0, 0)
+    plain = dsa.Ragged(*base)
+    planned = dsa.Ragged(*base, qoh.ctypes.data, koh.ctypes.data)
+    mn0, rec0 = dsa.dsa_workspace_size(shape, plain)
+    mn1, rec1 = dsa.dsa_workspace_size(shape, planned)
+    assert mn0 == mn1
+    assert rec1 != rec0 and rec1 >= w.total_q * w.top_k * 4
+    # a batch of one kind is planned as before
+    one = S.workload("prefill_t32768_k2048")
+    q1 = one.q_offsets.astype(np.int32)
+    k1 = one.kv_offsets.astype(np.int32)
+    b1 = (1, 0x1000, 0x2000, 32768, 32768, 32768, 32768, None, 0, 0)
+    assert dsa.dsa_workspace_size(dsa.workload_shape(one), dsa.Ragged(*b1)) == \
+        dsa.dsa_workspace_size(dsa.workload_shape(one), dsa.Ragged(*b1, q1.ctypes.data, k1.ctypes.data))
