@@ -290,7 +290,7 @@ dsa_status launch_index_scores(const DeviceState& dev, const dsa_params* P, cons
   const int mode = cand ? kIdxCand : var.bmax ? kIdxBlockMax : kIdxScores;
   CUtensorMap mq, mk;
   if (cand && bq > 16) {
-    // query-major candidate pass: 128 query rows per CTA, 64-key tiles, 2 segments per row
+    // query-major candidate pass: 128 query rows per CTA, 64-key tiles, 4 segments per row
     DSA_TRY(make_idx_map(&mq, q_idx, R->total_q, P->n_idx_heads, fp8, kCandBQ));
     DSA_TRY(make_idx_map(&mk, k_idx, R->total_kv, P->n_idx_heads, fp8, kCandKT));
     IdxArgs a;
@@ -564,7 +564,6 @@ dsa_status fused_pass(const DeviceState& dev, const dsa_params* P, const dsa_rag
   a.cnt = cnt;
   a.cand = reinterpret_cast<const float2*>(f.sc);
   a.cap = g.cap;
-  a.cand_segs = bq > 16 ? kCandSegs : 4;  // query-major pass : row-major pass
   a.cand_cnt = f.ccnt;
   a.fb_list = f.list;
   a.q_idx = q_idx;

@@ -12,8 +12,9 @@
 //  - Warp 0 issues TMA loads (128-byte swizzle, one box per indexer head; the query tile
 //    once, then a 3-stage ring of key tiles); warp 1 issues tcgen05.mma (A = query tile,
 //    B = key tile, one UMMA per head and K step) into one of two TMEM buffers of 4 x 64
-//    columns; warps 2-9 drain TMEM: the two warps of a lane quadrant take 32 key columns
-//    each (segment sub = 0 or 1 of the row's candidate list).
+//    columns; warps 2-17 drain TMEM: the four warps of a lane quadrant take 16 key columns
+//    each (segment sub = 0..3 of the row's candidate list), so that four warps per
+//    scheduler hide each other's TMEM-load and dependency latencies.
 //  - A thread appends its hits to a small staging area of its own in shared memory and
 //    writes them to its segment in whole 32-byte sectors (4 pairs), so the candidate stream
 //    leaves the SM in full sectors instead of one scattered 8-byte store per hit.
@@ -32,11 +33,12 @@ namespace dsa {
 constexpr int kCandBQ = 128;       // query rows per CTA (MMA M, TMEM lanes)
 constexpr int kCandKT = 64;        // keys per tile (MMA N)
 constexpr int kCandStages = 3;     // key-tile ring depth
-constexpr int kCandEpiWarps = 8;   // two per TMEM lane quadrant
+constexpr int kCandEpiWarps = 16;  // four per TMEM lane quadrant
 constexpr int kCandThreads = 64 + 32 * kCandEpiWarps;
-constexpr int kCandSegs = 2;       // candidate segments per row (one per key half of a tile)
-constexpr int kCandSlots = 22;     // staging slots (8-byte pairs) per (row, segment)
-constexpr int kCandSlotStride = kCandSlots * 8;  // 176 B: 16-byte aligned, banks spread by row
+constexpr int kCandSegs = 4;       // candidate segments per row (one per 16 key columns)
+constexpr int kCandCols = kCandKT / kCandSegs;   // key columns per epilogue warp and tile
+constexpr int kCandSlots = 14;     // staging slots (8-byte pairs) per (row, segment)
+constexpr int kCandSlotStride = kCandSlots * 8;  // 112 B: 16-byte aligned, banks spread by row
 
 template <bool FP8>
 __host__ __device__ constexpr size_t cand_q_bytes() { return (size_t)4 * kCandBQ * (FP8 ? 64 : 128); }
@@ -223,9 +225,9 @@ __global__ void __launch_bounds__(kCandThreads, 1)
       mbar_wait_bounded(smem_u32(&tfull[j & 1]), (j >> 1) & 1, nullptr, nullptr);
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2-9)
+    // ------------------------------------------------------------ epilogue (warps 2-17)
     const int quad = warp & 3;          // TMEM lanes 32 quad .. 32 quad + 31
-    const int sub = (warp - 2) >> 2;    // key columns 32 sub .. 32 sub + 31 of each tile
+    const int sub = (warp - 2) >> 2;    // key columns 16 sub .. 16 sub + 15 of each tile
     const int rr = quad * 32 + lane;    // this thread's row within the tile
     const int64_t row = r0 + rr;
     const bool in_launch = row <= r_last;
@@ -244,16 +246,17 @@ __global__ void __launch_bounds__(kCandThreads, 1)
     const int seg = a.cap / kCandSegs;
     float2* dst = a.cand + (in_launch ? (row - a.q_begin) : 0) * (int64_t)a.cap + sub * seg;
     uint8_t* stg = stage_base + ((size_t)sub * kCandBQ + rr) * kCandSlotStride;
+    const uint32_t stg_u32 = smem_u32(stg);
     uint32_t cnt = 0;      // hits so far (may exceed seg: the selection then falls back)
     uint32_t written = 0;  // pairs moved to global memory (multiple of 4 until the tail)
     uint32_t pend = 0;     // pairs waiting in the staging slots 0 .. pend-1
 
     // write every complete group of 4 pending pairs (whole 32-byte sectors) and move the
-    // rest (< 4) to the front of the staging area
+    // rest (< 4) to the front of the staging area (at most 3 + 8 pairs are pending)
     auto flush = [&]() {
       const uint32_t groups = pend >> 2;
 #pragma unroll
-      for (uint32_t g = 0; g < 5; ++g) {
+      for (uint32_t g = 0; g < 3; ++g) {
         if (g < groups) {
           const float4 x0 = *reinterpret_cast<const float4*>(stg + g * 32);
           const float4 x1 = *reinterpret_cast<const float4*>(stg + g * 32 + 16);
@@ -296,15 +299,17 @@ __global__ void __launch_bounds__(kCandThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t tbase = tmem + lane_base + (uint32_t)(buf * 4 * kCandKT + sub * 32);
-        float acc[32];
+        const uint32_t tbase = tmem + lane_base + (uint32_t)(buf * 4 * kCandKT + sub * kCandCols);
+        float acc[kCandCols];
         {
-          uint32_t v[2][32];
+          // two heads per TMEM wait (four in flight would exceed the 96 registers a thread
+          // has at 18 warps per SM)
+          uint32_t v[2][kCandCols];
 #pragma unroll
           for (int hp = 0; hp < 4; hp += 2) {
             if (hp >= H) break;
-            tmem_ld32_async(tbase + (uint32_t)(hp * kCandKT), v[0]);
-            if (hp + 1 < H) tmem_ld32_async(tbase + (uint32_t)((hp + 1) * kCandKT), v[1]);
+            tmem_ld16_async(tbase + (uint32_t)(hp * kCandKT), v[0]);
+            if (hp + 1 < H) tmem_ld16_async(tbase + (uint32_t)((hp + 1) * kCandKT), v[1]);
             tmem_wait_ld();
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
@@ -314,7 +319,7 @@ __global__ void __launch_bounds__(kCandThreads, 1)
               if (!row_w) {
                 const float2 w2 = make_float2(wsh[h], wsh[h]);
 #pragma unroll
-                for (int c = 0; c < 32; c += 2) {
+                for (int c = 0; c < kCandCols; c += 2) {
                   const float2 x = make_float2(fmaxf(__uint_as_float(v[q][c]), 0.f),
                                                fmaxf(__uint_as_float(v[q][c + 1]), 0.f));
                   const float2 prev = h == 0 ? make_float2(0.f, 0.f) : make_float2(acc[c], acc[c + 1]);
@@ -324,7 +329,7 @@ __global__ void __launch_bounds__(kCandThreads, 1)
                 }
               } else {
 #pragma unroll
-                for (int c = 0; c < 32; ++c)
+                for (int c = 0; c < kCandCols; ++c)
                   acc[c] = fmaf(wsh[h], fmaxf(__uint_as_float(v[q][c]) * a.scale, 0.f),
                                 h == 0 ? 0.f : acc[c]);
               }
@@ -336,22 +341,44 @@ __global__ void __launch_bounds__(kCandThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&tempty[buf]));
 
-        const int j0 = kt * kCandKT + sub * 32;  // position of key column 0
-        const bool interior = __all_sync(0xFFFFFFFFu, warp_in_seq && j0 + 31 <= p_min);
-        const int lim = prow - j0;               // keys k <= lim are visible to this row
+        const int j0 = kt * kCandKT + sub * kCandCols;  // position of key column 0
+        const bool interior = __all_sync(0xFFFFFFFFu, warp_in_seq && j0 + kCandCols - 1 <= p_min);
+        const int lim = prow - j0;                      // keys k <= lim are visible to this row
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          float2* p = reinterpret_cast<float2*>(stg) + pend;
+        for (int grp = 0; grp < kCandCols / 8; ++grp) {
+          // straight-line predicated appends (no branch per key): compare, then the store
+          // and the slot advance under the same predicate
+          uint32_t sp = stg_u32 + pend * 8;
+          if (interior) {
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const int k = half * 16 + c;
-            const bool hit = acc[k] >= thr && (interior || k <= lim);
-            if (hit) {
-              *p = make_float2(__int_as_float(j0 + k), acc[k]);
-              ++p;
+            for (int c = 0; c < 8; ++c) {
+              const int k = grp * 8 + c;
+              asm volatile(
+                  "{\n\t.reg .pred p;\n\t"
+                  "setp.ge.f32 p, %1, %2;\n\t"
+                  "@p st.shared.v2.b32 [%0], {%3, %4};\n\t"
+                  "@p add.u32 %0, %0, 8;\n\t}"
+                  : "+r"(sp)
+                  : "f"(acc[k]), "f"(thr), "r"(j0 + k), "r"(__float_as_uint(acc[k]))
+                  : "memory");
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const int k = grp * 8 + c;
+              asm volatile(
+                  "{\n\t.reg .pred p;\n\t"
+                  "setp.ge.f32 p, %1, %2;\n\t"
+                  "setp.le.and.s32 p, %5, %6, p;\n\t"
+                  "@p st.shared.v2.b32 [%0], {%3, %4};\n\t"
+                  "@p add.u32 %0, %0, 8;\n\t}"
+                  : "+r"(sp)
+                  : "f"(acc[k]), "f"(thr), "r"(j0 + k), "r"(__float_as_uint(acc[k])), "r"(k),
+                    "r"(lim)
+                  : "memory");
             }
           }
-          const uint32_t now = (uint32_t)(p - reinterpret_cast<float2*>(stg));
+          const uint32_t now = (sp - stg_u32) >> 3;
           cnt += now - pend;
           pend = now;
           if (pend >= 4) flush();
@@ -364,12 +391,7 @@ __global__ void __launch_bounds__(kCandThreads, 1)
       for (uint32_t t = 0; t < 3; ++t)
         if (t < pend && written + t < (uint32_t)seg)
           dst[written + t] = *reinterpret_cast<const float2*>(stg + t * 8);
-      int32_t* cc = a.cand_cnt + (row - a.q_begin) * 4;
-      cc[sub] = (int32_t)cnt;
-      if (sub == 0) {
-        cc[2] = 0;
-        cc[3] = 0;
-      }
+      a.cand_cnt[(row - a.q_begin) * 4 + sub] = (int32_t)cnt;
     }
   }
 

@@ -85,10 +85,9 @@ struct TopkArgs {
   int64_t ld_idx;
   int32_t* cnt;
   // fused selection: candidate lists of the candidate indexer pass
-  const float2* cand;       // [q_count, cap]: cand_segs segments of cap / cand_segs
-  int cap;                  //   (position bits, score) pairs
-  int cand_segs;            // 4 (row-major candidate pass) or 2 (query-major pass)
-  const int32_t* cand_cnt;  // [q_count, 4] pairs found per segment (0 for unused ones)
+  const float2* cand;       // [q_count, cap]: 4 segments of cap/4 (position bits, score)
+  int cap;
+  const int32_t* cand_cnt;  // [q_count, 4] per segment
   int32_t* fb_list;         // [1 + q_count]: count, then rows (within the launch) to redo
   int blk_shift;            // rows of block scores: n = (p >> blk_shift) + 1 entries
   int prefetch_ahead;       // fused selection: warm L2 with the candidates of the row this
@@ -860,7 +859,7 @@ __global__ void __launch_bounds__(kTopkThreads, 3) topk_fused_kernel(TopkArgs a)
     if (a.cnt && tid == 0) a.cnt[i] = (int32_t)n;
     return;
   }
-  const int seg = a.cap / a.cand_segs;
+  const int seg = a.cap >> 2;
   if (tid == 0 && a.prefetch_ahead > 0 && i >= a.prefetch_ahead) {
     // the CTA that will take row i2 starts about when this one ends: pull its candidate
     // segments towards L2 now (a hint only; nothing waits for it)
