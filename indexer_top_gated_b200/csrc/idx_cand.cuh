@@ -252,29 +252,32 @@ __global__ void __launch_bounds__(kCandThreads, 1)
     uint32_t pend = 0;     // pairs waiting in the staging slots 0 .. pend-1
 
     // write every complete group of 4 pending pairs (whole 32-byte sectors) and move the
-    // rest (< 4) to the front of the staging area (at most 3 + 8 pairs are pending)
+    // rest (< 4) to the front of the staging area.  At most 3 + 8 pairs are pending, so at
+    // most two groups; the work is predicated per lane under one warp-uniform branch (some
+    // lane of the warp almost always has a group to write).
     auto flush = [&]() {
       const uint32_t groups = pend >> 2;
-#pragma unroll
-      for (uint32_t g = 0; g < 3; ++g) {
-        if (g < groups) {
-          const float4 x0 = *reinterpret_cast<const float4*>(stg + g * 32);
-          const float4 x1 = *reinterpret_cast<const float4*>(stg + g * 32 + 16);
-          if (written + 4 * g + 4 <= (uint32_t)seg) {
-            float4* d4 = reinterpret_cast<float4*>(dst + written + 4 * g);
-            d4[0] = x0;
-            d4[1] = x1;
-          }
-        }
+      if (!__any_sync(0xFFFFFFFFu, groups > 0)) return;
+      const float4 x0 = *reinterpret_cast<const float4*>(stg);
+      const float4 x1 = *reinterpret_cast<const float4*>(stg + 16);
+      const float4 y0 = *reinterpret_cast<const float4*>(stg + 32);
+      const float4 y1 = *reinterpret_cast<const float4*>(stg + 48);
+      const float2 r0 = *reinterpret_cast<const float2*>(stg + (groups * 4 + 0) * 8);
+      const float2 r1 = *reinterpret_cast<const float2*>(stg + (groups * 4 + 1) * 8);
+      const float2 r2 = *reinterpret_cast<const float2*>(stg + (groups * 4 + 2) * 8);
+      float4* d4 = reinterpret_cast<float4*>(dst + written);
+      if (groups > 0 && written + 4 <= (uint32_t)seg) {
+        d4[0] = x0;
+        d4[1] = x1;
+      }
+      if (groups > 1 && written + 8 <= (uint32_t)seg) {
+        d4[2] = y0;
+        d4[3] = y1;
       }
       const uint32_t rest = pend & 3u;
-      if (groups > 0) {
-#pragma unroll
-        for (uint32_t t = 0; t < 3; ++t)
-          if (t < rest)
-            *reinterpret_cast<float2*>(stg + t * 8) =
-                *reinterpret_cast<const float2*>(stg + (groups * 4 + t) * 8);
-      }
+      if (groups > 0 && rest > 0) *reinterpret_cast<float2*>(stg) = r0;
+      if (groups > 0 && rest > 1) *reinterpret_cast<float2*>(stg + 8) = r1;
+      if (groups > 0 && rest > 2) *reinterpret_cast<float2*>(stg + 16) = r2;
       written += groups * 4;
       pend = rest;
     };
@@ -381,7 +384,7 @@ __global__ void __launch_bounds__(kCandThreads, 1)
           const uint32_t now = (sp - stg_u32) >> 3;
           cnt += now - pend;
           pend = now;
-          if (pend >= 4) flush();
+          flush();
         }
       }
     }

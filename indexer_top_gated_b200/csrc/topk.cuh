@@ -592,14 +592,18 @@ DSA_DEV void topk_scores_row(const TopkArgs& a, int nn, const float* row, int32_
   }
 }
 
-// Fused selection over the row's candidates: cnt[s] of them at the start of segment s
+// Fused selection over the row's candidates: cnt[s] <= seg of them at the start of segment s
 // (seg slots each) of cl, C = sum >= K in all, nn <= kTopkFusedMaxN.  Keys are mapped onto
 // the full 32-bit range by the order-preserving (key - kmin) << clz(kmax - kmin), so that
 // the 12-bit digit spreads although all candidates lie close together.  Returns false
 // (nothing written) when the threshold bin holds more than kTopkBinMax candidates.
+// Each quarter of the block (128 threads) loads one segment, so no thread searches for the
+// segment of an element; the normalised keys are recomputed where they are needed rather
+// than stored back.
 DSA_DEV bool topk_candidates_row(const TopkArgs& a, int nn, const float2* cl, int seg,
                                  const uint32_t (&cnt)[4], uint32_t C, int32_t* out,
                                  uint32_t* dyn, TopkShared& sh) {
+  static_assert(kTopkThreads == 512, "four segments of 128 threads");
   uint32_t* h = dyn;                     // [4096]
   uint32_t* sk = dyn + 4096;             // [cap] keys
   uint32_t* sp = sk + a.cap;             // [cap] positions
@@ -609,66 +613,50 @@ DSA_DEV bool topk_candidates_row(const TopkArgs& a, int nn, const float2* cl, in
   const int tid = threadIdx.x, lane = lane_id(), warp = tid >> 5;
   const int W = (nn + 31) >> 5;
   int bank = 0;
-  const uint32_t e1 = cnt[0], e2 = e1 + cnt[1], e3 = e2 + cnt[2];
-  for (int t = tid; t < 4096; t += kTopkThreads) h[t] = 0;
+  // this thread's segment and where its candidates go in the packed key / position arrays
+  const int sg = tid >> 7;
+  const uint32_t ns = cnt[sg];
+  const uint32_t pre = (sg > 0 ? cnt[0] : 0u) + (sg > 1 ? cnt[1] : 0u) + (sg > 2 ? cnt[2] : 0u);
+  const float2* src = cl + (int64_t)sg * seg;
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  for (uint32_t e0 = tid & 127; e0 < ns; e0 += 128 * kTopkCandBatch) {
+    float2 e[kTopkCandBatch];
+#pragma unroll
+    for (int u = 0; u < kTopkCandBatch; ++u) {
+      const uint32_t x = e0 + 128u * u;
+      e[u] = x < ns ? __ldg(src + x) : make_float2(0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kTopkCandBatch; ++u) {
+      const uint32_t x = e0 + 128u * u;
+      if (x < ns) {
+        const uint32_t key = topk_key(e[u].y);
+        lo = key < lo ? key : lo;
+        hi = key > hi ? key : hi;
+        sk[pre + x] = key;
+        sp[pre + x] = (uint32_t)__float_as_int(e[u].x);
+      }
+    }
+  }
+  for (int t = tid; t < 1024; t += kTopkThreads)
+    reinterpret_cast<uint4*>(h)[t] = make_uint4(0u, 0u, 0u, 0u);
   for (int t = tid; t < W; t += kTopkThreads) bm[t] = 0;
   if (tid == 0) {
     sh.kmin = 0xFFFFFFFFu;
     sh.kmax = 0u;
     sh.ncand = 0;
   }
-  // load the candidates (several loads in flight per thread)
-  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-  for (uint32_t c0 = 0; c0 < C; c0 += kTopkCandBatch * kTopkThreads) {
-    float2 e[kTopkCandBatch];
-#pragma unroll
-    for (int u = 0; u < kTopkCandBatch; ++u) {
-      const uint32_t c = c0 + u * kTopkThreads + tid;
-      const int s = (c >= e1) + (c >= e2) + (c >= e3);
-      const uint32_t sb = s == 0 ? 0u : s == 1 ? e1 : s == 2 ? e2 : e3;
-      e[u] = c < C ? __ldg(cl + (int64_t)s * seg + (c - sb)) : make_float2(0.f, 0.f);
-    }
-#pragma unroll
-    for (int u = 0; u < kTopkCandBatch; ++u) {
-      const uint32_t c = c0 + u * kTopkThreads + tid;
-      if (c < C) {
-        const uint32_t key = topk_key(e[u].y);
-        lo = key < lo ? key : lo;
-        hi = key > hi ? key : hi;
-        sk[c] = key;
-        sp[c] = (uint32_t)__float_as_int(e[u].x);
-      }
-    }
-  }
   lo = __reduce_min_sync(0xFFFFFFFFu, lo);
   hi = __reduce_max_sync(0xFFFFFFFFu, hi);
-  __syncthreads();  // kmin / kmax initialised, histogram and bitmap zeroed
+  __syncthreads();  // kmin / kmax initialised, histogram and bitmap zeroed, keys stored
   if (lane == 0) {
     atomicMin(&sh.kmin, lo);
     atomicMax(&sh.kmax, hi);
   }
   __syncthreads();
-  {
-    const uint32_t kmin = sh.kmin, span = sh.kmax - sh.kmin;
-    const int z = span ? __clz(span) : 0;
-    for (uint32_t c0 = 0; c0 < C; c0 += kTopkCandBatch * kTopkThreads) {
-      uint32_t kk[kTopkCandBatch];
-#pragma unroll
-      for (int u = 0; u < kTopkCandBatch; ++u) {
-        const uint32_t c = c0 + u * kTopkThreads + tid;
-        kk[u] = c < C ? sk[c] : 0u;
-      }
-#pragma unroll
-      for (int u = 0; u < kTopkCandBatch; ++u) {
-        const uint32_t c = c0 + u * kTopkThreads + tid;
-        if (c < C) {
-          const uint32_t nk = (kk[u] - kmin) << z;
-          sk[c] = nk;
-          atomicAdd(&h[nk >> 20], 1u);
-        }
-      }
-    }
-  }
+  const uint32_t kmin = sh.kmin, span = sh.kmax - sh.kmin;
+  const int z = span ? __clz(span) : 0;
+  for (uint32_t c = tid; c < C; c += kTopkThreads) atomicAdd(&h[((sk[c] - kmin) << z) >> 20], 1u);
   __syncthreads();
   if (warp == 0) warp_select<4096>(h, (uint32_t)a.K, sh.sel);
   __syncthreads();
@@ -678,27 +666,18 @@ DSA_DEV bool topk_candidates_row(const TopkArgs& a, int nn, const float2* cl, in
   if (!whole && n_bin > (uint32_t)kTopkBinMax) return false;  // uniform
   // keys in higher bins (or the whole threshold bin) are selected; the threshold bin's
   // keys are set aside for ranking
-  for (uint32_t c0 = 0; c0 < C; c0 += kTopkCandBatch * kTopkThreads) {
-    uint32_t kk[kTopkCandBatch], pp[kTopkCandBatch];
-#pragma unroll
-    for (int u = 0; u < kTopkCandBatch; ++u) {
-      const uint32_t c = c0 + u * kTopkThreads + tid;
-      kk[u] = c < C ? sk[c] : 0u;
-      pp[u] = c < C ? sp[c] : 0xFFFFFFFFu;
-    }
-#pragma unroll
-    for (int u = 0; u < kTopkCandBatch; ++u) {
-      // (also skips positions outside the row, which only a corrupted workspace can hold:
-      // they never index the bitmap)
-      if (pp[u] >= (uint32_t)nn) continue;
-      const uint32_t bin = kk[u] >> 20, pos = pp[u];
-      if (bin > b || (whole && bin == b)) {
-        atomicOr(&bm[pos >> 5], 1u << (pos & 31u));
-      } else if (bin == b) {
-        const uint32_t slot = atomicAdd(&sh.ncand, 1u);
-        bk[slot] = kk[u];
-        bp[slot] = pos;
-      }
+  for (uint32_t c = tid; c < C; c += kTopkThreads) {
+    const uint32_t nk = (sk[c] - kmin) << z, pos = sp[c];
+    // (also skips positions outside the row, which only a corrupted workspace can hold:
+    // they never index the bitmap)
+    if (pos >= (uint32_t)nn) continue;
+    const uint32_t bin = nk >> 20;
+    if (bin > b || (whole && bin == b)) {
+      atomicOr(&bm[pos >> 5], 1u << (pos & 31u));
+    } else if (bin == b) {
+      const uint32_t slot = atomicAdd(&sh.ncand, 1u);
+      bk[slot] = nk;
+      bp[slot] = pos;
     }
   }
   __syncthreads();
