@@ -47,11 +47,13 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
 
 def build_probe(force: bool = False, verbose: bool = False) -> str:
+    probe_hdr = os.path.join(INCLUDE, "dsa_probe.h")
     if (not force and os.path.exists(PROBE_LIB)
-            and os.path.getmtime(PROBE_LIB) >= os.path.getmtime(PROBE_SRC)):
+            and os.path.getmtime(PROBE_LIB) >= max(os.path.getmtime(PROBE_SRC),
+                                                   os.path.getmtime(probe_hdr))):
         return PROBE_LIB
     nvcc = os.environ.get("NVCC", "nvcc")
-    cmd = [nvcc, *NVCC_FLAGS, "-o", PROBE_LIB + ".tmp", PROBE_SRC]
+    cmd = [nvcc, *NVCC_FLAGS, "-I" + INCLUDE, "-o", PROBE_LIB + ".tmp", PROBE_SRC]
     if verbose:
         print(" ".join(cmd))
     subprocess.check_call(cmd)

@@ -16,6 +16,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "dsa_probe.h"
+
 namespace {
 
 __device__ __forceinline__ uint64_t mix64(uint64_t z) {
@@ -107,13 +109,7 @@ constexpr size_t kSmemRing = 8 * 2 * 16 * 32 * 16;  // 128 KiB per CTA
 
 extern "C" {
 
-// Gather rate of random 256-byte rows of `buf` (n_rows rows, a power of two, 16-byte
-// aligned).  idx: device int32 scratch of n_idx entries (a power of two) that receives the
-// row indices; sink: device scratch of >= blocks * 256 16-byte words (written only in a case
-// that does not occur).  variant 0: registers, 1: shared memory; `blocks` CTAs of 256 threads,
-// each warp gathering chunks_per_warp chunks of 32 rows; `reps` timed launches after one
-// untimed.  Returns bytes gathered per second (0 on an invalid argument or a CUDA error).
-// Synchronous, on the legacy default stream.
+// Declared and documented in include/dsa_probe.h.
 double dsa_probe_gather(const void* buf, uint32_t n_rows, int32_t* idx, uint32_t n_idx,
                         int variant, int blocks, int chunks_per_warp, int reps, void* sink) {
   if (!buf || !idx || !sink || n_rows == 0 || (n_rows & (n_rows - 1)) || n_idx < 32 ||

@@ -44,3 +44,46 @@ def test_reference_arm_is_silent_on_other_ranks():
     r = _run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
+
+
+def test_stage_report_rooflines():
+    """bench.stage_report: each stage against the resource that bounds it -- the indexer's
+    flops against the sustained bf16 peak, the Top-K bytes of the path that ran (fused rows
+    counted by the library, materialised otherwise, both in a mixed batch) against HBM, the
+    attention's algorithmic bytes against the measured L2 gather ceiling -- and an 'hbm'
+    fraction above 1 is refused."""
+    import pytest
+
+    sys.path.insert(0, ROOT)
+    import bench
+    import dsa_synth as S
+
+    peaks = {"hbm_gbs": 6500.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    gather = {"l2": {"gbs": 20000.0}}
+    w = S.workload("prefill_t32768_k2048")
+    a = bench.algorithmic(w)
+    st = bench.stage_report(w, [1.0, 1.0, 8.0], [3, 3, 1], peaks, gather, fused_rows=w.total_q)
+    assert st[0]["achieved"] == pytest.approx(a["idx_flops"] / 1e-3 / 1e12)
+    assert st[0]["frac"] == pytest.approx(st[0]["achieved"] / 1400.0)
+    # fused: the bytes the fused selection moves are the primary figure, the scope table's
+    # definition is the equivalent rate beside it
+    assert st[1]["achieved"] == pytest.approx(a["topk_bytes_fused_moved"] / 1e-3 / 1e9)
+    assert st[1]["scope_equivalent_gbs"] == pytest.approx(a["topk_bytes"] / 1e-3 / 1e9)
+    assert a["topk_bytes_fused_moved"] < a["topk_bytes"]
+    assert st[2]["bound"] == "l2" and st[2]["peak"] == 20000.0
+    assert st[2]["frac"] == pytest.approx(a["attn_bytes"] / 8e-3 / 1e9 / 20000.0)
+    # materialised: the scope table's bytes are what the path moves
+    st = bench.stage_report(w, [1.0, 1.0, 8.0], [8, 8, 1], peaks, gather, fused_rows=0)
+    assert st[1]["achieved"] == pytest.approx(a["topk_bytes"] / 1e-3 / 1e9)
+    assert st[1]["scope_equivalent_gbs"] is None
+    # an 'hbm' rate above the copy peak is not an HBM rate
+    with pytest.raises(AssertionError):
+        bench.stage_report(w, [1.0, 0.1, 8.0], [8, 8, 1], peaks, gather, fused_rows=0)
+    # mixed batch: the long query groups fused, the decode rows materialised
+    m = S.workload("mixed_serving", scale_down=64)
+    long_rows = sum(q for q in m.q_lens if q >= 128)
+    st = bench.stage_report(m, [1.0, 1.0, 8.0], [4, 4, 1], peaks, gather, fused_rows=long_rows)
+    lw = bench._sub_workload(m, [b for b, q in enumerate(m.q_lens) if q >= 128])
+    sw = bench._sub_workload(m, [b for b, q in enumerate(m.q_lens) if q < 128])
+    moved = bench.algorithmic(lw)["topk_bytes_fused_moved"] + bench.algorithmic(sw)["topk_bytes"]
+    assert st[1]["achieved"] == pytest.approx(moved / 1e-3 / 1e9)

@@ -233,3 +233,22 @@ def test_mixed_batch_workspace_plan_uses_host_offsets():
     b1 = (1, 0x1000, 0x2000, 32768, 32768, 32768, 32768, None, 0, 0)
     assert dsa.dsa_workspace_size(dsa.workload_shape(one), dsa.Ragged(*b1)) == \
         dsa.dsa_workspace_size(dsa.workload_shape(one), dsa.Ragged(*b1, q1.ctypes.data, k1.ctypes.data))
+
+
+def test_probe_library_exports_its_declared_entry_point():
+    """The benchmark's gather-ceiling probe (libdsaprobe.so) builds for sm_100a and exports
+    the function include/dsa_probe.h declares; argument checks return 0 without a launch."""
+    import ctypes
+    import os
+    import re
+
+    from indexer_top_gated_b200 import _build, peaks
+    hdr = open(os.path.join(_build.INCLUDE, "dsa_probe.h")).read()
+    names = re.findall(r"^\w[\w\s\*]*?\b(dsa_\w+)\(", hdr, re.M)
+    assert names == ["dsa_probe_gather"]
+    L = peaks._load()
+    for n in names:
+        assert hasattr(L, n)
+    # n_rows not a power of two / null buffers: rejected on the host
+    assert L.dsa_probe_gather(0x1000, 3, 0x2000, 64, 0, 1, 1, 1, 0x3000) == 0.0
+    assert L.dsa_probe_gather(None, 4, 0x2000, 64, 0, 1, 1, 1, 0x3000) == 0.0
