@@ -682,16 +682,19 @@ DSA_DEV bool topk_candidates_row(const TopkArgs& a, int nn, const float2* cl, in
   }
   __syncthreads();
   const uint32_t n_set = sh.ncand;  // the bin's candidates set aside (n_bin unless skipped)
-  if (!whole && tid < (int)n_set) {
-    // rank among the bin: larger keys first, then lower positions
-    const uint32_t k0 = bk[tid], p0 = bp[tid];
-    uint32_t rank = 0;
-#pragma unroll 4
-    for (uint32_t x = 0; x < n_set; ++x) {
-      const uint32_t k1 = bk[x];
-      rank += (k1 > k0) || (k1 == k0 && bp[x] < p0);
+  if (!whole) {
+    // rank among the bin (larger keys first, then lower positions), spread over every warp:
+    // warp w ranks candidates w, w + 16, ...; its lanes compare 32 others at a time
+    for (uint32_t x = (uint32_t)warp; x < n_set; x += kTopkWarps) {
+      const uint32_t k0 = bk[x], p0 = bp[x];
+      uint32_t rank = 0;
+      for (uint32_t y0 = 0; y0 < n_set; y0 += 32) {
+        const uint32_t y = y0 + (uint32_t)lane;
+        const bool before = y < n_set && (bk[y] > k0 || (bk[y] == k0 && bp[y] < p0));
+        rank += (uint32_t)__popc(__ballot_sync(0xFFFFFFFFu, before));
+      }
+      if (lane == 0 && rank < need) atomicOr(&bm[p0 >> 5], 1u << (p0 & 31u));
     }
-    if (rank < need) atomicOr(&bm[p0 >> 5], 1u << (p0 & 31u));
   }
   __syncthreads();
   // ascending output: each thread writes the positions of its run of bitmap words
