@@ -578,10 +578,10 @@ dsa_status fused_pass(const DeviceState& dev, const dsa_params* P, const dsa_rag
   a.pages = cache_pages(R);
   const size_t smem = topk_smem_bytes(R->max_kv_len);
   a.bm_words = topk_fused_bm_words(std::max(R->max_kv_len, 1));
-  a.prefetch_ahead = 3 * dev.num_sms;  // three selection CTAs share an SM
+  a.prefetch_ahead = kFusedCtasPerSm * dev.num_sms;  // about one wave of selection CTAs
   {  // (4) exact selection over the candidates
     StageScope scope(1, stream);
-    topk_fused_kernel<<<(unsigned)q_count, kTopkThreads,
+    topk_fused_kernel<<<(unsigned)q_count, kFusedThreads,
                         topk_fused_smem_bytes(g.cap, R->max_kv_len), stream>>>(a);
     ++t_launches;
     DSA_TRY(launch_status("topk_kernel (fused selection)"));

@@ -66,8 +66,14 @@ constexpr int kTopkBinMax = 512;     // threshold-bin candidates ranked directly
 __host__ __device__ inline int topk_fused_bm_words(int64_t max_n) {
   return (int)(((max_n + 31) / 32 + 3) / 4 * 4);
 }
-__host__ inline size_t topk_fused_smem_bytes(int cap, int64_t max_n) {
-  return (size_t)(4096 + 2 * cap + topk_fused_bm_words(max_n) + 2 * kTopkBinMax) * 4;
+// The fused selection runs 256-thread CTAs (up to six per SM): it re-reads a row's candidates
+// from L2 in each of its passes instead of staging them, so a CTA's shared memory is the
+// histogram, the position bitmap and the threshold bin only.
+constexpr int kFusedThreads = 256;
+constexpr int kFusedWarps = kFusedThreads / 32;
+constexpr int kFusedCtasPerSm = 6;
+__host__ inline size_t topk_fused_smem_bytes(int /*cap*/, int64_t max_n) {
+  return (size_t)(4096 + topk_fused_bm_words(max_n) + 2 * kTopkBinMax) * 4;
 }
 
 enum TopkMode { kTopkScores = 0, kTopkFallback = 2 };
@@ -147,6 +153,21 @@ DSA_DEV uint32_t warp_incl_scan(uint32_t x) {
 // Block-wide exclusive scan of one value per thread with a single barrier.  `tot` holds
 // two banks of per-warp totals used alternately (`bank` flips on every call), so a bank
 // is rewritten only after every thread has passed the next call's barrier.
+template <int NW>
+DSA_DEV uint32_t block_scan_w(uint32_t v, uint32_t* tot, int& bank, uint32_t& total) {
+  const int lane = lane_id(), warp = threadIdx.x >> 5;
+  const uint32_t x = warp_incl_scan(v);
+  uint32_t* t = tot + bank * 32;
+  if (lane == 31) t[warp] = x;
+  __syncthreads();
+  const uint32_t wt = lane < NW ? t[lane] : 0u;
+  const uint32_t wi = warp_incl_scan(wt);
+  total = __shfl_sync(0xFFFFFFFFu, wi, 31);
+  const uint32_t wbase = __shfl_sync(0xFFFFFFFFu, wi - wt, warp);
+  bank ^= 1;
+  return wbase + x - v;
+}
+
 DSA_DEV uint32_t block_scan(uint32_t v, uint32_t* tot, int& bank, uint32_t& total) {
   const int lane = lane_id(), warp = threadIdx.x >> 5;
   const uint32_t x = warp_incl_scan(v);
@@ -597,50 +618,47 @@ DSA_DEV void topk_scores_row(const TopkArgs& a, int nn, const float* row, int32_
 // the full 32-bit range by the order-preserving (key - kmin) << clz(kmax - kmin), so that
 // the 12-bit digit spreads although all candidates lie close together.  Returns false
 // (nothing written) when the threshold bin holds more than kTopkBinMax candidates.
-// Each quarter of the block (128 threads) loads one segment, so no thread searches for the
-// segment of an element; the normalised keys are recomputed where they are needed rather
-// than stored back.
+// kFusedThreads threads: each quarter of the block reads one segment in every pass (the key
+// range, the histogram, the marking), straight from global memory -- the first pass brings
+// the row's candidates into L2, the later ones hit there.
 DSA_DEV bool topk_candidates_row(const TopkArgs& a, int nn, const float2* cl, int seg,
                                  const uint32_t (&cnt)[4], uint32_t C, int32_t* out,
                                  uint32_t* dyn, TopkShared& sh) {
-  static_assert(kTopkThreads == 512, "four segments of 128 threads");
+  constexpr int kQuarter = kFusedThreads / 4;
   uint32_t* h = dyn;                     // [4096]
-  uint32_t* sk = dyn + 4096;             // [cap] keys
-  uint32_t* sp = sk + a.cap;             // [cap] positions
-  uint32_t* bm = sp + a.cap;             // [bm_words] selected positions
+  uint32_t* bm = h + 4096;               // [bm_words] selected positions
   uint32_t* bk = bm + a.bm_words;        // [kTopkBinMax] threshold-bin keys
   uint32_t* bp = bk + kTopkBinMax;       // [kTopkBinMax] threshold-bin positions
   const int tid = threadIdx.x, lane = lane_id(), warp = tid >> 5;
   const int W = (nn + 31) >> 5;
   int bank = 0;
-  // this thread's segment and where its candidates go in the packed key / position arrays
-  const int sg = tid >> 7;
+  const int sg = tid / kQuarter;
   const uint32_t ns = cnt[sg];
-  const uint32_t pre = (sg > 0 ? cnt[0] : 0u) + (sg > 1 ? cnt[1] : 0u) + (sg > 2 ? cnt[2] : 0u);
   const float2* src = cl + (int64_t)sg * seg;
-  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-  for (uint32_t e0 = tid & 127; e0 < ns; e0 += 128 * kTopkCandBatch) {
-    float2 e[kTopkCandBatch];
+  const uint32_t x0 = (uint32_t)(tid % kQuarter);
+  constexpr uint32_t kStep = (uint32_t)kQuarter * kTopkCandBatch;
+  // one pass over this thread's candidates, kTopkCandBatch loads in flight
+  auto for_cands = [&](auto&& f) {
+    for (uint32_t e0 = x0; e0 < ns; e0 += kStep) {
+      float2 e[kTopkCandBatch];
 #pragma unroll
-    for (int u = 0; u < kTopkCandBatch; ++u) {
-      const uint32_t x = e0 + 128u * u;
-      e[u] = x < ns ? __ldg(src + x) : make_float2(0.f, 0.f);
-    }
-#pragma unroll
-    for (int u = 0; u < kTopkCandBatch; ++u) {
-      const uint32_t x = e0 + 128u * u;
-      if (x < ns) {
-        const uint32_t key = topk_key(e[u].y);
-        lo = key < lo ? key : lo;
-        hi = key > hi ? key : hi;
-        sk[pre + x] = key;
-        sp[pre + x] = (uint32_t)__float_as_int(e[u].x);
+      for (int u = 0; u < kTopkCandBatch; ++u) {
+        const uint32_t x = e0 + (uint32_t)kQuarter * u;
+        e[u] = x < ns ? __ldg(src + x) : make_float2(0.f, 0.f);
       }
+#pragma unroll
+      for (int u = 0; u < kTopkCandBatch; ++u)
+        if (e0 + (uint32_t)kQuarter * u < ns) f(topk_key(e[u].y), (uint32_t)__float_as_int(e[u].x));
     }
-  }
-  for (int t = tid; t < 1024; t += kTopkThreads)
+  };
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  for_cands([&](uint32_t key, uint32_t) {
+    lo = key < lo ? key : lo;
+    hi = key > hi ? key : hi;
+  });
+  for (int t = tid; t < 1024; t += kFusedThreads)
     reinterpret_cast<uint4*>(h)[t] = make_uint4(0u, 0u, 0u, 0u);
-  for (int t = tid; t < W; t += kTopkThreads) bm[t] = 0;
+  for (int t = tid; t < W; t += kFusedThreads) bm[t] = 0;
   if (tid == 0) {
     sh.kmin = 0xFFFFFFFFu;
     sh.kmax = 0u;
@@ -648,7 +666,7 @@ DSA_DEV bool topk_candidates_row(const TopkArgs& a, int nn, const float2* cl, in
   }
   lo = __reduce_min_sync(0xFFFFFFFFu, lo);
   hi = __reduce_max_sync(0xFFFFFFFFu, hi);
-  __syncthreads();  // kmin / kmax initialised, histogram and bitmap zeroed, keys stored
+  __syncthreads();  // kmin / kmax initialised, histogram and bitmap zeroed
   if (lane == 0) {
     atomicMin(&sh.kmin, lo);
     atomicMax(&sh.kmax, hi);
@@ -656,7 +674,7 @@ DSA_DEV bool topk_candidates_row(const TopkArgs& a, int nn, const float2* cl, in
   __syncthreads();
   const uint32_t kmin = sh.kmin, span = sh.kmax - sh.kmin;
   const int z = span ? __clz(span) : 0;
-  for (uint32_t c = tid; c < C; c += kTopkThreads) atomicAdd(&h[((sk[c] - kmin) << z) >> 20], 1u);
+  for_cands([&](uint32_t key, uint32_t) { atomicAdd(&h[((key - kmin) << z) >> 20], 1u); });
   __syncthreads();
   if (warp == 0) warp_select<4096>(h, (uint32_t)a.K, sh.sel);
   __syncthreads();
@@ -665,27 +683,27 @@ DSA_DEV bool topk_candidates_row(const TopkArgs& a, int nn, const float2* cl, in
   const uint32_t n_bin = h[b];
   if (!whole && n_bin > (uint32_t)kTopkBinMax) return false;  // uniform
   // keys in higher bins (or the whole threshold bin) are selected; the threshold bin's
-  // keys are set aside for ranking
-  for (uint32_t c = tid; c < C; c += kTopkThreads) {
-    const uint32_t nk = (sk[c] - kmin) << z, pos = sp[c];
-    // (also skips positions outside the row, which only a corrupted workspace can hold:
-    // they never index the bitmap)
-    if (pos >= (uint32_t)nn) continue;
-    const uint32_t bin = nk >> 20;
+  // keys are set aside for ranking.  (Positions outside the row, which only a corrupted
+  // workspace can hold, are skipped: they never index the bitmap.)
+  for_cands([&](uint32_t key, uint32_t pos) {
+    if (pos >= (uint32_t)nn) return;
+    const uint32_t nk = (key - kmin) << z, bin = nk >> 20;
     if (bin > b || (whole && bin == b)) {
       atomicOr(&bm[pos >> 5], 1u << (pos & 31u));
     } else if (bin == b) {
       const uint32_t slot = atomicAdd(&sh.ncand, 1u);
-      bk[slot] = nk;
-      bp[slot] = pos;
+      if (slot < (uint32_t)kTopkBinMax) {
+        bk[slot] = nk;
+        bp[slot] = pos;
+      }
     }
-  }
+  });
   __syncthreads();
-  const uint32_t n_set = sh.ncand;  // the bin's candidates set aside (n_bin unless skipped)
+  const uint32_t n_set = sh.ncand < (uint32_t)kTopkBinMax ? sh.ncand : (uint32_t)kTopkBinMax;
   if (!whole) {
     // rank among the bin (larger keys first, then lower positions), spread over every warp:
-    // warp w ranks candidates w, w + 16, ...; its lanes compare 32 others at a time
-    for (uint32_t x = (uint32_t)warp; x < n_set; x += kTopkWarps) {
+    // warp w ranks candidates w, w + kFusedWarps, ...; its lanes compare 32 others at a time
+    for (uint32_t x = (uint32_t)warp; x < n_set; x += kFusedWarps) {
       const uint32_t k0 = bk[x], p0 = bp[x];
       uint32_t rank = 0;
       for (uint32_t y0 = 0; y0 < n_set; y0 += 32) {
@@ -698,12 +716,12 @@ DSA_DEV bool topk_candidates_row(const TopkArgs& a, int nn, const float2* cl, in
   }
   __syncthreads();
   // ascending output: each thread writes the positions of its run of bitmap words
-  const int wpt = (W + kTopkThreads - 1) / kTopkThreads;
+  const int wpt = (W + kFusedThreads - 1) / kFusedThreads;
   const int w0 = tid * wpt, w1 = w0 + wpt < W ? w0 + wpt : W;
   uint32_t mine = 0;
   for (int w = w0; w < w1; ++w) mine += __popc(bm[w]);
   uint32_t total;
-  uint32_t at = block_scan(mine, sh.tot, bank, total);
+  uint32_t at = block_scan_w<kFusedWarps>(mine, sh.tot, bank, total);
   for (int w = w0; w < w1; ++w) {
     uint32_t bits = bm[w];
     while (bits) {
@@ -825,8 +843,8 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkArgs a) {
   if (tid == 0 && a.cnt) a.cnt[i] = K;
 }
 
-// Fused selection, one CTA per row (three CTAs share an SM).
-__global__ void __launch_bounds__(kTopkThreads, 3) topk_fused_kernel(TopkArgs a) {
+// Fused selection, one CTA of kFusedThreads per row (up to six CTAs share an SM).
+__global__ void __launch_bounds__(kFusedThreads, kFusedCtasPerSm) topk_fused_kernel(TopkArgs a) {
   extern __shared__ uint32_t dyn[];
   __shared__ TopkShared sh;
   const int tid = threadIdx.x;
@@ -837,7 +855,7 @@ __global__ void __launch_bounds__(kTopkThreads, 3) topk_fused_kernel(TopkArgs a)
   const int64_t n = topk_row_len(a, r, &b);
   int32_t* out = a.idx + i * a.ld_idx;
   if (n <= K) {
-    for (int j = tid; j < K; j += kTopkThreads) out[j] = j < n ? j : -1;
+    for (int j = tid; j < K; j += kFusedThreads) out[j] = j < n ? j : -1;
     if (a.cnt && tid == 0) a.cnt[i] = (int32_t)n;
     return;
   }
