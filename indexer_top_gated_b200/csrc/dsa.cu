@@ -290,7 +290,7 @@ dsa_status launch_index_scores(const DeviceState& dev, const dsa_params* P, cons
   const int mode = cand ? kIdxCand : var.bmax ? kIdxBlockMax : kIdxScores;
   CUtensorMap mq, mk;
   if (cand && bq > 16) {
-    // query-major candidate pass: 128 query rows per CTA, 64-key tiles, 4 segments per row
+    // query-major candidate pass: 128 query rows per CTA, 128-key tiles, 4 segments per row
     DSA_TRY(make_idx_map(&mq, q_idx, R->total_q, P->n_idx_heads, fp8, kCandBQ));
     DSA_TRY(make_idx_map(&mk, k_idx, R->total_kv, P->n_idx_heads, fp8, kCandKT));
     IdxArgs a;

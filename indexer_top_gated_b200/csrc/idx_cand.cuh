@@ -6,15 +6,20 @@
 // Same scores as idx_scores_kernel, laid out the other way round on the tensor core:
 //  - One CTA owns 128 consecutive packed query rows and every key tile they can see (so it
 //    owns their candidate lists).  The query tile is the MMA's M side: TMEM lane = query
-//    row, columns = keys (64 per tile and head), so each epilogue thread owns one query row.
-//    The ReLU-weighted head sum, the threshold compare and the candidate emission are then
-//    private to the thread: no transposition, no shuffles, no shared counters.
+//    row, columns = keys (128 per tile and head), so each epilogue thread owns one query
+//    row.  The ReLU-weighted head sum, the threshold compare and the candidate emission are
+//    then private to the thread: no transposition, no shuffles, no shared counters.
+//  - The accumulators are two TMEM slots of 256 columns, one per head pair (heads 0-1 and
+//    2-3 of a 128-key tile).  A 128 x 128 x 16 UMMA runs at the tensor core's full rate
+//    where a 128 x 64 one is bound by its shared-memory operand reads, and the slot of one
+//    head pair is drained while the MMAs of the other run, so the commit -> drain -> release
+//    round trip overlaps tensor-core work.
 //  - Warp 0 issues TMA loads (128-byte swizzle, one box per indexer head; the query tile
-//    once, then a 3-stage ring of key tiles); warp 1 issues tcgen05.mma (A = query tile,
-//    B = key tile, one UMMA per head and K step) into one of two TMEM buffers of 4 x 64
-//    columns; warps 2-17 drain TMEM: the four warps of a lane quadrant take 16 key columns
-//    each (segment sub = 0..3 of the row's candidate list), so that four warps per
-//    scheduler hide each other's TMEM-load and dependency latencies.
+//    once, then a 3-stage ring of half key tiles, one head pair each); warp 1 issues
+//    tcgen05.mma (A = query tile, B = key tile, one UMMA per head and K step); warps 2-17
+//    drain TMEM: the four warps of a lane quadrant take 32 key columns each (segment
+//    sub = 0..3 of the row's candidate list), so that four warps per scheduler hide each
+//    other's TMEM-load and dependency latencies.
 //  - A thread appends its hits to a small staging area of its own in shared memory and
 //    writes them to its segment in whole 32-byte sectors (4 pairs), so the candidate stream
 //    leaves the SM in full sectors instead of one scattered 8-byte store per hit.
@@ -31,19 +36,20 @@
 namespace dsa {
 
 constexpr int kCandBQ = 128;       // query rows per CTA (MMA M, TMEM lanes)
-constexpr int kCandKT = 64;        // keys per tile (MMA N)
-constexpr int kCandStages = 3;     // key-tile ring depth
+constexpr int kCandKT = 128;       // keys per tile (MMA N)
+constexpr int kCandStages = 3;     // ring depth in half key tiles (one head pair each)
 constexpr int kCandEpiWarps = 16;  // four per TMEM lane quadrant
 constexpr int kCandThreads = 64 + 32 * kCandEpiWarps;
-constexpr int kCandSegs = 4;       // candidate segments per row (one per 16 key columns)
+constexpr int kCandSegs = 4;       // candidate segments per row (one per 32 key columns)
 constexpr int kCandCols = kCandKT / kCandSegs;   // key columns per epilogue warp and tile
+constexpr int kCandSlotCols = 2 * kCandKT;       // TMEM columns of one head-pair slot
 constexpr int kCandSlots = 14;     // staging slots (8-byte pairs) per (row, segment)
 constexpr int kCandSlotStride = kCandSlots * 8;  // 112 B: 16-byte aligned, banks spread by row
 
 template <bool FP8>
 __host__ __device__ constexpr size_t cand_q_bytes() { return (size_t)4 * kCandBQ * (FP8 ? 64 : 128); }
 template <bool FP8>
-__host__ __device__ constexpr size_t cand_k_stage_bytes() { return (size_t)4 * kCandKT * (FP8 ? 64 : 128); }
+__host__ __device__ constexpr size_t cand_k_stage_bytes() { return (size_t)2 * kCandKT * (FP8 ? 64 : 128); }
 
 __host__ inline size_t idx_cand_smem_bytes(bool fp8) {
   const size_t q = fp8 ? cand_q_bytes<true>() : cand_q_bytes<false>();
@@ -64,16 +70,16 @@ __global__ void __launch_bounds__(kCandThreads, 1)
   constexpr uint32_t kQHead = kCandBQ * Geo::kRowBytes;  // one head of the query tile
   constexpr uint32_t kKHead = kCandKT * Geo::kRowBytes;  // one head of a key tile
   constexpr int ST = kCandStages;
-  constexpr int kCols = 2 * 4 * kCandKT;                 // TMEM columns (2 buffers x 4 heads)
+  constexpr int kCols = 2 * kCandSlotCols;               // TMEM columns (2 head-pair slots)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + 4 * kQHead;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sK + (size_t)ST * 4 * kKHead);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sK + (size_t)ST * 2 * kKHead);
   uint64_t* full = bars;            // [ST]
   uint64_t* empty = bars + ST;      // [ST]
-  uint64_t* tfull = bars + 2 * ST;  // [2]
+  uint64_t* tfull = bars + 2 * ST;  // [2] per head-pair slot
   uint64_t* tempty = tfull + 2;     // [2]
   uint64_t* qfull = tempty + 2;     // [1]
   uint8_t* stage_base = reinterpret_cast<uint8_t*>(bars) + 256;  // [segs][128 rows][slots]
@@ -83,6 +89,7 @@ __global__ void __launch_bounds__(kCandThreads, 1)
   __shared__ int s_consumed;
 
   const int H = a.n_heads;
+  const int n_pairs = (H + 1) >> 1;  // head pairs (the last may hold one head)
   const int warp = threadIdx.x >> 5;
   const int lane = lane_id();
   const int tile = a.n_tiles - 1 - (int)blockIdx.x;  // largest first
@@ -154,76 +161,83 @@ __global__ void __launch_bounds__(kCandThreads, 1)
       mbar_arrive_expect_tx(smem_u32(qfull), H * kQHead);
       for (int h = 0; h < H; ++h)
         tma_load_2d(smem_u32(sQ + h * kQHead), &tmap_q, smem_u32(qfull), h * 64, (int)r0);
-      int i = 0;
+      int u = 0;  // half key tiles issued
       bool ok = true;
       for (int b = b_first; b <= b_last && ok; ++b) {
         int64_t rs, re, pb;
         int kh;
         if (!seq_range(b, rs, re, kh, pb)) continue;
         const int64_t kbase = __ldg(a.kv_offsets + b);
-        for (int kt = 0; kt < kh; ++kt, ++i) {
-          // a 64-key tile never straddles a page (pages are multiples of 128 positions)
+        for (int kt = 0; kt < kh && ok; ++kt) {
+          // a 128-key tile never straddles a page (pages are multiples of 128 positions)
           const int64_t krow = a.pages.table ? cache_row(a.kv_offsets, a.pages, b, (int64_t)kt * kCandKT)
                                              : kbase + (int64_t)kt * kCandKT;
-          const int s = i % ST;
-          if (!mbar_wait_bounded(smem_u32(&empty[s]), ((i / ST) & 1) ^ 1, a.status, &s_abort)) {
-            ok = false;
-            break;
+          for (int pr = 0; pr < n_pairs; ++pr, ++u) {
+            const int s = u % ST;
+            const int nh = H - 2 * pr < 2 ? H - 2 * pr : 2;
+            if (!mbar_wait_bounded(smem_u32(&empty[s]), ((u / ST) & 1) ^ 1, a.status, &s_abort)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(smem_u32(&full[s]), nh * kKHead);
+            for (int hh = 0; hh < nh; ++hh)
+              tma_load_2d(smem_u32(sK + ((size_t)s * 2 + hh) * kKHead), &tmap_k, smem_u32(&full[s]),
+                          (2 * pr + hh) * 64, (int)krow);
           }
-          mbar_arrive_expect_tx(smem_u32(&full[s]), H * kKHead);
-          for (int h = 0; h < H; ++h)
-            tma_load_2d(smem_u32(sK + ((size_t)s * 4 + h) * kKHead), &tmap_k, smem_u32(&full[s]),
-                        h * 64, (int)krow);
         }
       }
       if (!ok) {
         mbar_wait_bounded(smem_u32(qfull), 0, nullptr, nullptr);
-        for (int j = s_consumed; j < i; ++j)
+        for (int j = s_consumed; j < u; ++j)
           mbar_wait_bounded(smem_u32(&full[j % ST]), (j / ST) & 1, nullptr, nullptr);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     const uint32_t idesc = umma_idesc(kCandBQ, kCandKT, FP8 ? 0u : 1u);
-    int i = 0, issued = 0;
+    int i = 0, u = 0;                // key tiles, half key tiles consumed
+    int last_pr = -1, last_i = 0;    // slot and tile of the last commit
     bool ok = mbar_wait_bounded(smem_u32(qfull), 0, a.status, &s_abort);
     for (int b = b_first; b <= b_last && ok; ++b) {
       int64_t rs, re, pb;
       int kh;
       if (!seq_range(b, rs, re, kh, pb)) continue;
-      for (int kt = 0; kt < kh; ++kt, ++i) {
-        const int s = i % ST, buf = i & 1;
-        if (!mbar_wait_bounded(smem_u32(&full[s]), (i / ST) & 1, a.status, &s_abort) ||
-            !mbar_wait_bounded(smem_u32(&tempty[buf]), ((i >> 1) & 1) ^ 1, a.status, &s_abort)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (lane == 0) {
-          for (int h = 0; h < H; ++h) {
-            const uint32_t a_base = smem_u32(sQ + h * kQHead);
-            const uint32_t b_base = smem_u32(sK + ((size_t)s * 4 + h) * kKHead);
-            const uint32_t d = tmem + (uint32_t)(buf * 4 * kCandKT + h * kCandKT);
-#pragma unroll
-            for (int kk = 0; kk < Geo::kKSteps; ++kk) {
-              const uint64_t ad = umma_smem_desc(a_base + kk * 32, Geo::kSbo, Geo::kLayout);
-              const uint64_t bd = umma_smem_desc(b_base + kk * 32, Geo::kSbo, Geo::kLayout);
-              if (FP8) umma_fp8(d, ad, bd, idesc, kk > 0);
-              else umma_bf16(d, ad, bd, idesc, kk > 0);
-            }
+      for (int kt = 0; kt < kh && ok; ++kt, ++i) {
+        for (int pr = 0; pr < n_pairs; ++pr, ++u) {
+          // slot pr is used once per key tile: its i-th use waits for the (i-1)-th release
+          const int s = u % ST;
+          const int nh = H - 2 * pr < 2 ? H - 2 * pr : 2;
+          if (!mbar_wait_bounded(smem_u32(&full[s]), (u / ST) & 1, a.status, &s_abort) ||
+              !mbar_wait_bounded(smem_u32(&tempty[pr]), (i & 1) ^ 1, a.status, &s_abort)) {
+            ok = false;
+            break;
           }
-          umma_commit(smem_u32(&empty[s]));
-          umma_commit(smem_u32(&tfull[buf]));
+          tc_fence_after();
+          if (lane == 0) {
+            for (int hh = 0; hh < nh; ++hh) {
+              const uint32_t a_base = smem_u32(sQ + (2 * pr + hh) * kQHead);
+              const uint32_t b_base = smem_u32(sK + ((size_t)s * 2 + hh) * kKHead);
+              const uint32_t d = tmem + (uint32_t)(pr * kCandSlotCols + hh * kCandKT);
+#pragma unroll
+              for (int kk = 0; kk < Geo::kKSteps; ++kk) {
+                const uint64_t ad = umma_smem_desc(a_base + kk * 32, Geo::kSbo, Geo::kLayout);
+                const uint64_t bd = umma_smem_desc(b_base + kk * 32, Geo::kSbo, Geo::kLayout);
+                if (FP8) umma_fp8(d, ad, bd, idesc, kk > 0);
+                else umma_bf16(d, ad, bd, idesc, kk > 0);
+              }
+            }
+            umma_commit(smem_u32(&empty[s]));
+            umma_commit(smem_u32(&tfull[pr]));
+          }
+          __syncwarp();
+          last_pr = pr;
+          last_i = i;
+          if (lane == 0) s_consumed = u + 1;
         }
-        __syncwarp();
-        issued = i + 1;
-        if (lane == 0) s_consumed = i + 1;
       }
     }
-    if (!ok && issued > 0 && lane == 0) {
-      const int j = issued - 1;  // the last commit completes after every earlier MMA
-      mbar_wait_bounded(smem_u32(&tfull[j & 1]), (j >> 1) & 1, nullptr, nullptr);
-    }
+    if (!ok && last_pr >= 0 && lane == 0)  // the last commit completes after every earlier MMA
+      mbar_wait_bounded(smem_u32(&tfull[last_pr]), last_i & 1, nullptr, nullptr);
   } else {
     // ------------------------------------------------------------ epilogue (warps 2-17)
     const int quad = warp & 3;          // TMEM lanes 32 quad .. 32 quad + 31
@@ -296,53 +310,59 @@ __global__ void __launch_bounds__(kCandThreads, 1)
       const int p_min = (int)(pbase + r0 + quad * 32);
       const bool warp_in_seq = r0 + quad * 32 >= rs && r0 + quad * 32 + 31 < re;
       for (int kt = 0; kt < kh; ++kt, ++i) {
-        const int buf = i & 1;
-        if (!mbar_wait_bounded(smem_u32(&tfull[buf]), (i >> 1) & 1, a.status, &s_abort)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t tbase = tmem + lane_base + (uint32_t)(buf * 4 * kCandKT + sub * kCandCols);
         float acc[kCandCols];
-        {
-          // two heads per TMEM wait (four in flight would exceed the 96 registers a thread
-          // has at 18 warps per SM)
-          uint32_t v[2][kCandCols];
+        bool waited = true;
 #pragma unroll
-          for (int hp = 0; hp < 4; hp += 2) {
-            if (hp >= H) break;
-            tmem_ld16_async(tbase + (uint32_t)(hp * kCandKT), v[0]);
-            if (hp + 1 < H) tmem_ld16_async(tbase + (uint32_t)((hp + 1) * kCandKT), v[1]);
-            tmem_wait_ld();
+        for (int pr = 0; pr < 2; ++pr) {
+          if (pr >= n_pairs) break;
+          if (!mbar_wait_bounded(smem_u32(&tfull[pr]), i & 1, a.status, &s_abort)) {
+            waited = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t tbase = tmem + lane_base + (uint32_t)(pr * kCandSlotCols + sub * kCandCols);
+          // one head and 16 key columns per TMEM wait: the 96 registers a thread has at 18
+          // warps per SM hold the 32 partial sums, one load and the emission state (two
+          // heads per wait spill)
+#pragma unroll
+          for (int c0 = 0; c0 < kCandCols; c0 += 16) {
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
-              const int h = hp + q;
+              const int h = 2 * pr + q;
               if (h >= H) break;
-              reg_fence(v[q]);
+              uint32_t v[16];
+              tmem_ld16_async(tbase + (uint32_t)(q * kCandKT + c0), v);
+              tmem_wait_ld();
+              reg_fence(v);
               if (!row_w) {
                 const float2 w2 = make_float2(wsh[h], wsh[h]);
 #pragma unroll
-                for (int c = 0; c < kCandCols; c += 2) {
-                  const float2 x = make_float2(fmaxf(__uint_as_float(v[q][c]), 0.f),
-                                               fmaxf(__uint_as_float(v[q][c + 1]), 0.f));
-                  const float2 prev = h == 0 ? make_float2(0.f, 0.f) : make_float2(acc[c], acc[c + 1]);
+                for (int c = 0; c < 16; c += 2) {
+                  const float2 x = make_float2(fmaxf(__uint_as_float(v[c]), 0.f),
+                                               fmaxf(__uint_as_float(v[c + 1]), 0.f));
+                  const float2 prev =
+                      h == 0 ? make_float2(0.f, 0.f) : make_float2(acc[c0 + c], acc[c0 + c + 1]);
                   const float2 r2 = __ffma2_rn(w2, x, prev);
-                  acc[c] = r2.x;
-                  acc[c + 1] = r2.y;
+                  acc[c0 + c] = r2.x;
+                  acc[c0 + c + 1] = r2.y;
                 }
               } else {
 #pragma unroll
-                for (int c = 0; c < kCandCols; ++c)
-                  acc[c] = fmaf(wsh[h], fmaxf(__uint_as_float(v[q][c]) * a.scale, 0.f),
-                                h == 0 ? 0.f : acc[c]);
+                for (int c = 0; c < 16; ++c)
+                  acc[c0 + c] = fmaf(wsh[h], fmaxf(__uint_as_float(v[c]) * a.scale, 0.f),
+                                     h == 0 ? 0.f : acc[c0 + c]);
               }
             }
           }
+          // the pair is in registers: hand its TMEM slot back to the MMA warp
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&tempty[pr]));
         }
-        // the four heads are in registers: hand the TMEM buffer back to the MMA warp
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&tempty[buf]));
+        if (!waited) {
+          ok = false;
+          break;
+        }
 
         const int j0 = kt * kCandKT + sub * kCandCols;  // position of key column 0
         const bool interior = __all_sync(0xFFFFFFFFu, warp_in_seq && j0 + kCandCols - 1 <= p_min);
