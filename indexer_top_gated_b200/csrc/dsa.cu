@@ -445,8 +445,8 @@ bool fused_geom(const dsa_params* P, const dsa_ragged* R, FusedGeom* g) {
   g->samp_rows = (logical >> kSampleShift) + R->batch + 1;
   g->key_row = (int64_t)P->n_idx_heads * 64 * (P->idx_dtype == DSA_FP8_E4M3 ? 1 : 2);
   g->fixed_bytes = round_up(g->samp_rows * g->key_row, 256) +
-                   round_up((int64_t)kFallbackCtas * g->ld_fb * 4, 256) + 256 * 4;
-  g->row_bytes = std::max<int64_t>(g->ld_s * 4, cap * 8) + 6 * 4;
+                   round_up((int64_t)kFallbackCtas * g->ld_fb * 4, 256) + 256 * 5;
+  g->row_bytes = std::max<int64_t>(g->ld_s * 4, cap * 8) + 7 * 4;
   return true;
 }
 
@@ -473,6 +473,7 @@ struct FusedWs {
   float* fb_scores;
   char* sc;        // samples [rows, ld_s] floats, later candidates [rows, cap] float2
   float* thr;
+  uint32_t* khi;   // [rows] largest sample key
   int32_t* ccnt;   // [rows, 4]
   int32_t* list;   // [1 + rows]
 };
@@ -487,6 +488,8 @@ FusedWs fused_carve(const FusedGeom& g, void* ws, int64_t rows) {
   f.sc = p;
   p += round_up(rows * std::max<int64_t>(g.ld_s * 4, (int64_t)g.cap * 8), 256);
   f.thr = reinterpret_cast<float*>(p);
+  p += round_up(rows * 4, 256);
+  f.khi = reinterpret_cast<uint32_t*>(p);
   p += round_up(rows * 4, 256);
   f.ccnt = reinterpret_cast<int32_t*>(p);
   p += round_up(rows * 16, 256);
@@ -535,6 +538,7 @@ dsa_status fused_pass(const DeviceState& dev, const dsa_params* P, const dsa_rag
     t.samp = samp;
     t.ld_s = g.ld_s;
     t.thr = f.thr;
+    t.khi = f.khi;
     t.fb_list = f.list;
     StageScope scope(1, stream);
     topk_thr_kernel<<<(unsigned)((q_count + kThrWarps - 1) / kThrWarps), 32 * kThrWarps, 0,
@@ -565,6 +569,8 @@ dsa_status fused_pass(const DeviceState& dev, const dsa_params* P, const dsa_rag
   a.cand = reinterpret_cast<const float2*>(f.sc);
   a.cap = g.cap;
   a.cand_cnt = f.ccnt;
+  a.thr = f.thr;
+  a.khi = f.khi;
   a.fb_list = f.list;
   a.q_idx = q_idx;
   a.k_idx = k_idx;

@@ -94,6 +94,8 @@ struct TopkArgs {
   const float2* cand;       // [q_count, cap]: 4 segments of cap/4 (position bits, score)
   int cap;
   const int32_t* cand_cnt;  // [q_count, 4] per segment
+  const float* thr;         // [q_count] the candidates' threshold (every candidate >= it)
+  const uint32_t* khi;      // [q_count] largest sample key of the row, 0 if not sampled
   int32_t* fb_list;         // [1 + q_count]: count, then rows (within the launch) to redo
   int blk_shift;            // rows of block scores: n = (p >> blk_shift) + 1 entries
   int prefetch_ahead;       // fused selection: warm L2 with the candidates of the row this
@@ -125,6 +127,7 @@ struct TopkThrArgs {
   const float* samp;  // [q_count, ld_s]
   int64_t ld_s;
   float* thr;         // [q_count]
+  uint32_t* khi;      // [q_count] largest sample key (0: the row was not sampled)
   int32_t* fb_list;   // its count is reset here
 };
 
@@ -616,14 +619,18 @@ DSA_DEV void topk_scores_row(const TopkArgs& a, int nn, const float* row, int32_
 // Fused selection over the row's candidates: cnt[s] <= seg of them at the start of segment s
 // (seg slots each) of cl, C = sum >= K in all, nn <= kTopkFusedMaxN.  Keys are mapped onto
 // the full 32-bit range by the order-preserving (key - kmin) << clz(kmax - kmin), so that
-// the 12-bit digit spreads although all candidates lie close together.  Returns false
-// (nothing written) when the threshold bin holds more than kTopkBinMax candidates.
+// the 12-bit digit spreads although all candidates lie close together.  A sampled row brings
+// its range: every candidate is >= the threshold, key k_lo, and about 16 of them exceed the
+// largest sample, key k_hi; keys are clamped into [k_lo, k_hi] for the binning only (the top
+// bin takes those few), and the threshold bin is ranked on the exact keys.  Other rows
+// (k_hi = 0) take the range in a first pass.  Returns false (nothing written) when the
+// threshold bin holds more than kTopkBinMax candidates.
 // kFusedThreads threads: each quarter of the block reads one segment in every pass (the key
 // range, the histogram, the marking), straight from global memory -- the first pass brings
 // the row's candidates into L2, the later ones hit there.
 DSA_DEV bool topk_candidates_row(const TopkArgs& a, int nn, const float2* cl, int seg,
-                                 const uint32_t (&cnt)[4], uint32_t C, int32_t* out,
-                                 uint32_t* dyn, TopkShared& sh) {
+                                 const uint32_t (&cnt)[4], uint32_t C, uint32_t k_lo,
+                                 uint32_t k_hi, int32_t* out, uint32_t* dyn, TopkShared& sh) {
   constexpr int kQuarter = kFusedThreads / 4;
   uint32_t* h = dyn;                     // [4096]
   uint32_t* bm = h + 4096;               // [bm_words] selected positions
@@ -651,30 +658,40 @@ DSA_DEV bool topk_candidates_row(const TopkArgs& a, int nn, const float2* cl, in
         if (e0 + (uint32_t)kQuarter * u < ns) f(topk_key(e[u].y), (uint32_t)__float_as_int(e[u].x));
     }
   };
+  const bool ranged = k_hi != 0u && k_hi >= k_lo;  // uniform
   uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-  for_cands([&](uint32_t key, uint32_t) {
-    lo = key < lo ? key : lo;
-    hi = key > hi ? key : hi;
-  });
+  if (!ranged)
+    for_cands([&](uint32_t key, uint32_t) {
+      lo = key < lo ? key : lo;
+      hi = key > hi ? key : hi;
+    });
   for (int t = tid; t < 1024; t += kFusedThreads)
     reinterpret_cast<uint4*>(h)[t] = make_uint4(0u, 0u, 0u, 0u);
   for (int t = tid; t < W; t += kFusedThreads) bm[t] = 0;
   if (tid == 0) {
-    sh.kmin = 0xFFFFFFFFu;
-    sh.kmax = 0u;
+    sh.kmin = ranged ? k_lo : 0xFFFFFFFFu;
+    sh.kmax = ranged ? k_hi : 0u;
     sh.ncand = 0;
   }
-  lo = __reduce_min_sync(0xFFFFFFFFu, lo);
-  hi = __reduce_max_sync(0xFFFFFFFFu, hi);
-  __syncthreads();  // kmin / kmax initialised, histogram and bitmap zeroed
-  if (lane == 0) {
-    atomicMin(&sh.kmin, lo);
-    atomicMax(&sh.kmax, hi);
+  if (!ranged) {
+    lo = __reduce_min_sync(0xFFFFFFFFu, lo);
+    hi = __reduce_max_sync(0xFFFFFFFFu, hi);
+    __syncthreads();  // kmin / kmax initialised
+    if (lane == 0) {
+      atomicMin(&sh.kmin, lo);
+      atomicMax(&sh.kmax, hi);
+    }
   }
-  __syncthreads();
-  const uint32_t kmin = sh.kmin, span = sh.kmax - sh.kmin;
+  __syncthreads();  // range known, histogram and bitmap zeroed
+  const uint32_t kmin = sh.kmin, kmax = sh.kmax, span = kmax - kmin;
   const int z = span ? __clz(span) : 0;
-  for_cands([&](uint32_t key, uint32_t) { atomicAdd(&h[((key - kmin) << z) >> 20], 1u); });
+  // order-preserving map of a key onto the 32-bit range (clamped to [kmin, kmax])
+  auto norm = [&](uint32_t key) -> uint32_t {
+    key = key < kmin ? kmin : key;
+    key = key > kmax ? kmax : key;
+    return (key - kmin) << z;
+  };
+  for_cands([&](uint32_t key, uint32_t) { atomicAdd(&h[norm(key) >> 20], 1u); });
   __syncthreads();
   if (warp == 0) warp_select<4096>(h, (uint32_t)a.K, sh.sel);
   __syncthreads();
@@ -687,13 +704,13 @@ DSA_DEV bool topk_candidates_row(const TopkArgs& a, int nn, const float2* cl, in
   // workspace can hold, are skipped: they never index the bitmap.)
   for_cands([&](uint32_t key, uint32_t pos) {
     if (pos >= (uint32_t)nn) return;
-    const uint32_t nk = (key - kmin) << z, bin = nk >> 20;
+    const uint32_t bin = norm(key) >> 20;
     if (bin > b || (whole && bin == b)) {
       atomicOr(&bm[pos >> 5], 1u << (pos & 31u));
     } else if (bin == b) {
       const uint32_t slot = atomicAdd(&sh.ncand, 1u);
       if (slot < (uint32_t)kTopkBinMax) {
-        bk[slot] = nk;
+        bk[slot] = key;  // the exact key: clamping may have merged keys of the top bin
         bp[slot] = pos;
       }
     }
@@ -879,8 +896,11 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedCtasPerSm) topk_fused_ker
   const uint32_t C = cnt[0] + cnt[1] + cnt[2] + cnt[3];
   const bool over = cnt[0] > (uint32_t)seg || cnt[1] > (uint32_t)seg || cnt[2] > (uint32_t)seg ||
                     cnt[3] > (uint32_t)seg;
+  const uint32_t k_hi = a.khi ? __ldg(a.khi + i) : 0u;
+  const uint32_t k_lo = k_hi ? topk_key(__ldg(a.thr + i)) : 0u;
   if (over || C < (uint32_t)K ||
-      !topk_candidates_row(a, (int)n, a.cand + i * (int64_t)a.cap, seg, cnt, C, out, dyn, sh)) {
+      !topk_candidates_row(a, (int)n, a.cand + i * (int64_t)a.cap, seg, cnt, C, k_lo, k_hi, out,
+                           dyn, sh)) {
     if (tid == 0) a.fb_list[1 + atomicAdd(a.fb_list, 1)] = (int32_t)i;
     return;
   }
@@ -982,7 +1002,10 @@ __global__ void __launch_bounds__(32 * kThrWarps) topk_thr_kernel(TopkThrArgs a)
   const int64_t p = L - (qn - qo) + (r - qo);
   const int64_t n = p + 1;
   if (n <= a.K || n <= a.cap) {
-    if (lane == 0) a.thr[i] = n <= a.K ? INFINITY : -INFINITY;
+    if (lane == 0) {
+      a.thr[i] = n <= a.K ? INFINITY : -INFINITY;
+      a.khi[i] = 0u;
+    }
     return;
   }
   const int S = (int)(p >> a.shift) + 1;
@@ -1083,7 +1106,10 @@ __global__ void __launch_bounds__(32 * kThrWarps) topk_thr_kernel(TopkThrArgs a)
     for (int q = 0; q < 8; ++q) h[lane * 8 + q] = 0;
     __syncwarp();
   }
-  if (lane == 0) a.thr[i] = topk_key_value(lo + (prefix >> z));
+  if (lane == 0) {
+    a.thr[i] = topk_key_value(lo + (prefix >> z));
+    a.khi[i] = hi;
+  }
 }
 
 }  // namespace dsa
