@@ -868,6 +868,10 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedCtasPerSm) topk_fused_ker
   const int K = a.K;
   const int64_t i = a.q_count - 1 - (int64_t)blockIdx.x;
   const int64_t r = a.q_begin + i;
+  // the row's counts and range do not depend on its length: load them with it
+  const int4 c4 = __ldg(reinterpret_cast<const int4*>(a.cand_cnt) + i);
+  const uint32_t k_hi = a.khi ? __ldg(a.khi + i) : 0u;
+  const float thr_i = __ldg(a.thr + i);
   int b;
   const int64_t n = topk_row_len(a, r, &b);
   int32_t* out = a.idx + i * a.ld_idx;
@@ -877,7 +881,7 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedCtasPerSm) topk_fused_ker
     return;
   }
   const int seg = a.cap >> 2;
-  if (tid == 0 && a.prefetch_ahead > 0 && i >= a.prefetch_ahead) {
+  if (tid == kFusedThreads - 32 && a.prefetch_ahead > 0 && i >= a.prefetch_ahead) {
     // the CTA that will take row i2 starts about when this one ends: pull its candidate
     // segments towards L2 now (a hint only; nothing waits for it)
     const int64_t i2 = i - a.prefetch_ahead;
@@ -891,13 +895,11 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedCtasPerSm) topk_fused_ker
                          (uint32_t)(((int64_t)n * 8 + 15) & ~int64_t(15)));
     }
   }
-  const int4 c4 = __ldg(reinterpret_cast<const int4*>(a.cand_cnt) + i);
   const uint32_t cnt[4] = {(uint32_t)c4.x, (uint32_t)c4.y, (uint32_t)c4.z, (uint32_t)c4.w};
   const uint32_t C = cnt[0] + cnt[1] + cnt[2] + cnt[3];
   const bool over = cnt[0] > (uint32_t)seg || cnt[1] > (uint32_t)seg || cnt[2] > (uint32_t)seg ||
                     cnt[3] > (uint32_t)seg;
-  const uint32_t k_hi = a.khi ? __ldg(a.khi + i) : 0u;
-  const uint32_t k_lo = k_hi ? topk_key(__ldg(a.thr + i)) : 0u;
+  const uint32_t k_lo = k_hi ? topk_key(thr_i) : 0u;
   if (over || C < (uint32_t)K ||
       !topk_candidates_row(a, (int)n, a.cand + i * (int64_t)a.cap, seg, cnt, C, k_lo, k_hi, out,
                            dyn, sh)) {
