@@ -644,8 +644,8 @@ DSA_DEV bool topk_candidates_row(const TopkArgs& a, int nn, const float2* cl, in
   const float2* src = cl + (int64_t)sg * seg;
   const uint32_t x0 = (uint32_t)(tid % kQuarter);
   constexpr uint32_t kStep = (uint32_t)kQuarter * kTopkCandBatch;
-  // one pass over this thread's candidates, kTopkCandBatch loads in flight
-  auto for_cands = [&](auto&& f) {
+  // one pass over this thread's candidates (score, position), kTopkCandBatch loads in flight
+  auto for_pairs = [&](auto&& f) {
     for (uint32_t e0 = x0; e0 < ns; e0 += kStep) {
       float2 e[kTopkCandBatch];
 #pragma unroll
@@ -655,8 +655,11 @@ DSA_DEV bool topk_candidates_row(const TopkArgs& a, int nn, const float2* cl, in
       }
 #pragma unroll
       for (int u = 0; u < kTopkCandBatch; ++u)
-        if (e0 + (uint32_t)kQuarter * u < ns) f(topk_key(e[u].y), (uint32_t)__float_as_int(e[u].x));
+        if (e0 + (uint32_t)kQuarter * u < ns) f(e[u].y, (uint32_t)__float_as_int(e[u].x));
     }
+  };
+  auto for_cands = [&](auto&& f) {
+    for_pairs([&](float x, uint32_t pos) { f(topk_key(x), pos); });
   };
   const bool ranged = k_hi != 0u && k_hi >= k_lo;  // uniform
   uint32_t lo = 0xFFFFFFFFu, hi = 0u;
@@ -700,17 +703,31 @@ DSA_DEV bool topk_candidates_row(const TopkArgs& a, int nn, const float2* cl, in
   const uint32_t n_bin = h[b];
   if (!whole && n_bin > (uint32_t)kTopkBinMax) return false;  // uniform
   // keys in higher bins (or the whole threshold bin) are selected; the threshold bin's
-  // keys are set aside for ranking.  (Positions outside the row, which only a corrupted
-  // workspace can hold, are skipped: they never index the bitmap.)
-  for_cands([&](uint32_t key, uint32_t pos) {
+  // keys are set aside for ranking.  The bins are intervals of keys: a (clamped) key's bin
+  // is >= bb iff the key is >= kmin + ceil(bb 2^20 / 2^z), so with the order-preserving key
+  // map (-0.0 == +0.0) two float compares against the bounds of bins b and b + 1 classify a
+  // candidate, and only the threshold bin's few candidates form their key.  Keys above kmax
+  // share the bin of kmax (bin_top), keys below kmin (none but in a corrupted workspace) bin 0,
+  // as in the histogram.  (Positions outside the row, which only a corrupted workspace can
+  // hold, are skipped: they never index the bitmap.)
+  auto first_key = [&](uint32_t bb) -> uint32_t {
+    return (uint32_t)((uint64_t)kmin + ((((uint64_t)bb << 20) + ((1ull << z) - 1ull)) >> z));
+  };
+  const uint32_t bin_top = (span << z) >> 20;
+  const bool none_above = b >= bin_top;  // no key lies in a bin above b
+  const bool all_from_b = b == 0;         // every key lies in bin b or above
+  const float f_above = none_above ? 0.f : topk_key_value(first_key(b + 1));
+  const float f_in_b = all_from_b ? 0.f : topk_key_value(first_key(b));
+  for_pairs([&](float x, uint32_t pos) {
     if (pos >= (uint32_t)nn) return;
-    const uint32_t bin = norm(key) >> 20;
-    if (bin > b || (whole && bin == b)) {
+    const bool above = !none_above && x >= f_above;
+    const bool in_b = !above && (all_from_b || x >= f_in_b);
+    if (above || (whole && in_b)) {
       atomicOr(&bm[pos >> 5], 1u << (pos & 31u));
-    } else if (bin == b) {
+    } else if (in_b) {
       const uint32_t slot = atomicAdd(&sh.ncand, 1u);
       if (slot < (uint32_t)kTopkBinMax) {
-        bk[slot] = key;  // the exact key: clamping may have merged keys of the top bin
+        bk[slot] = topk_key(x);  // the exact key: clamping may have merged keys of the top bin
         bp[slot] = pos;
       }
     }
