@@ -749,19 +749,36 @@ DSA_DEV bool topk_candidates_row(const TopkArgs& a, int nn, const float2* cl, in
     }
   }
   __syncthreads();
-  // ascending output: each thread writes the positions of its run of bitmap words
+  // ascending output: each thread lists the positions of its run of bitmap words, into the
+  // histogram's words (free since the bin pick) when the row fits there, and the row then
+  // leaves in coalesced stores.  (At most K bits are set: the bins above b hold fewer than
+  // K candidates, the ranking marks the rest, and a position is marked once.)
   const int wpt = (W + kFusedThreads - 1) / kFusedThreads;
   const int w0 = tid * wpt, w1 = w0 + wpt < W ? w0 + wpt : W;
   uint32_t mine = 0;
   for (int w = w0; w < w1; ++w) mine += __popc(bm[w]);
   uint32_t total;
   uint32_t at = block_scan_w<kFusedWarps>(mine, sh.tot, bank, total);
+  const bool staged = a.K <= 4096;  // uniform
+  uint32_t* ob = h;
   for (int w = w0; w < w1; ++w) {
     uint32_t bits = bm[w];
     while (bits) {
       const int q = __ffs(bits) - 1;
       bits &= bits - 1;
-      out[at++] = w * 32 + q;
+      if (staged) ob[at] = (uint32_t)(w * 32 + q);
+      else out[at] = w * 32 + q;
+      ++at;
+    }
+  }
+  if (staged) {
+    __syncthreads();
+    const uint32_t n_out = total < (uint32_t)a.K ? total : (uint32_t)a.K;
+    if ((reinterpret_cast<uintptr_t>(out) & 15u) == 0 && (n_out & 3u) == 0) {
+      for (uint32_t j = tid; j < n_out / 4; j += kFusedThreads)
+        reinterpret_cast<int4*>(out)[j] = reinterpret_cast<const int4*>(ob)[j];
+    } else {
+      for (uint32_t j = tid; j < n_out; j += kFusedThreads) out[j] = (int32_t)ob[j];
     }
   }
   return true;
