@@ -86,10 +86,15 @@ __host__ inline size_t attn_smem_bytes() {
          128 /*align*/;
 }
 
-// OFF32: each of the K and V caches spans at most 4 GiB, so a selected row's piece is addressed
-// as the cache's base plus a 32-bit byte offset (one shuffle and one add per piece instead of
-// 64-bit address arithmetic for K and for V).
-template <int HKV_CTA, int NT, bool OFF32>
+// How a selected row's 16-byte pieces are addressed (AM): kAddr64, 64-bit arithmetic per piece
+// for K and for V; kAddrBytes32, each cache spans at most 4 GiB, so a piece is the cache's base
+// plus a shuffled 32-bit byte offset; kAddrUnits32, each cache spans at most 64 GiB, the same
+// with the offset counted in 16-byte units.
+constexpr int kAddr64 = 0;
+constexpr int kAddrBytes32 = 1;
+constexpr int kAddrUnits32 = 2;
+
+template <int HKV_CTA, int NT, int AM>
 __global__ void __launch_bounds__(AttnGeom<HKV_CTA>::kThreads, AttnShape<HKV_CTA>::kCtasPerSm)
     sparse_attn_kernel(AttnArgs a) {
   using Geo = AttnGeom<HKV_CTA>;
@@ -154,8 +159,11 @@ __global__ void __launch_bounds__(AttnGeom<HKV_CTA>::kThreads, AttnShape<HKV_CTA
   const int64_t v_minus_k = a.v - a.k;  // V row = K row + this many elements
   const __nv_bfloat16* kpiece = kh + lt * 8;  // this lane's piece of cache row 0
   const uint32_t swz = (uint32_t)((lt ^ lhi) << 4);  // lt ^ ((2k + lhi) & 7) = (lt ^ lhi) ^ 2k&7
-  const uint32_t row_bytes = (uint32_t)row_stride * 2u;                          // OFF32 only
-  const uint32_t piece_off = (uint32_t)((hg * kHeadDim + lt * 8) * 2);          // OFF32 only
+  // 32-bit addressing: a cache row's size and this lane's piece within it, in bytes or in
+  // 16-byte units
+  constexpr uint32_t kUnit = AM == kAddrUnits32 ? 16u : 1u;
+  const uint32_t row_off = (uint32_t)row_stride * 2u / kUnit;
+  const uint32_t piece_off = (uint32_t)((hg * kHeadDim + lt * 8) * 2) / kUnit;
   const char* kb = reinterpret_cast<const char*>(a.k);
   const char* vb = reinterpret_cast<const char*>(a.v);
   auto load_chunk = [&](int c, int st) -> uint32_t {
@@ -168,14 +176,19 @@ __global__ void __launch_bounds__(AttnGeom<HKV_CTA>::kThreads, AttnShape<HKV_CTA
                                    : (int)kbase + (valid ? j : 0);
     const uint32_t kdst = smem_u32(wsm + st * Geo::kWarpStage) + lhi * 256;
     const uint32_t vdst = kdst + Geo::kWarpHalf;
-    if (OFF32) {
-      const uint32_t myoff = (uint32_t)rowi * row_bytes;
+    if (AM != kAddr64) {
+      const uint32_t myoff = (uint32_t)rowi * row_off;
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const uint32_t off = __shfl_sync(0xFFFFFFFFu, myoff, 2 * k + lhi) + piece_off;
         const uint32_t so = (uint32_t)(k * 512) + (swz ^ (uint32_t)(((2 * k) & 7) << 4));
-        cp_async_16(kdst + so, kb + off, 16u);
-        cp_async_16(vdst + so, vb + off, 16u);
+        if (AM == kAddrUnits32) {
+          cp_async_16(kdst + so, reinterpret_cast<const uint4*>(kb) + off, 16u);
+          cp_async_16(vdst + so, reinterpret_cast<const uint4*>(vb) + off, 16u);
+        } else {
+          cp_async_16(kdst + so, kb + off, 16u);
+          cp_async_16(vdst + so, vb + off, 16u);
+        }
       }
     } else {
 #pragma unroll
