@@ -25,7 +25,9 @@ extern "C" {
  *   idx      device int32 scratch of n_idx entries (a power of two, >= 32): receives the row
  *            indices (a counter-based hash masked to n_rows, so every access is in bounds)
  *   variant  0: loads into registers (all 16 row pairs of a 32-row chunk in flight);
- *            1: cp.async into a shared-memory ring of two chunks per warp
+ *            1: cp.async into a shared-memory ring of two chunks per warp;
+ *            2, 3: as 0, 1 with each piece addressed by a 32-bit index of 16-byte units
+ *            added to buf (n_rows <= 2^28) instead of 64-bit arithmetic
  *   blocks   CTAs of 256 threads; chunks_per_warp chunks of 32 rows per warp
  *   reps     timed launches after one untimed launch
  *   sink     device scratch of >= blocks * 256 16-byte words (written only in a case that

@@ -55,9 +55,10 @@ def gather_peaks(num_sms: int, l2_bytes: int = 64 << 20, hbm_bytes: int = 8 << 3
     out = {}
     for name, size in (("l2", l2_bytes), ("hbm", hbm_bytes)):
         tries = {}
-        for variant, blocks in ((1, num_sms), (0, num_sms * 8)):
-            tries[f"{'cp.async smem' if variant else 'ld.global regs'} x{blocks} CTAs"] = \
-                gather_rate(size, variant, blocks)
+        for variant, blocks in ((1, num_sms), (0, num_sms * 8), (3, num_sms), (2, num_sms * 8)):
+            kind = "cp.async smem" if variant & 1 else "ld.global regs"
+            addr = ", 32-bit index" if variant >= 2 else ""
+            tries[f"{kind}{addr} x{blocks} CTAs"] = gather_rate(size, variant, blocks)
         best = max(tries, key=tries.get)
         out[name] = {"gbs": tries[best], "best": best, "tried": tries, "buffer_bytes": size}
     return out

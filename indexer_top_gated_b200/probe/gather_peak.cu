@@ -32,8 +32,17 @@ __global__ void fill_rows_kernel(int32_t* idx, uint32_t n_idx, uint32_t row_mask
     idx[i] = (int32_t)(mix64(seed ^ i) & row_mask);
 }
 
+// Address of piece lt of row r: 64-bit arithmetic, or (IDX32) a 32-bit index of 16-byte
+// units (buffers up to 64 GiB) added to the base.
+template <bool IDX32>
+__device__ __forceinline__ const uint4* piece(const uint4* buf, int r, int lt) {
+  if (IDX32) return buf + ((uint32_t)r * 16u + (uint32_t)lt);
+  return buf + (int64_t)r * 16 + lt;
+}
+
 // Warp w handles chunks c = 0 .. chunks_per_warp-1, each 32 row indices starting at
 // ((w * chunks_per_warp + c) * 32) & idx_mask of idx.
+template <bool IDX32>
 __global__ void __launch_bounds__(256) gather_regs_kernel(const uint4* __restrict__ buf,
                                                           const int32_t* __restrict__ idx,
                                                           uint32_t idx_mask, int chunks_per_warp,
@@ -48,7 +57,7 @@ __global__ void __launch_bounds__(256) gather_regs_kernel(const uint4* __restric
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
       const int r = __shfl_sync(0xFFFFFFFFu, row, 2 * k + lhi);
-      v[k] = __ldg(buf + (int64_t)r * 16 + lt);
+      v[k] = __ldg(piece<IDX32>(buf, r, lt));
     }
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
@@ -61,6 +70,7 @@ __global__ void __launch_bounds__(256) gather_regs_kernel(const uint4* __restric
   if ((acc.x & acc.y & acc.z & acc.w) == 0xFFFFFFFFu) sink[gw * 32 + lane] = acc;  // keeps the loads
 }
 
+template <bool IDX32>
 __global__ void __launch_bounds__(256) gather_smem_kernel(const uint4* __restrict__ buf,
                                                           const int32_t* __restrict__ idx,
                                                           uint32_t idx_mask, int chunks_per_warp,
@@ -78,7 +88,7 @@ __global__ void __launch_bounds__(256) gather_smem_kernel(const uint4* __restric
       const int r = __shfl_sync(0xFFFFFFFFu, row, 2 * k + lhi);
       const uint32_t dst = (uint32_t)__cvta_generic_to_shared(slot + k * 32 + lane);
       asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
-                   "l"(buf + (int64_t)r * 16 + lt)
+                   "l"(piece<IDX32>(buf, r, lt))
                    : "memory");
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
@@ -114,22 +124,28 @@ double dsa_probe_gather(const void* buf, uint32_t n_rows, int32_t* idx, uint32_t
                         int variant, int blocks, int chunks_per_warp, int reps, void* sink) {
   if (!buf || !idx || !sink || n_rows == 0 || (n_rows & (n_rows - 1)) || n_idx < 32 ||
       (n_idx & (n_idx - 1)) || blocks < 1 || chunks_per_warp < 1 || reps < 1 ||
-      (variant != 0 && variant != 1))
+      variant < 0 || variant > 3 || (variant >= 2 && n_rows > (1u << 28)))
     return 0.0;
   if ((reinterpret_cast<uintptr_t>(buf) & 15) || (reinterpret_cast<uintptr_t>(sink) & 15))
     return 0.0;
   fill_rows_kernel<<<256, 256>>>(idx, n_idx, n_rows - 1, 0x5EEDull);
-  if (variant == 1 &&
-      cudaFuncSetAttribute(gather_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kSmemRing) != cudaSuccess)
+  if ((variant & 1) &&
+      (cudaFuncSetAttribute(gather_smem_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            (int)kSmemRing) != cudaSuccess ||
+       cudaFuncSetAttribute(gather_smem_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            (int)kSmemRing) != cudaSuccess))
     return 0.0;
   const uint4* b = static_cast<const uint4*>(buf);
   uint4* s = static_cast<uint4*>(sink);
   auto launch = [&]() {
     if (variant == 0)
-      gather_regs_kernel<<<blocks, 256>>>(b, idx, n_idx - 1, chunks_per_warp, s);
+      gather_regs_kernel<false><<<blocks, 256>>>(b, idx, n_idx - 1, chunks_per_warp, s);
+    else if (variant == 1)
+      gather_smem_kernel<false><<<blocks, 256, kSmemRing>>>(b, idx, n_idx - 1, chunks_per_warp, s);
+    else if (variant == 2)
+      gather_regs_kernel<true><<<blocks, 256>>>(b, idx, n_idx - 1, chunks_per_warp, s);
     else
-      gather_smem_kernel<<<blocks, 256, kSmemRing>>>(b, idx, n_idx - 1, chunks_per_warp, s);
+      gather_smem_kernel<true><<<blocks, 256, kSmemRing>>>(b, idx, n_idx - 1, chunks_per_warp, s);
   };
   cudaEvent_t e0 = nullptr, e1 = nullptr;
   double result = 0.0;

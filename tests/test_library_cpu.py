@@ -252,3 +252,6 @@ def test_probe_library_exports_its_declared_entry_point():
     # n_rows not a power of two / null buffers: rejected on the host
     assert L.dsa_probe_gather(0x1000, 3, 0x2000, 64, 0, 1, 1, 1, 0x3000) == 0.0
     assert L.dsa_probe_gather(None, 4, 0x2000, 64, 0, 1, 1, 1, 0x3000) == 0.0
+    # unknown variant; a 32-bit index of 16-byte units covers at most 2^28 rows of 256 B
+    assert L.dsa_probe_gather(0x1000, 4, 0x2000, 64, 4, 1, 1, 1, 0x3000) == 0.0
+    assert L.dsa_probe_gather(0x1000, 1 << 29, 0x2000, 64, 2, 1, 1, 1, 0x3000) == 0.0
