@@ -248,6 +248,10 @@ dsa_status dsa_index_topk_blocks(const dsa_params* params, const dsa_ragged* rag
  * weights enter the P.V product rounded to bf16 (fp32 accumulation), and out is rounded
  * to bf16 (nearest even).  A row's result does not depend on q_begin / q_count (how the
  * rows are split into calls).
+ * Addressing of the gathered rows: a 32-bit offset per row when each of k_cache and v_cache
+ * spans at most 64 GiB, a general form otherwise; the environment variable
+ * DSA_ATTN_ADDR_ROWS=1 (read once per process) forces the general form, for tests.  The
+ * choice changes no result bit.
  * Requirements: q, k_cache, v_cache, gate, out 16-byte aligned.
  */
 dsa_status dsa_sparse_attn_gated(const dsa_params* params, const dsa_ragged* ragged,

@@ -7,6 +7,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -162,14 +163,14 @@ dsa_status device_setup(DeviceState** out) {
     e = e ? e : allow_smem(topk_kernel<kTopkScores>, topk_smem_bytes(0));
     e = e ? e : allow_smem(topk_fused_kernel, topk_fused_smem_bytes(kTopkFastCap, kTopkFusedMaxN));
     e = e ? e : allow_smem(topk_kernel<kTopkFallback>, topk_smem_bytes(0));
-    e = e ? e : allow_smem(sparse_attn_kernel<1, 1, kAddr64>, attn_smem_bytes());
-    e = e ? e : allow_smem(sparse_attn_kernel<2, 1, kAddr64>, attn_smem_bytes());
-    e = e ? e : allow_smem(sparse_attn_kernel<1, 2, kAddr64>, attn_smem_bytes());
-    e = e ? e : allow_smem(sparse_attn_kernel<2, 2, kAddr64>, attn_smem_bytes());
     e = e ? e : allow_smem(sparse_attn_kernel<1, 1, kAddrBytes32>, attn_smem_bytes());
     e = e ? e : allow_smem(sparse_attn_kernel<2, 1, kAddrBytes32>, attn_smem_bytes());
     e = e ? e : allow_smem(sparse_attn_kernel<1, 2, kAddrBytes32>, attn_smem_bytes());
     e = e ? e : allow_smem(sparse_attn_kernel<2, 2, kAddrBytes32>, attn_smem_bytes());
+    e = e ? e : allow_smem(sparse_attn_kernel<1, 1, kAddrRows>, attn_smem_bytes());
+    e = e ? e : allow_smem(sparse_attn_kernel<2, 1, kAddrRows>, attn_smem_bytes());
+    e = e ? e : allow_smem(sparse_attn_kernel<1, 2, kAddrRows>, attn_smem_bytes());
+    e = e ? e : allow_smem(sparse_attn_kernel<2, 2, kAddrRows>, attn_smem_bytes());
     e = e ? e : allow_smem(sparse_attn_kernel<1, 1, kAddrUnits32>, attn_smem_bytes());
     e = e ? e : allow_smem(sparse_attn_kernel<2, 1, kAddrUnits32>, attn_smem_bytes());
     e = e ? e : allow_smem(sparse_attn_kernel<1, 2, kAddrUnits32>, attn_smem_bytes());
@@ -647,26 +648,32 @@ dsa_status launch_attn(const DeviceState& dev, const dsa_params* P, const dsa_ra
   // (the warps' partial softmax states are merged in an order set by the CTA shape).
   const int hkv_cta = (decode || P->n_kv_heads == 1) ? 1 : 2;
   const int nt = a.G > 8 ? 2 : 1;
-  // 32-bit offsets: in bytes when each cache array (rows of Hkv x d bf16) spans at most 4 GiB,
-  // in 16-byte units up to 64 GiB
+  // 32-bit offsets when each cache array (rows of Hkv x d bf16) spans at most 4 GiB (bytes) or
+  // 64 GiB (16-byte units); the general form beyond, or everywhere when DSA_ATTN_ADDR_ROWS is
+  // set to a non-zero value in the environment (so that tests reach it with small caches)
   const uint64_t cache_bytes = (uint64_t)R->total_kv * (uint64_t)P->n_kv_heads * kHeadDim * 2;
-  const int am = cache_bytes <= (1ull << 32)   ? kAddrBytes32
+  static const bool force_rows = [] {
+    const char* e = std::getenv("DSA_ATTN_ADDR_ROWS");
+    return e && std::atoi(e) != 0;
+  }();
+  const int am = force_rows                    ? kAddrRows
+                 : cache_bytes <= (1ull << 32) ? kAddrBytes32
                  : cache_bytes <= (1ull << 36) ? kAddrUnits32
-                                               : kAddr64;
+                                               : kAddrRows;
   dim3 grid((unsigned)q_count, (unsigned)(P->n_kv_heads / hkv_cta));
   const size_t smem = attn_smem_bytes();
   StageScope scope(2, stream);
 #define DSA_ATTN_CASE(H, N, O)                                                      \
   if (hkv_cta == H && nt == N && am == O)                                           \
     sparse_attn_kernel<H, N, O><<<grid, AttnGeom<H>::kThreads, smem, stream>>>(a);
-  DSA_ATTN_CASE(1, 1, kAddr64)
-  DSA_ATTN_CASE(2, 1, kAddr64)
-  DSA_ATTN_CASE(1, 2, kAddr64)
-  DSA_ATTN_CASE(2, 2, kAddr64)
   DSA_ATTN_CASE(1, 1, kAddrBytes32)
   DSA_ATTN_CASE(2, 1, kAddrBytes32)
   DSA_ATTN_CASE(1, 2, kAddrBytes32)
   DSA_ATTN_CASE(2, 2, kAddrBytes32)
+  DSA_ATTN_CASE(1, 1, kAddrRows)
+  DSA_ATTN_CASE(2, 1, kAddrRows)
+  DSA_ATTN_CASE(1, 2, kAddrRows)
+  DSA_ATTN_CASE(2, 2, kAddrRows)
   DSA_ATTN_CASE(1, 1, kAddrUnits32)
   DSA_ATTN_CASE(2, 1, kAddrUnits32)
   DSA_ATTN_CASE(1, 2, kAddrUnits32)

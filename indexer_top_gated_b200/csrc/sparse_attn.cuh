@@ -86,13 +86,14 @@ __host__ inline size_t attn_smem_bytes() {
          128 /*align*/;
 }
 
-// How a selected row's 16-byte pieces are addressed (AM): kAddr64, 64-bit arithmetic per piece
-// for K and for V; kAddrBytes32, each cache spans at most 4 GiB, so a piece is the cache's base
-// plus a shuffled 32-bit byte offset; kAddrUnits32, each cache spans at most 64 GiB, the same
-// with the offset counted in 16-byte units.
-constexpr int kAddr64 = 0;
+// How a selected row's 16-byte pieces are addressed (AM): kAddrBytes32, each cache spans at
+// most 4 GiB, so a piece is the cache's base plus a shuffled 32-bit byte offset;
+// kAddrUnits32, at most 64 GiB, the same with the offset in 16-byte units; kAddrRows, any
+// size: the shuffled 32-bit row index times the row's size in 16-byte units, widened to 64
+// bits per piece and array.
 constexpr int kAddrBytes32 = 1;
 constexpr int kAddrUnits32 = 2;
+constexpr int kAddrRows = 3;
 
 template <int HKV_CTA, int NT, int AM>
 __global__ void __launch_bounds__(AttnGeom<HKV_CTA>::kThreads, AttnShape<HKV_CTA>::kCtasPerSm)
@@ -147,22 +148,18 @@ __global__ void __launch_bounds__(AttnGeom<HKV_CTA>::kThreads, AttnShape<HKV_CTA
   const int sub = warp % Geo::kWPG;
   const int hg = g0 + g;  // KV head
   uint8_t* wsm = smem + (size_t)warp * kAttnStages * Geo::kWarpStage;  // this warp's ring
-  const __nv_bfloat16* kh = a.k + (int64_t)hg * kHeadDim;
-  const int64_t row_stride = (int64_t)a.Hkv * kHeadDim;
+  const uint32_t row_stride = (uint32_t)a.Hkv * kHeadDim;  // elements per cache row
 
   // gather chunk c into ring slot st; returns the validity mask of its 16 positions.
   // Lane t < 16 reads the index of position t; every cp.async step then moves two whole
-  // 256-byte head slices (512 contiguous bytes per warp instruction), the row arriving by
-  // shuffle.  Padding and out-of-range entries copy the sequence's first row (finite data)
-  // and are masked in the softmax, so the copies need no per-piece predicate.
+  // 256-byte head slices (512 contiguous bytes per warp instruction), the row's offset
+  // arriving by shuffle.  Padding and out-of-range entries copy the sequence's first row
+  // (finite data) and are masked in the softmax, so the copies need no per-piece predicate.
   const int lt = lane & 15, lhi = lane >> 4;
-  const int64_t v_minus_k = a.v - a.k;  // V row = K row + this many elements
-  const __nv_bfloat16* kpiece = kh + lt * 8;  // this lane's piece of cache row 0
   const uint32_t swz = (uint32_t)((lt ^ lhi) << 4);  // lt ^ ((2k + lhi) & 7) = (lt ^ lhi) ^ 2k&7
-  // 32-bit addressing: a cache row's size and this lane's piece within it, in bytes or in
-  // 16-byte units
-  constexpr uint32_t kUnit = AM == kAddrUnits32 ? 16u : 1u;
-  const uint32_t row_off = (uint32_t)row_stride * 2u / kUnit;
+  // a cache row's size and this lane's piece within it, in bytes or in 16-byte units
+  constexpr uint32_t kUnit = AM == kAddrBytes32 ? 1u : 16u;
+  const uint32_t row_off = row_stride * 2u / kUnit;
   const uint32_t piece_off = (uint32_t)((hg * kHeadDim + lt * 8) * 2) / kUnit;
   const char* kb = reinterpret_cast<const char*>(a.k);
   const char* vb = reinterpret_cast<const char*>(a.v);
@@ -176,7 +173,7 @@ __global__ void __launch_bounds__(AttnGeom<HKV_CTA>::kThreads, AttnShape<HKV_CTA
                                    : (int)kbase + (valid ? j : 0);
     const uint32_t kdst = smem_u32(wsm + st * Geo::kWarpStage) + lhi * 256;
     const uint32_t vdst = kdst + Geo::kWarpHalf;
-    if (AM != kAddr64) {
+    if (AM != kAddrRows) {
       const uint32_t myoff = (uint32_t)rowi * row_off;
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
@@ -193,11 +190,11 @@ __global__ void __launch_bounds__(AttnGeom<HKV_CTA>::kThreads, AttnShape<HKV_CTA
     } else {
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        const int rt = __shfl_sync(0xFFFFFFFFu, rowi, 2 * k + lhi);
-        const __nv_bfloat16* src = kpiece + (int64_t)rt * row_stride;
+        const uint32_t rt = (uint32_t)__shfl_sync(0xFFFFFFFFu, rowi, 2 * k + lhi);
+        const uint64_t off = (uint64_t)rt * row_off + piece_off;
         const uint32_t so = (uint32_t)(k * 512) + (swz ^ (uint32_t)(((2 * k) & 7) << 4));
-        cp_async_16(kdst + so, src, 16u);
-        cp_async_16(vdst + so, src + v_minus_k, 16u);
+        cp_async_16(kdst + so, reinterpret_cast<const uint4*>(kb) + off, 16u);
+        cp_async_16(vdst + so, reinterpret_cast<const uint4*>(vb) + off, 16u);
       }
     }
     return vmask;
