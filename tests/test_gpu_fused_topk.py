@@ -131,6 +131,25 @@ def test_index_topk_row_window_row_weights_and_wide_idx():
     np.testing.assert_array_equal(cnt, ref_cnt)
 
 
+@pytest.mark.parametrize("weights", [(1.0, -0.5, 0.25, -1.0), (-0.25, -1.0, -0.5, -0.125)])
+def test_index_topk_negative_and_mixed_sign_weights(weights):
+    """Head weights of mixed sign, or all negative, give negative scores and thresholds, and
+    (all negative) many rows whose best scores are exact zeros: the selection's key range,
+    its clamping and the marking pass's float compares must still reproduce the materialised
+    path bit for bit."""
+    w = _workload([5000], [7000], K=256)
+    host = S.make_host_inputs(w)
+    host["w"] = np.array(weights, dtype=np.float32)
+    dev = _dev(host)
+    shape = dsa.workload_shape(w)
+    rg = _rg(w, dev)
+    ref_idx, ref_cnt = _materialised(w, shape, rg, dev, 0, w.total_q)
+    idx, cnt = _fused(w, shape, rg, dev, 0, w.total_q)
+    np.testing.assert_array_equal(idx, ref_idx)
+    np.testing.assert_array_equal(cnt, ref_cnt)
+    _check_oracle_rows(w, host, idx, 0, PT.sample_rows(w, 12, seed=4))
+
+
 def test_index_topk_threshold_misses_fall_back():
     """Rows whose q_idx is zero have all scores tied at 0: every score passes the sampled
     threshold, the candidates overflow their slots and the row is recomputed on CUDA cores
