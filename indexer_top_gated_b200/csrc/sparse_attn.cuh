@@ -7,8 +7,10 @@
 //  - gather: the warp's 16 positions x (K and V slices of its head, 256 B each) arrive
 //    through 16-byte cp.async (32 lanes = 512 contiguous bytes per instruction) into the
 //    warp's own 2-stage ring (XOR-swizzled 16-byte chunks, conflict-free for ldmatrix).
-//    Index entries are read once per position and shared across the warp by shuffles;
-//    padding / out-of-range entries are zero-filled and masked (a ballot mask).
+//    Index entries are read once per position, and the row's offset (32 bits: bytes or
+//    16-byte units, or the row index for the largest caches) is shared across the warp by
+//    shuffles; padding / out-of-range entries copy the sequence's first row (finite data)
+//    and are masked (a ballot mask).
 //  - logits are computed transposed, S^T = K_sel Q^T (mma.sync m16n8k16, keys on M, the
 //    group's 8 query heads on N, two independent accumulation chains), so a group of 8
 //    heads needs no padding and the query heads of a GQA group share the gather.

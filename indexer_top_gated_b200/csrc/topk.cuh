@@ -29,10 +29,11 @@
 // topk_fused_kernel selects among them: when the row has between K and `cap` candidates
 // they contain every score >= t, hence the whole Top-K with all of its ties, and the
 // selection is exact.  The candidates arrive in no particular order, which one radix
-// level (12 bits of the keys, spread over the candidates' range) does not need; the few
-// candidates in the threshold bin are then ranked exactly (score descending, position
-// ascending), the selected positions are marked in a bitmap over the row, and one ordered
-// scan turns it into the ascending index row.  A row whose estimate missed (fewer than
+// level (12 bits of the keys, spread over the candidates' range -- for a sampled row the
+// range the threshold kernel found) does not need; the few candidates in the threshold bin
+// are then ranked exactly (score descending, position ascending), the selected positions
+// are marked in a bitmap over the row, and one ordered scan lists them in shared memory,
+// from where the ascending index row leaves in coalesced stores.  A row whose estimate missed (fewer than
 // K candidates, or more than its slots) or whose threshold bin is too crowded goes to a
 // list that topk_kernel<kTopkFallback> works through: it recomputes the row's scores on
 // CUDA cores into a scratch row and runs the full selection on it.
@@ -57,9 +58,9 @@ __host__ inline size_t topk_smem_bytes(int64_t /*max_kv_len*/) {
   return (size_t)kTopkSmemWords * sizeof(uint32_t);
 }
 
-// Fused selection: shared memory of one CTA = a 4096-bin histogram, the candidates' keys
-// and positions (cap words each), a position bitmap of ceil(max_n / 32) words (rounded up
-// to a multiple of 4) and the threshold bin's keys and positions (kTopkBinMax each).
+// Fused selection: shared memory of one CTA = a 4096-bin histogram (which later holds the
+// listing of the index row, K <= 4096), a position bitmap of ceil(max_n / 32) words (rounded
+// up to a multiple of 4) and the threshold bin's keys and positions (kTopkBinMax each).
 constexpr int kTopkFusedMaxN = 314496;
 constexpr int kTopkCandBatch = 8;    // candidate loads in flight per thread
 constexpr int kTopkBinMax = 512;     // threshold-bin candidates ranked directly
