@@ -64,6 +64,10 @@ def parse_args():
     ap.add_argument("--also", default=",".join(EXTRA_WORKLOADS),
                     help="comma-separated workloads also measured (not the headline); '' for none")
     ap.add_argument("--no-peaks", action="store_true", help="skip the live gather-ceiling probe")
+    ap.add_argument("--seq-stride", type=int, default=1,
+                    help="keep every N-th sequence of the workload: a smaller case with the same "
+                         "mix of sequences, for profile captures of workloads whose inputs exceed "
+                         "what a capture may hold (not a bench line)")
     a = ap.parse_args()
     if a.lean:
         a.no_e2e = a.no_decode = a.no_cpu_baseline = a.no_peaks = True
@@ -206,7 +210,10 @@ def committed_traffic(kernel_file: str, summary: str, key: str = "traffic_bytes_
 ATTN_SRC = "indexer_top_gated_b200/csrc/sparse_attn.cuh"
 
 
-def attn_traffic(workload: str):
+def attn_traffic(workload: str, seq_stride: int = 1):
+    # a committed capture is of the full workload (or scaled to it): none for a reduced case
+    if seq_stride > 1:
+        return None
     return committed_traffic(ATTN_SRC, f"sparse_attn_gated_{workload}.txt")
 
 
@@ -254,7 +261,7 @@ def stage_report(w, stage_ms, stage_n, peaks, gather, fused_rows=0):
     tk_m = alg["topk_bytes_fused_moved"] / sec1 / 1e9 if sec1 > 0 else None
     tk = tk_m if fused else tk_s
     at = alg["attn_bytes"] / (stage_ms[2] / 1e3) / 1e9 if stage_ms[2] > 0 else None
-    traffic = attn_traffic(w.name)
+    traffic = attn_traffic(w.name, getattr(w, "seq_stride", 1))
     l2p = gather.get("l2", {}).get("gbs") if gather else None
     dram_gbs = traffic / stage_n[2] / (stage_ms[2] / stage_n[2] / 1e3) / 1e9 \
         if traffic and stage_ms[2] > 0 else None
@@ -367,6 +374,10 @@ def run_ours(args, rank, world, local_rank):
     dev_id = local_rank
     torch.cuda.set_device(dev_id)
     w = rank_workload(S.workload(args.workload), world, rank)
+    if args.seq_stride > 1:
+        w = _sub_workload(w, [b for b in range(w.batch) if b % args.seq_stride == 0])
+        w.needle_pos, w.needle_rows = [], []  # planted rows belong to the full layout
+        w.seq_stride = args.seq_stride
     inputs = S.make_device_inputs(w)
     shape = dsa.workload_shape(w)
     rg = dsa.ragged(inputs["q_offsets"], inputs["kv_offsets"], w.q_lens, w.kv_lens)
@@ -765,7 +776,8 @@ def main():
                                    f"whole sequences dealt to ranks by cost; no collective "
                                    f"on the data path)" if world > 1 else "dp1"),
                    "l2": l2_note(w),
-                   "workspace_bytes": res["ws_bytes"]},
+                   "workspace_bytes": res["ws_bytes"],
+                   **({"seq_stride": args.seq_stride} if args.seq_stride > 1 else {})},
         "roofline": roof,
         "stages": stages,
         "cpu_baseline": cpu,
