@@ -87,3 +87,22 @@ def test_stage_report_rooflines():
     sw = bench._sub_workload(m, [b for b, q in enumerate(m.q_lens) if q < 128])
     moved = bench.algorithmic(lw)["topk_bytes_fused_moved"] + bench.algorithmic(sw)["topk_bytes"]
     assert st[1]["achieved"] == pytest.approx(moved / 1e-3 / 1e9)
+
+
+def test_committed_attention_traffic_and_reduced_cases():
+    """Each committed attention capture parses to a full-launch DRAM traffic keyed to the
+    current kernel source; a reduced case (--seq-stride) never borrows the full launch's
+    figure, and its workload keeps every N-th sequence."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    import dsa_synth as S
+    for name in ("prefill_t32768_k2048", "prefill_t131072_needles", "mixed_serving"):
+        t = b.attn_traffic(name)
+        assert t is not None and t > 1e9, name
+        assert b.attn_traffic(name, 8) is None
+    w = S.workload("mixed_serving")
+    sw = b._sub_workload(w, [i for i in range(w.batch) if i % 8 == 0])
+    assert sw.batch == 33 and sw.q_lens[0] == 8192 and all(q == 1 for q in sw.q_lens[1:])
+    assert abs(b.algorithmic(w)["attn_bytes"] / b.algorithmic(sw)["attn_bytes"] - 8.0) < 0.05
