@@ -163,6 +163,7 @@ dsa_status device_setup(DeviceState** out) {
     e = e ? e : allow_smem(topk_kernel<kTopkScores>, topk_smem_bytes(0));
     e = e ? e : allow_smem(topk_fused_kernel, topk_fused_smem_bytes(kTopkFastCap, kTopkFusedMaxN));
     e = e ? e : allow_smem(topk_kernel<kTopkFallback>, topk_smem_bytes(0));
+    e = e ? e : allow_smem(topk_rows_alone_kernel, topk_smem_bytes(0));
     e = e ? e : allow_smem(sparse_attn_kernel<1, 1, kAddrBytes32>, attn_smem_bytes());
     e = e ? e : allow_smem(sparse_attn_kernel<2, 1, kAddrBytes32>, attn_smem_bytes());
     e = e ? e : allow_smem(sparse_attn_kernel<1, 2, kAddrBytes32>, attn_smem_bytes());
@@ -406,7 +407,13 @@ dsa_status launch_topk(const dsa_params* P, const dsa_ragged* R, const float* sc
   a.blk_shift = blk_shift;
   const size_t smem = topk_smem_bytes(R->max_kv_len);
   StageScope scope(1, stream);
-  topk_kernel<kTopkScores><<<(unsigned)q_count, kTopkThreads, smem, stream>>>(a);
+  // at most one row per SM (decode): CTAs that have their SM alone pipeline their row loads
+  DeviceState* dev = nullptr;
+  DSA_TRY(device_setup(&dev));
+  if (q_count <= dev->num_sms)
+    topk_rows_alone_kernel<<<(unsigned)q_count, kTopkThreads, smem, stream>>>(a);
+  else
+    topk_kernel<kTopkScores><<<(unsigned)q_count, kTopkThreads, smem, stream>>>(a);
   ++t_launches;
   return launch_status("topk_kernel");
 }

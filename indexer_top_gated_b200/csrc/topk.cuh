@@ -337,8 +337,10 @@ DSA_DEV float topk_ld1(const float* p) {
 
 // Top-K of one materialised score row row[0 .. nn), nn > K, into out[0 .. K).  NC: the row
 // was written by an earlier launch (read through the non-coherent cache); otherwise this
-// CTA wrote it, and it is read with coherent loads.
-template <bool NC>
+// CTA wrote it, and it is read with coherent loads.  PIPE: the candidate pass loads the
+// next run of the row while it compacts the current one (twice the registers for the
+// loads: for a CTA that has its SM alone).
+template <bool NC, bool PIPE = false>
 DSA_DEV void topk_scores_row(const TopkArgs& a, int nn, const float* row, int32_t* out,
                              uint32_t* dyn, TopkShared& sh) {
   uint32_t* hA = dyn;            // 4096: sample, top 12 bits
@@ -416,19 +418,30 @@ DSA_DEV void topk_scores_row(const TopkArgs& a, int nn, const float* row, int32_
     const float t_val = topk_key_value(t_est);
     uint32_t run = 0;
     bool overflow = false;
-    for (int cb = 0; cb < nn && !overflow; cb += kTopkRun) {
-      float4 xb[kTopkBatch];
+    // one run of kTopkRun positions: warp w owns positions cb + 1024 w .. + 1023
+    auto load_run = [&](int cb, float4 (&xr)[kTopkBatch]) {
 #pragma unroll
-      for (int it = 0; it < kTopkBatch; ++it) {  // warp w owns positions cb + 1024 w .. + 1023
+      for (int it = 0; it < kTopkBatch; ++it) {
         const int j0 = cb + warp * 1024 + it * 128 + lane * 4;
         if (j0 + 3 < nn) {
-          xb[it] = topk_ld4<NC>(row + j0);
+          xr[it] = topk_ld4<NC>(row + j0);
         } else {
-          xb[it].x = j0 < nn ? topk_ld1<NC>(row + j0) : -INFINITY;
-          xb[it].y = j0 + 1 < nn ? topk_ld1<NC>(row + j0 + 1) : -INFINITY;
-          xb[it].z = j0 + 2 < nn ? topk_ld1<NC>(row + j0 + 2) : -INFINITY;
-          xb[it].w = j0 + 3 < nn ? topk_ld1<NC>(row + j0 + 3) : -INFINITY;
+          xr[it].x = j0 < nn ? topk_ld1<NC>(row + j0) : -INFINITY;
+          xr[it].y = j0 + 1 < nn ? topk_ld1<NC>(row + j0 + 1) : -INFINITY;
+          xr[it].z = j0 + 2 < nn ? topk_ld1<NC>(row + j0 + 2) : -INFINITY;
+          xr[it].w = j0 + 3 < nn ? topk_ld1<NC>(row + j0 + 3) : -INFINITY;
         }
+      }
+    };
+    float4 xb[kTopkBatch], xn[kTopkBatch];
+    if (PIPE) load_run(0, xn);
+    for (int cb = 0; cb < nn && !overflow; cb += kTopkRun) {
+      if (PIPE) {
+#pragma unroll
+        for (int it = 0; it < kTopkBatch; ++it) xb[it] = xn[it];
+        if (cb + kTopkRun < nn) load_run(cb + kTopkRun, xn);
+      } else {
+        load_run(cb, xb);
       }
       uint32_t fl = 0;                  // bit 4*it + q: score q of step it is kept
       uint32_t cnt_lo = 0, cnt_hi = 0;  // per-step counts packed in bytes
@@ -892,6 +905,28 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkArgs a) {
     return;
   }
   topk_scores_row<true>(a, (int)n, a.scores + i * a.ld, out, dyn, sh);
+  if (tid == 0 && a.cnt) a.cnt[i] = K;
+}
+
+// topk_kernel<kTopkScores> for launches of at most one row per SM (decode): one CTA per SM,
+// so the candidate pass can hold the next run of the row in registers while it compacts the
+// current one.
+__global__ void __launch_bounds__(kTopkThreads, 1) topk_rows_alone_kernel(TopkArgs a) {
+  extern __shared__ uint32_t dyn[];
+  __shared__ TopkShared sh;
+  const int tid = threadIdx.x;
+  const int K = a.K;
+  const int64_t i = a.q_count - 1 - (int64_t)blockIdx.x;
+  const int64_t r = a.q_begin + i;
+  int b;
+  const int64_t n = topk_row_len(a, r, &b);
+  int32_t* out = a.idx + i * a.ld_idx;
+  if (n <= K) {
+    for (int j = tid; j < K; j += kTopkThreads) out[j] = j < n ? j : -1;
+    if (a.cnt && tid == 0) a.cnt[i] = (int32_t)n;
+    return;
+  }
+  topk_scores_row<true, true>(a, (int)n, a.scores + i * a.ld, out, dyn, sh);
   if (tid == 0 && a.cnt) a.cnt[i] = K;
 }
 
