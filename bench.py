@@ -106,7 +106,7 @@ def algorithmic(w):
         # fused path: the selection never sees the score matrix; its floor is reading the
         # K selected (position, score) pairs and writing the index rows
         "topk_bytes_fused": 12 * sel_sum,
-        # what the fused path's selection stage moves: each row's samples (every 16th score),
+        # what the fused path's selection stage moves: each row's bf16 samples (every 16th score),
         # its candidate pairs (about 16 R of them, R = e + 5 sqrt(e) + 16 samples, e = K S / n,
         # or all n when n <= cap) and its index row
         "topk_bytes_fused_moved": fused_moved_bytes(w),
@@ -139,7 +139,7 @@ def fused_moved_bytes(w) -> int:
         R = np.minimum(np.ceil(K * S_ / n + 5.0 * np.sqrt(K * S_ / n) + 16.0), S_)
         cand = np.where(n <= K, 0.0, np.where(n <= cap, n, 16.0 * R))
         samples = np.where(n <= cap, 0.0, S_)
-        total += float((4.0 * samples + 8.0 * cand + 4.0 * K).sum())
+        total += float((2.0 * samples + 8.0 * cand + 4.0 * K).sum())  # bf16 samples
     return int(total)
 
 

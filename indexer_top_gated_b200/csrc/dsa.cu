@@ -149,6 +149,10 @@ dsa_status device_setup(DeviceState** out) {
     e = e ? e : allow_smem(idx_scores_kernel<16, false, kIdxScores>, idx_max);
     e = e ? e : allow_smem(idx_scores_kernel<64, true, kIdxScores>, idx_max);
     e = e ? e : allow_smem(idx_scores_kernel<16, true, kIdxScores>, idx_max);
+    e = e ? e : allow_smem(idx_scores_kernel<64, false, kIdxSamples>, idx_max);
+    e = e ? e : allow_smem(idx_scores_kernel<16, false, kIdxSamples>, idx_max);
+    e = e ? e : allow_smem(idx_scores_kernel<64, true, kIdxSamples>, idx_max);
+    e = e ? e : allow_smem(idx_scores_kernel<16, true, kIdxSamples>, idx_max);
     const size_t cand_max = idx_smem_bytes(4, 64, false, true);
     e = e ? e : allow_smem(idx_scores_kernel<64, false, kIdxCand>, cand_max);
     e = e ? e : allow_smem(idx_scores_kernel<16, false, kIdxCand>, cand_max);
@@ -164,6 +168,7 @@ dsa_status device_setup(DeviceState** out) {
     e = e ? e : allow_smem(topk_fused_kernel, topk_fused_smem_bytes(kTopkFastCap, kTopkFusedMaxN));
     e = e ? e : allow_smem(topk_kernel<kTopkFallback>, topk_smem_bytes(0));
     e = e ? e : allow_smem(topk_rows_alone_kernel, topk_smem_bytes(0));
+    e = e ? e : allow_smem(topk_thr_kernel, topk_thr_smem_bytes(kThrStageMax));
     e = e ? e : allow_smem(sparse_attn_kernel<1, 1, kAddrBytes32>, attn_smem_bytes());
     e = e ? e : allow_smem(sparse_attn_kernel<2, 1, kAddrBytes32>, attn_smem_bytes());
     e = e ? e : allow_smem(sparse_attn_kernel<1, 2, kAddrBytes32>, attn_smem_bytes());
@@ -288,6 +293,7 @@ struct IdxVariant {
   int cap = 0;
   int32_t* cand_cnt = nullptr;
   bool bmax = false;               // 32-key maxima instead of scores (scores = ld-strided rows)
+  bool samples16 = false;          // scores as bf16 rounded down (the sampled pass)
 };
 
 dsa_status launch_index_scores(const DeviceState& dev, const dsa_params* P, const dsa_ragged* R,
@@ -297,7 +303,7 @@ dsa_status launch_index_scores(const DeviceState& dev, const dsa_params* P, cons
   if (q_count == 0 || R->total_kv == 0) return DSA_OK;
   const bool fp8 = P->idx_dtype == DSA_FP8_E4M3;
   const bool cand = var.thr != nullptr;
-  const int mode = cand ? kIdxCand : var.bmax ? kIdxBlockMax : kIdxScores;
+  const int mode = cand ? kIdxCand : var.bmax ? kIdxBlockMax : var.samples16 ? kIdxSamples : kIdxScores;
   CUtensorMap mq, mk;
   if (cand && bq > 16) {
     // query-major candidate pass: 128 query rows per CTA, 128-key tiles, 4 segments per row
@@ -364,7 +370,8 @@ dsa_status launch_index_scores(const DeviceState& dev, const dsa_params* P, cons
   a.cand = var.cand;
   a.cap = var.cap;
   a.cand_cnt = var.cand_cnt;
-  const size_t smem = idx_smem_bytes(P->n_idx_heads, bq, fp8, mode != kIdxScores);
+  const size_t smem =
+      idx_smem_bytes(P->n_idx_heads, bq, fp8, mode == kIdxCand || mode == kIdxBlockMax);
   dim3 grid((unsigned)a.n_tiles, (unsigned)ysplit);
   StageScope scope(0, stream);
 #define DSA_IDX_CASE(BQ, F8, M)                                                      \
@@ -374,6 +381,10 @@ dsa_status launch_index_scores(const DeviceState& dev, const dsa_params* P, cons
   DSA_IDX_CASE(64, true, kIdxScores)
   DSA_IDX_CASE(16, false, kIdxScores)
   DSA_IDX_CASE(16, true, kIdxScores)
+  DSA_IDX_CASE(64, false, kIdxSamples)
+  DSA_IDX_CASE(64, true, kIdxSamples)
+  DSA_IDX_CASE(16, false, kIdxSamples)
+  DSA_IDX_CASE(16, true, kIdxSamples)
   DSA_IDX_CASE(64, false, kIdxCand)
   DSA_IDX_CASE(64, true, kIdxCand)
   DSA_IDX_CASE(16, false, kIdxCand)
@@ -430,7 +441,7 @@ constexpr int kFallbackCtas = 128;
 
 struct FusedGeom {
   int cap;              // candidate slots per row
-  int64_t ld_s;         // floats per sample row
+  int64_t ld_s;         // samples (bf16) per sample row
   int64_t ld_fb;        // floats per fallback scratch row
   int64_t samp_rows;    // rows of the sampled key tensor
   int64_t key_row;      // bytes per key row
@@ -462,7 +473,7 @@ bool fused_geom(const dsa_params* P, const dsa_ragged* R, FusedGeom* g) {
   g->key_row = (int64_t)P->n_idx_heads * 64 * (P->idx_dtype == DSA_FP8_E4M3 ? 1 : 2);
   g->fixed_bytes = round_up(g->samp_rows * g->key_row, 256) +
                    round_up((int64_t)kFallbackCtas * g->ld_fb * 4, 256) + 256 * 5;
-  g->row_bytes = std::max<int64_t>(g->ld_s * 4, cap * 8) + 7 * 4;
+  g->row_bytes = std::max<int64_t>(g->ld_s * 2, cap * 8) + 7 * 4;
   return true;
 }
 
@@ -487,7 +498,7 @@ bool fused_wanted(const dsa_params* P, const dsa_ragged* R, FusedGeom* g) {
 struct FusedWs {
   uint4* k_samp;
   float* fb_scores;
-  char* sc;        // samples [rows, ld_s] floats, later candidates [rows, cap] float2
+  char* sc;        // samples [rows, ld_s] bf16, later candidates [rows, cap] float2
   float* thr;
   uint32_t* khi;   // [rows] largest sample key
   int32_t* ccnt;   // [rows, 4]
@@ -502,7 +513,7 @@ FusedWs fused_carve(const FusedGeom& g, void* ws, int64_t rows) {
   f.fb_scores = reinterpret_cast<float*>(p);
   p += round_up((int64_t)kFallbackCtas * g.ld_fb * 4, 256);
   f.sc = p;
-  p += round_up(rows * std::max<int64_t>(g.ld_s * 4, (int64_t)g.cap * 8), 256);
+  p += round_up(rows * std::max<int64_t>(g.ld_s * 2, (int64_t)g.cap * 8), 256);
   f.thr = reinterpret_cast<float*>(p);
   p += round_up(rows * 4, 256);
   f.khi = reinterpret_cast<uint32_t*>(p);
@@ -531,10 +542,12 @@ dsa_status fused_pass(const DeviceState& dev, const dsa_params* P, const dsa_rag
                       const FusedGeom& g, const FusedWs& f, cudaStream_t stream) {
   if (q_count == 0) return DSA_OK;
   const int bq = R->max_q_len <= 16 ? 16 : 64;
+  // samples: bf16 [rows, ld_s], rounded toward -infinity
   float* samp = reinterpret_cast<float*>(f.sc);
   t_fused_rows += q_count;
   {  // (1) sampled scores
     IdxVariant v;
+    v.samples16 = true;
     v.shift = kSampleShift;
     v.k_rows = f.k_samp;
     v.k_rows_n = g.samp_rows;
@@ -551,14 +564,15 @@ dsa_status fused_pass(const DeviceState& dev, const dsa_params* P, const dsa_rag
     t.K = P->top_k;
     t.cap = g.cap;
     t.shift = kSampleShift;
-    t.samp = samp;
+    t.samp = reinterpret_cast<const uint16_t*>(f.sc);
     t.ld_s = g.ld_s;
+    t.stage = (int)std::min<int64_t>(kThrStageMax, g.ld_s);  // ld_s: a multiple of 32
     t.thr = f.thr;
     t.khi = f.khi;
     t.fb_list = f.list;
     StageScope scope(1, stream);
-    topk_thr_kernel<<<(unsigned)((q_count + kThrWarps - 1) / kThrWarps), 32 * kThrWarps, 0,
-                      stream>>>(t);
+    topk_thr_kernel<<<(unsigned)((q_count + kThrWarps - 1) / kThrWarps), 32 * kThrWarps,
+                      topk_thr_smem_bytes(t.stage), stream>>>(t);
     ++t_launches;
     DSA_TRY(launch_status("topk_thr_kernel"));
   }

@@ -116,7 +116,10 @@ __host__ inline size_t idx_smem_bytes(int n_heads, int bq, bool fp8, bool cand =
 }
 
 // Variants of the epilogue: every score, candidates only, or the maximum of each 32 keys.
-enum IdxMode { kIdxScores = 0, kIdxCand = 1, kIdxBlockMax = 2 };
+// kIdxSamples: as kIdxScores, stored as bf16 rounded toward -infinity (the sampled pass of
+// the fused path: its samples only set a lower bound of a threshold, so rounding them down
+// keeps every bound valid and halves their bytes).
+enum IdxMode { kIdxScores = 0, kIdxCand = 1, kIdxBlockMax = 2, kIdxSamples = 3 };
 
 template <int BQ, bool FP8, int MODE>
 __global__ void __launch_bounds__(kIdxThreads, 1)
@@ -460,20 +463,32 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             __syncwarp();  // the block is read before the next chunk overwrites it
             continue;
           }
-          float* dst = a.scores + (int64_t)(row0 + c0) * a.ld + j;
           const bool interior = inside && (int64_t)kt * kIdxKeyTile + kIdxKeyTile <= a.ld;
-          if (interior) {
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              *dst = acc[c];
-              dst += a.ld;
-            }
-          } else {
+          if (MODE == kIdxSamples) {
+            __nv_bfloat16* dst16 =
+                reinterpret_cast<__nv_bfloat16*>(a.scores) + (int64_t)(row0 + c0) * a.ld + j;
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
               const int cc = c0 + c;
-              if (cc >= c_lo && cc < c_hi && j <= ((p0 + cc) >> a.shift) && j < a.ld) *dst = acc[c];
-              dst += a.ld;
+              if (interior || (cc >= c_lo && cc < c_hi && j <= ((p0 + cc) >> a.shift) && j < a.ld))
+                *dst16 = __float2bfloat16_rd(acc[c]);
+              dst16 += a.ld;
+            }
+          } else {
+            float* dst = a.scores + (int64_t)(row0 + c0) * a.ld + j;
+            if (interior) {
+#pragma unroll
+              for (int c = 0; c < 16; ++c) {
+                *dst = acc[c];
+                dst += a.ld;
+              }
+            } else {
+#pragma unroll
+              for (int c = 0; c < 16; ++c) {
+                const int cc = c0 + c;
+                if (cc >= c_lo && cc < c_hi && j <= ((p0 + cc) >> a.shift) && j < a.ld) *dst = acc[c];
+                dst += a.ld;
+              }
             }
           }
         }

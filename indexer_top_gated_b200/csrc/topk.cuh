@@ -125,8 +125,9 @@ struct TopkThrArgs {
   int K;
   int cap;
   int shift;          // sample m of a row is the score of position m << shift
-  const float* samp;  // [q_count, ld_s]
+  const uint16_t* samp;  // [q_count, ld_s] bf16 samples, rounded toward -infinity
   int64_t ld_s;
+  int stage;          // samples a warp stages in shared memory (a multiple of 8)
   float* thr;         // [q_count]
   uint32_t* khi;      // [q_count] largest sample key (0: the row was not sampled)
   int32_t* fb_list;   // its count is reset here
@@ -1052,17 +1053,33 @@ __global__ void __launch_bounds__(256) block_expand_kernel(BlockArgs a) {
   }
 }
 
-// One warp per row: a lower bound of the R-th largest of the row's S samples, R = S K / n
-// plus a margin of 5 sigma + 16, so that at least K scores of the row are >= it with
-// overwhelming probability while about R n / S are.  The sample keys are mapped onto the
-// full 32-bit range ((key - kmin) << clz(kmax - kmin), order-preserving), and two 8-bit
-// radix levels give the top 16 bits of the R-th largest; the estimate rounds it down.
-// Rows with n <= K need no candidates (+inf); rows with n <= cap keep every score (-inf).
+// One warp per row: the R-th largest of the row's S samples, R = S K / n plus a margin of
+// 5 sigma + 16, so that at least K scores of the row are >= it with overwhelming probability
+// while about R n / S are.  The samples are bf16 rounded toward -infinity (each is at most its
+// score), so the R-th largest of them is a lower bound of the exact one and the estimate stays
+// on the safe side.  They become 16-bit order-preserving keys (-0.0 folded onto +0.0), mapped
+// onto the full 16-bit range ((key - kmin) << clz16(kmax - kmin)), and two 8-bit radix levels
+// find the R-th largest exactly.  Rows with n <= K need no candidates (+inf); rows with
+// n <= cap keep every score (-inf).  The largest sample's key (as a 32-bit score key) is kept
+// for the selection's key range.  A warp stages up to a.stage samples in shared memory; longer
+// rows are read from global memory in each pass.
 constexpr int kThrWarps = 4;
-constexpr int kThrStage = 2048;  // samples a warp stages in shared memory as keys
+constexpr int kThrStageMax = 2048;  // samples a warp stages at most (4 KiB)
+__host__ inline size_t topk_thr_smem_bytes(int stage) {
+  return (size_t)kThrWarps * stage * 2;
+}
+DSA_DEV uint32_t thr_key16(uint32_t b) {
+  b &= 0xFFFFu;
+  if (b == 0x8000u) b = 0u;  // -0.0 == +0.0
+  return (b & 0x8000u) ? (~b & 0xFFFFu) : (b | 0x8000u);
+}
+DSA_DEV float thr_key16_value(uint32_t k) {
+  const uint32_t b = (k & 0x8000u) ? (k ^ 0x8000u) : (~k & 0xFFFFu);
+  return __uint_as_float(b << 16);
+}
 __global__ void __launch_bounds__(32 * kThrWarps) topk_thr_kernel(TopkThrArgs a) {
   __shared__ uint32_t hist[kThrWarps][256];
-  __shared__ __align__(16) uint32_t stage[kThrWarps][kThrStage];
+  extern __shared__ __align__(16) uint16_t thr_stage[];  // [kThrWarps][a.stage]
   const int warp = threadIdx.x >> 5, lane = lane_id();
   if (blockIdx.x == 0 && threadIdx.x == 0) a.fb_list[0] = 0;
   const int64_t i = (int64_t)blockIdx.x * kThrWarps + warp;
@@ -1087,63 +1104,82 @@ __global__ void __launch_bounds__(32 * kThrWarps) topk_thr_kernel(TopkThrArgs a)
   uint32_t* h = hist[warp];
 #pragma unroll
   for (int q = 0; q < 8; ++q) h[lane * 8 + q] = 0;
-  const float* row = a.samp + i * a.ld_s;
-  // short sample rows (the usual case) are staged once as keys; longer ones are read
-  // from global memory on every pass, several loads in flight per lane
-  const bool staged = S <= kThrStage;
-  uint32_t* st = stage[warp];
-  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  const uint16_t* row = a.samp + i * a.ld_s;
+  const bool staged = S <= a.stage;
+  uint16_t* st = thr_stage + (size_t)warp * a.stage;
+  uint32_t lo = 0xFFFFu, hi = 0u;
+  // every key of the row, f(key), from the staged keys or from global memory (8 samples per
+  // 16-byte load, several loads in flight per lane)
   auto for_keys = [&](auto&& f) {
     if (staged) {
-      for (int m = lane; m < S; m += 32) f(st[m], true);
+      for (int m = lane; m < S; m += 32) f((uint32_t)st[m]);
     } else {
-      for (int m0 = 0; m0 < S; m0 += 8 * 32) {
-        float x[8];
+      for (int m0 = 0; m0 < S; m0 += 4 * 32 * 8) {
+        uint4 u[4];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int m = m0 + u * 32 + lane;
-          x[u] = m < S ? __ldg(row + m) : 0.f;
+        for (int v = 0; v < 4; ++v) {
+          const int m = m0 + (v * 32 + lane) * 8;
+          u[v] = m < S ? __ldg(reinterpret_cast<const uint4*>(row + m)) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
-        for (int u = 0; u < 8; ++u) f(topk_key(x[u]), m0 + u * 32 + lane < S);
+        for (int v = 0; v < 4; ++v) {
+          const int m = m0 + (v * 32 + lane) * 8;
+          const uint32_t w4[4] = {u[v].x, u[v].y, u[v].z, u[v].w};
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            if (m + q < S) f(thr_key16(w4[q >> 1] >> (16 * (q & 1))));
+        }
       }
     }
   };
   if (staged) {
-    const int S4 = (S + 3) & ~3;  // rows are 16-byte aligned and padded to ld_s >= S4
-    for (int m0 = 0; m0 < S4; m0 += 4 * 32 * 4) {
-      float4 f[4];
+    // stage the keys and take their range on the way (rows are 16-byte aligned and padded to
+    // ld_s >= a multiple of 8 >= S)
+    const int S8 = (S + 7) & ~7;
+    for (int m0 = 0; m0 < S8; m0 += 4 * 32 * 8) {
+      uint4 u[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int m = m0 + (u * 32 + lane) * 4;
-        f[u] = m < S4 ? __ldg(reinterpret_cast<const float4*>(row + m)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int v = 0; v < 4; ++v) {
+        const int m = m0 + (v * 32 + lane) * 8;
+        u[v] = m < S8 ? __ldg(reinterpret_cast<const uint4*>(row + m)) : make_uint4(0u, 0u, 0u, 0u);
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int m = m0 + (u * 32 + lane) * 4;
-        if (m < S4)
+      for (int v = 0; v < 4; ++v) {
+        const int m = m0 + (v * 32 + lane) * 8;
+        if (m < S8) {
+          const uint32_t w4[4] = {u[v].x, u[v].y, u[v].z, u[v].w};
+          uint32_t k[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            k[q] = thr_key16(w4[q >> 1] >> (16 * (q & 1)));
+            if (m + q < S) {
+              lo = k[q] < lo ? k[q] : lo;
+              hi = k[q] > hi ? k[q] : hi;
+            }
+          }
           *reinterpret_cast<uint4*>(st + m) =
-              make_uint4(topk_key(f[u].x), topk_key(f[u].y), topk_key(f[u].z), topk_key(f[u].w));
+              make_uint4(k[0] | (k[1] << 16), k[2] | (k[3] << 16), k[4] | (k[5] << 16),
+                         k[6] | (k[7] << 16));
+        }
       }
     }
     __syncwarp();
-  }
-  for_keys([&](uint32_t k, bool ok) {
-    if (ok) {
+  } else {
+    for_keys([&](uint32_t k) {
       lo = k < lo ? k : lo;
       hi = k > hi ? k : hi;
-    }
-  });
+    });
+  }
   lo = __reduce_min_sync(0xFFFFFFFFu, lo);
   hi = __reduce_max_sync(0xFFFFFFFFu, hi);
-  const int z = hi != lo ? __clz(hi - lo) : 0;
+  const int z = hi != lo ? __clz(hi - lo) - 16 : 0;  // normalised keys fill 16 bits
   __syncwarp();
   uint32_t prefix = 0, mask = 0, remaining = (uint32_t)R;
   for (int level = 0; level < 2; ++level) {
-    const int sh = 24 - 8 * level;
-    for_keys([&](uint32_t k, bool ok) {
-      const uint32_t nk = (k - lo) << z;
-      if (ok && (nk & mask) == prefix) atomicAdd(&h[(nk >> sh) & 255u], 1u);
+    const int sh = 8 - 8 * level;
+    for_keys([&](uint32_t k) {
+      const uint32_t nk = ((k - lo) << z) & 0xFFFFu;
+      if ((nk & mask) == prefix) atomicAdd(&h[(nk >> sh) & 255u], 1u);
     });
     __syncwarp();
     // lane l owns bins 255 - 8l - q, q = 0..7 (from the top)
@@ -1179,8 +1215,8 @@ __global__ void __launch_bounds__(32 * kThrWarps) topk_thr_kernel(TopkThrArgs a)
     __syncwarp();
   }
   if (lane == 0) {
-    a.thr[i] = topk_key_value(lo + (prefix >> z));
-    a.khi[i] = hi;
+    a.thr[i] = thr_key16_value(lo + (prefix >> z));
+    a.khi[i] = topk_key(thr_key16_value(hi));
   }
 }
 
