@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(kCandThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue (warps 2-17)
     const int quad = warp & 3;          // TMEM lanes 32 quad .. 32 quad + 31
-    const int sub = (warp - 2) >> 2;    // key columns 16 sub .. 16 sub + 15 of each tile
+    const int sub = (warp - 2) >> 2;    // key columns 32 sub .. 32 sub + 31 of each tile
     const int rr = quad * 32 + lane;    // this thread's row within the tile
     const int64_t row = r0 + rr;
     const bool in_launch = row <= r_last;
