@@ -131,11 +131,27 @@ __global__ void __launch_bounds__(AttnGeom<HKV_CTA>::kThreads, AttnShape<HKV_CTA
   __syncthreads();
   {
     int last = -1, err = 0;
-    for (int e = tid; e < K; e += kAttnThreads) {
-      const int j = __ldg(irow + e);
-      if (j >= 0) {
-        if ((int64_t)j <= p) last = e;
-        else ++err;
+    if ((K & 3) == 0 && (reinterpret_cast<uintptr_t>(irow) & 15) == 0) {
+      // four entries per 16-byte load, all of a thread's loads in flight
+      const int4* i4 = reinterpret_cast<const int4*>(irow);
+      for (int e4 = tid; e4 < (K >> 2); e4 += kAttnThreads) {
+        const int4 v = __ldg(i4 + e4);
+        const int jj[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (jj[q] >= 0) {
+            if ((int64_t)jj[q] <= p) last = 4 * e4 + q;
+            else ++err;
+          }
+        }
+      }
+    } else {
+      for (int e = tid; e < K; e += kAttnThreads) {
+        const int j = __ldg(irow + e);
+        if (j >= 0) {
+          if ((int64_t)j <= p) last = e;
+          else ++err;
+        }
       }
     }
     if (last >= 0) atomicMax(&s_last, last);
