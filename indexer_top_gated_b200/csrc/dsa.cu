@@ -567,14 +567,25 @@ dsa_status fused_pass(const DeviceState& dev, const dsa_params* P, const dsa_rag
     t.samp = reinterpret_cast<const uint16_t*>(f.sc);
     t.ld_s = g.ld_s;
     t.stage = (int)std::min<int64_t>(kThrStageMax, g.ld_s);  // ld_s: a multiple of 32
+    // rows of more than t.stage samples (possible when ld_s exceeds it) take a CTA each
+    t.long_rows = g.ld_s > t.stage ? 1 : 0;
     t.thr = f.thr;
     t.khi = f.khi;
     t.fb_list = f.list;
-    StageScope scope(1, stream);
-    topk_thr_kernel<<<(unsigned)((q_count + kThrWarps - 1) / kThrWarps), 32 * kThrWarps,
-                      topk_thr_smem_bytes(t.stage), stream>>>(t);
-    ++t_launches;
-    DSA_TRY(launch_status("topk_thr_kernel"));
+    {
+      StageScope scope(1, stream);
+      topk_thr_kernel<<<(unsigned)((q_count + kThrWarps - 1) / kThrWarps), 32 * kThrWarps,
+                        topk_thr_smem_bytes(t.stage), stream>>>(t);
+      ++t_launches;
+      DSA_TRY(launch_status("topk_thr_kernel"));
+    }
+    if (t.long_rows) {
+      StageScope scope(1, stream);
+      topk_thr_long_kernel<<<(unsigned)q_count, kThrLongThreads,
+                             topk_thr_long_smem_bytes((int)g.ld_s), stream>>>(t, (int)g.ld_s);
+      ++t_launches;
+      DSA_TRY(launch_status("topk_thr_long_kernel"));
+    }
   }
   {  // (3) candidates
     IdxVariant v;

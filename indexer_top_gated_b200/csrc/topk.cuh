@@ -128,6 +128,8 @@ struct TopkThrArgs {
   const uint16_t* samp;  // [q_count, ld_s] bf16 samples, rounded toward -infinity
   int64_t ld_s;
   int stage;          // samples a warp stages in shared memory (a multiple of 8)
+  int long_rows;      // non-zero: rows of more than `stage` samples are left to
+                      // topk_thr_long_kernel
   float* thr;         // [q_count]
   uint32_t* khi;      // [q_count] largest sample key (0: the row was not sampled)
   int32_t* fb_list;   // its count is reset here
@@ -1098,6 +1100,7 @@ __global__ void __launch_bounds__(32 * kThrWarps) topk_thr_kernel(TopkThrArgs a)
     return;
   }
   const int S = (int)(p >> a.shift) + 1;
+  if (a.long_rows && S > a.stage) return;  // a CTA of topk_thr_long_kernel takes the row
   const float e = (float)a.K * (float)S / (float)n;
   int R = (int)ceilf(e + 5.f * sqrtf(e) + 16.f);
   if (R > S) R = S;
@@ -1215,6 +1218,125 @@ __global__ void __launch_bounds__(32 * kThrWarps) topk_thr_kernel(TopkThrArgs a)
     __syncwarp();
   }
   if (lane == 0) {
+    a.thr[i] = thr_key16_value(lo + (prefix >> z));
+    a.khi[i] = topk_key(thr_key16_value(hi));
+  }
+}
+
+// topk_thr_kernel's selection for rows of more than a.stage samples, one CTA of
+// kThrLongThreads per row: the row's bf16 samples are read once, with many loads in flight, and
+// staged as 16-bit keys in shared memory (long_stage >= every row's sample count: the launch
+// passes ld_s), and the CTA's warps build the two 8-bit radix histograms together; one warp
+// picks each level's bin.  The result is the one topk_thr_kernel would give for the row.
+// Other rows return at once.
+constexpr int kThrLongThreads = 256;
+__host__ inline size_t topk_thr_long_smem_bytes(int long_stage) { return (size_t)long_stage * 2; }
+__global__ void __launch_bounds__(kThrLongThreads) topk_thr_long_kernel(TopkThrArgs a, int long_stage) {
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t s_lo, s_hi, s_sel[2];
+  extern __shared__ __align__(16) uint16_t thr_long_stage[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = lane_id();
+  const int64_t i = blockIdx.x;
+  const int64_t r = a.q_begin + i;
+  const int b = seq_of_row(a.q_offsets, a.batch, r);
+  const int64_t qo = __ldg(a.q_offsets + b), qn = __ldg(a.q_offsets + b + 1);
+  const int64_t L = (int64_t)__ldg(a.kv_offsets + b + 1) - __ldg(a.kv_offsets + b);
+  const int64_t p = L - (qn - qo) + (r - qo);
+  const int64_t n = p + 1;
+  if (n <= a.K || n <= a.cap) return;  // topk_thr_kernel writes these rows
+  const int S = (int)(p >> a.shift) + 1;
+  if (S <= a.stage || S > long_stage) return;  // uniform (S > long_stage never happens)
+  const float e = (float)a.K * (float)S / (float)n;
+  int R = (int)ceilf(e + 5.f * sqrtf(e) + 16.f);
+  if (R > S) R = S;
+  const uint16_t* row = a.samp + i * a.ld_s;
+  uint16_t* st = thr_long_stage;
+  for (int t = tid; t < 256; t += kThrLongThreads) hist[t] = 0;
+  if (tid == 0) {
+    s_lo = 0xFFFFu;
+    s_hi = 0u;
+  }
+  __syncthreads();
+  // stage the keys (8 per 16-byte load, every thread's loads in flight) and their range
+  uint32_t lo = 0xFFFFu, hi = 0u;
+  const int S8 = (S + 7) & ~7;  // rows are 16-byte aligned and padded to ld_s >= S8
+  constexpr int kLd = 4;
+  for (int m0 = 0; m0 < S8; m0 += kLd * kThrLongThreads * 8) {
+    uint4 u[kLd];
+#pragma unroll
+    for (int v = 0; v < kLd; ++v) {
+      const int m = m0 + (v * kThrLongThreads + tid) * 8;
+      u[v] = m < S8 ? __ldg(reinterpret_cast<const uint4*>(row + m)) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int v = 0; v < kLd; ++v) {
+      const int m = m0 + (v * kThrLongThreads + tid) * 8;
+      if (m < S8) {
+        const uint32_t w4[4] = {u[v].x, u[v].y, u[v].z, u[v].w};
+        uint32_t k[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          k[q] = thr_key16(w4[q >> 1] >> (16 * (q & 1)));
+          if (m + q < S) {
+            lo = k[q] < lo ? k[q] : lo;
+            hi = k[q] > hi ? k[q] : hi;
+          }
+        }
+        *reinterpret_cast<uint4*>(st + m) =
+            make_uint4(k[0] | (k[1] << 16), k[2] | (k[3] << 16), k[4] | (k[5] << 16),
+                       k[6] | (k[7] << 16));
+      }
+    }
+  }
+  lo = __reduce_min_sync(0xFFFFFFFFu, lo);
+  hi = __reduce_max_sync(0xFFFFFFFFu, hi);
+  if (lane == 0) {
+    atomicMin(&s_lo, lo);
+    atomicMax(&s_hi, hi);
+  }
+  __syncthreads();  // keys staged, range known
+  lo = s_lo;
+  hi = s_hi;
+  const int z = hi != lo ? __clz(hi - lo) - 16 : 0;  // normalised keys fill 16 bits
+  uint32_t prefix = 0, mask = 0, remaining = (uint32_t)R;
+  for (int level = 0; level < 2; ++level) {
+    const int sh = 8 - 8 * level;
+    for (int m = tid; m < S; m += kThrLongThreads) {
+      const uint32_t nk = (((uint32_t)st[m] - lo) << z) & 0xFFFFu;
+      if ((nk & mask) == prefix) atomicAdd(&hist[(nk >> sh) & 255u], 1u);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // lane l owns bins 255 - 8l - q, q = 0..7 (from the top)
+      uint32_t c[8], sum = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        c[q] = hist[255 - 8 * lane - q];
+        sum += c[q];
+      }
+      const uint32_t incl = warp_incl_scan(sum);
+      const unsigned own = __ballot_sync(0xFFFFFFFFu, incl - sum < remaining && remaining <= incl);
+      const int o = __ffs(own) - 1;
+      if (lane == o) {
+        uint32_t above = incl - sum;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (above < remaining && remaining <= above + c[q]) {
+            s_sel[0] = 255u - 8u * (uint32_t)lane - (uint32_t)q;
+            s_sel[1] = remaining - above;
+          }
+          above += c[q];
+        }
+      }
+    }
+    __syncthreads();  // bin picked, histogram read
+    prefix |= s_sel[0] << sh;
+    mask |= 255u << sh;
+    remaining = s_sel[1];
+    for (int t = tid; t < 256; t += kThrLongThreads) hist[t] = 0;
+    __syncthreads();  // histogram zeroed, s_sel read
+  }
+  if (tid == 0) {
     a.thr[i] = thr_key16_value(lo + (prefix >> z));
     a.khi[i] = topk_key(thr_key16_value(hi));
   }

@@ -4,7 +4,7 @@ On dyadic-grid inputs every score is exact in fp32, so the fused path must give,
 bit, the index rows of dsa_index_scores + dsa_topk (which are pinned to the oracle in
 test_gpu_parity.py); sampled rows are also checked against the oracle directly.  The
 cases cover rows shorter than the candidate slots (every score kept), long rows (sampled
-threshold), ragged batches with history, e4m3 inputs, per-row weights, K = 1 and a K
+threshold; beyond 2048 samples a CTA per row), ragged batches with history, e4m3 inputs, per-row weights, K = 1 and a K
 near the slot limit, rows whose threshold misses (all scores tied: the CUDA-core
 fallback), passes forced by a small workspace, and the layer taking the fused path.
 """
@@ -96,6 +96,9 @@ FUSED_CASES = {
     "k1": dict(q_lens=[1500], kv_lens=[1500], K=1),
     "k4096": dict(q_lens=[600], kv_lens=[20000], K=4096),
     "one_head": dict(q_lens=[2000], kv_lens=[5000], Hi=1, K=200),
+    # rows of more than 2048 samples (n > 32768): their thresholds come from the one-CTA-per-row
+    # kernel
+    "long_rows": dict(q_lens=[96], kv_lens=[40000], K=512),
 }
 
 
