@@ -294,6 +294,8 @@ struct IdxVariant {
   int32_t* cand_cnt = nullptr;
   bool bmax = false;               // 32-key maxima instead of scores (scores = ld-strided rows)
   bool samples16 = false;          // scores as bf16 rounded down (the sampled pass)
+  int32_t* tile_order = nullptr;   // candidate pass: room for ceil(rows / 128) query tiles,
+                                   // ordered longest first when the batch has several sequences
 };
 
 dsa_status launch_index_scores(const DeviceState& dev, const dsa_params* P, const dsa_ragged* R,
@@ -327,6 +329,14 @@ dsa_status launch_index_scores(const DeviceState& dev, const dsa_params* P, cons
     a.cand = var.cand;
     a.cap = var.cap;
     a.cand_cnt = var.cand_cnt;
+    a.tile_order = nullptr;
+    if (var.tile_order && R->batch > 1 && a.n_tiles > 1 && a.n_tiles <= kCandOrderMax) {
+      StageScope scope(0, stream);
+      idx_cand_order_kernel<<<1, kCandOrderThreads, 0, stream>>>(a, var.tile_order);
+      ++t_launches;
+      DSA_TRY(launch_status("idx_cand_order_kernel"));
+      a.tile_order = var.tile_order;
+    }
     StageScope scope(0, stream);
     if (fp8)
       idx_cand_kernel<true><<<a.n_tiles, kCandThreads, idx_cand_smem_bytes(true), stream>>>(mq, mk, a);
@@ -472,8 +482,10 @@ bool fused_geom(const dsa_params* P, const dsa_ragged* R, FusedGeom* g) {
   g->samp_rows = (logical >> kSampleShift) + R->batch + 1;
   g->key_row = (int64_t)P->n_idx_heads * 64 * (P->idx_dtype == DSA_FP8_E4M3 ? 1 : 2);
   g->fixed_bytes = round_up(g->samp_rows * g->key_row, 256) +
-                   round_up((int64_t)kFallbackCtas * g->ld_fb * 4, 256) + 256 * 5;
-  g->row_bytes = std::max<int64_t>(g->ld_s * 2, cap * 8) + 7 * 4;
+                   round_up((int64_t)kFallbackCtas * g->ld_fb * 4, 256) + 256 * 6;
+  // per row: samples / candidates (shared), threshold, largest sample key, 4 counts, a list
+  // entry, and a byte for the tile order (4 bytes per 128 rows, one more tile at most)
+  g->row_bytes = std::max<int64_t>(g->ld_s * 2, cap * 8) + 7 * 4 + 1;
   return true;
 }
 
@@ -503,6 +515,7 @@ struct FusedWs {
   uint32_t* khi;   // [rows] largest sample key
   int32_t* ccnt;   // [rows, 4]
   int32_t* list;   // [1 + rows]
+  int32_t* order;  // [ceil(rows / 128)] candidate-pass tile order
 };
 
 FusedWs fused_carve(const FusedGeom& g, void* ws, int64_t rows) {
@@ -521,6 +534,8 @@ FusedWs fused_carve(const FusedGeom& g, void* ws, int64_t rows) {
   f.ccnt = reinterpret_cast<int32_t*>(p);
   p += round_up(rows * 16, 256);
   f.list = reinterpret_cast<int32_t*>(p);
+  p += round_up((1 + rows) * 4, 256);
+  f.order = reinterpret_cast<int32_t*>(p);
   return f;
 }
 
@@ -593,6 +608,7 @@ dsa_status fused_pass(const DeviceState& dev, const dsa_params* P, const dsa_rag
     v.cand = reinterpret_cast<float2*>(f.sc);
     v.cap = g.cap;
     v.cand_cnt = f.ccnt;
+    v.tile_order = f.order;
     DSA_TRY(launch_index_scores(dev, P, R, q_idx, k_idx, w, q_begin, q_count, nullptr, 0, bq,
                                 stream, v));
   }

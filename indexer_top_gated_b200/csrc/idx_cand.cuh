@@ -92,7 +92,9 @@ __global__ void __launch_bounds__(kCandThreads, 1)
   const int n_pairs = (H + 1) >> 1;  // head pairs (the last may hold one head)
   const int warp = threadIdx.x >> 5;
   const int lane = lane_id();
-  const int tile = a.n_tiles - 1 - (int)blockIdx.x;  // largest first
+  // longest first: for one sequence the last tiles; for a batch the order idx_cand_order_kernel
+  // found
+  const int tile = a.tile_order ? __ldg(a.tile_order + blockIdx.x) : a.n_tiles - 1 - (int)blockIdx.x;
   const int64_t r0 = a.q_begin + (int64_t)tile * kCandBQ;
   const int64_t q_end = a.q_begin + a.q_count;
   const int64_t r_last = (r0 + kCandBQ < q_end ? r0 + kCandBQ : q_end) - 1;
@@ -424,6 +426,60 @@ __global__ void __launch_bounds__(kCandThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, (uint32_t)kCols);
   }
+}
+
+// Launch order of the candidate pass for a batch of several sequences: the query tiles sorted
+// by their number of key tiles (the CTA's work), longest first, ties by tile index, so that the
+// CTAs of the longest histories start first and the shorter ones fill in (list scheduling in
+// decreasing order).  One CTA of kCandOrderThreads; n_tiles <= kCandOrderMax (else the launch
+// keeps the default order).  Bitonic sort of (work, tile) keys in shared memory.
+constexpr int kCandOrderThreads = 1024;
+constexpr int kCandOrderMax = 4096;
+__global__ void __launch_bounds__(kCandOrderThreads) idx_cand_order_kernel(IdxArgs a, int32_t* order) {
+  __shared__ uint64_t key[kCandOrderMax];
+  const int n = a.n_tiles;
+  int m = 1;
+  while (m < n) m <<= 1;
+  const int64_t q_end = a.q_begin + a.q_count;
+  for (int t = threadIdx.x; t < m; t += kCandOrderThreads) {
+    uint64_t k = ~0ull;  // padding sorts last
+    if (t < n) {
+      const int64_t r0 = a.q_begin + (int64_t)t * kCandBQ;
+      const int64_t r_last = (r0 + kCandBQ < q_end ? r0 + kCandBQ : q_end) - 1;
+      const int b_first = seq_of_row(a.q_offsets, a.batch, r0);
+      const int b_last = seq_of_row(a.q_offsets, a.batch, r_last);
+      uint32_t work = 0;
+      for (int b = b_first; b <= b_last; ++b) {
+        const int64_t qo = __ldg(a.q_offsets + b), qn = __ldg(a.q_offsets + b + 1);
+        const int64_t ko = __ldg(a.kv_offsets + b), kn = __ldg(a.kv_offsets + b + 1);
+        const int64_t rs = r0 > qo ? r0 : qo;
+        const int64_t re = (r_last + 1) < qn ? (r_last + 1) : qn;
+        const int64_t pmax = (kn - ko) - (qn - qo) - qo + re - 1;
+        if (rs < re && pmax >= 0) work += (uint32_t)(pmax / kCandKT) + 1;
+      }
+      // descending work, then ascending tile: sort ascending on (~work, tile)
+      k = ((uint64_t)(~work) << 32) | (uint32_t)t;
+    }
+    key[t] = k;
+  }
+  __syncthreads();
+  for (int size = 2; size <= m; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int t = threadIdx.x; t < m; t += kCandOrderThreads) {
+        const int u = t ^ stride;
+        if (u > t) {
+          const bool up = (t & size) == 0;
+          const uint64_t x = key[t], y = key[u];
+          if ((x > y) == up) {
+            key[t] = y;
+            key[u] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int t = threadIdx.x; t < n; t += kCandOrderThreads) order[t] = (int32_t)(key[t] & 0xFFFFFFFFu);
 }
 
 }  // namespace dsa

@@ -65,6 +65,7 @@ struct IdxArgs {
   int cap;             // a multiple of 4
   int32_t* cand_cnt;   // [q_count, 4] candidates found per segment (may exceed cap/4)
   CachePages pages;    // paged k_idx (not with sampled keys, which are always contiguous)
+  const int32_t* tile_order;  // candidate pass: query tile of each CTA (longest first), or null
 };
 
 // first key-tensor row of sequence b
