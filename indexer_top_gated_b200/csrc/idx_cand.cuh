@@ -269,33 +269,41 @@ __global__ void __launch_bounds__(kCandThreads, 1)
 
     // write every complete group of 4 pending pairs (whole 32-byte sectors) and move the
     // rest (< 4) to the front of the staging area.  At most 3 + 8 pairs are pending, so at
-    // most two groups; the work is predicated per lane under one warp-uniform branch (some
-    // lane of the warp almost always has a group to write).
+    // most two groups.  Only the lanes with a group to write read their staging area (a
+    // lane's hits fill a group every few calls), so the shared-memory loads scale with the
+    // sectors written rather than with the calls.
     auto flush = [&]() {
       const uint32_t groups = pend >> 2;
       if (!__any_sync(0xFFFFFFFFu, groups > 0)) return;
-      const float4 x0 = *reinterpret_cast<const float4*>(stg);
-      const float4 x1 = *reinterpret_cast<const float4*>(stg + 16);
-      const float4 y0 = *reinterpret_cast<const float4*>(stg + 32);
-      const float4 y1 = *reinterpret_cast<const float4*>(stg + 48);
-      const float2 r0 = *reinterpret_cast<const float2*>(stg + (groups * 4 + 0) * 8);
-      const float2 r1 = *reinterpret_cast<const float2*>(stg + (groups * 4 + 1) * 8);
-      const float2 r2 = *reinterpret_cast<const float2*>(stg + (groups * 4 + 2) * 8);
-      float4* d4 = reinterpret_cast<float4*>(dst + written);
-      if (groups > 0 && written + 4 <= (uint32_t)seg) {
-        d4[0] = x0;
-        d4[1] = x1;
+      if (groups > 0) {
+        float4* d4 = reinterpret_cast<float4*>(dst + written);
+        const float4 x0 = *reinterpret_cast<const float4*>(stg);
+        const float4 x1 = *reinterpret_cast<const float4*>(stg + 16);
+        if (written + 4 <= (uint32_t)seg) {
+          d4[0] = x0;
+          d4[1] = x1;
+        }
+        if (groups > 1) {
+          const float4 y0 = *reinterpret_cast<const float4*>(stg + 32);
+          const float4 y1 = *reinterpret_cast<const float4*>(stg + 48);
+          if (written + 8 <= (uint32_t)seg) {
+            d4[2] = y0;
+            d4[3] = y1;
+          }
+        }
+        const uint32_t rest = pend & 3u;
+        const uint8_t* src = stg + groups * 32;
+        if (rest > 0) {
+          const float2 r0 = *reinterpret_cast<const float2*>(src);
+          const float2 r1 = *reinterpret_cast<const float2*>(src + 8);
+          const float2 r2 = *reinterpret_cast<const float2*>(src + 16);
+          *reinterpret_cast<float2*>(stg) = r0;
+          if (rest > 1) *reinterpret_cast<float2*>(stg + 8) = r1;
+          if (rest > 2) *reinterpret_cast<float2*>(stg + 16) = r2;
+        }
+        written += groups * 4;
+        pend = rest;
       }
-      if (groups > 1 && written + 8 <= (uint32_t)seg) {
-        d4[2] = y0;
-        d4[3] = y1;
-      }
-      const uint32_t rest = pend & 3u;
-      if (groups > 0 && rest > 0) *reinterpret_cast<float2*>(stg) = r0;
-      if (groups > 0 && rest > 1) *reinterpret_cast<float2*>(stg + 8) = r1;
-      if (groups > 0 && rest > 2) *reinterpret_cast<float2*>(stg + 16) = r2;
-      written += groups * 4;
-      pend = rest;
     };
 
     int i = 0;
