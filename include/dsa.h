@@ -331,7 +331,10 @@ typedef struct {
  * When the workspace also holds the index rows of every row (K int32 each) next to one pass
  * of steps 1-2 over all rows (the dsa_workspace_size recommendation does for a prefill whose
  * steps 1-2 run fused), steps 1-2 run once as soon as q_idx and k_idx have landed, and only
- * the attention runs per range (in row order); otherwise the whole layer runs per range.
+ * the attention runs per range (in row order; the last of the n_chunks ranges is then cut in
+ * halves of halves, at most three times and not below 256 rows, since its attention and
+ * read-back are what remains after the last upload); otherwise the whole layer runs per
+ * range.
  *   host  every input and the output in host memory (page-locked memory lets the copies
  *         run asynchronously and overlap); host->q_offsets / kv_offsets are also read by
  *         the host to plan the ranges.

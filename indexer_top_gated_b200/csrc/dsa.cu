@@ -1264,12 +1264,7 @@ dsa_status dsa_prefill_from_host(const dsa_params* P, const dsa_ragged* R,
   n_chunks = (int32_t)std::max<int64_t>(1, std::min<int64_t>(n_chunks, std::max<int64_t>(TQ, 1)));
   DeviceState* d = nullptr;
   DSA_TRY(device_setup(&d));
-  DSA_TRY(copy_streams(d, 2 * n_chunks + 3));
-  // the copy streams and events are shared by the device's calls: one enqueue at a time
-  // (a later call's records do not disturb the waits an earlier call already enqueued)
-  std::lock_guard<std::mutex> enqueue_lock(d->enqueue_mu);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaEvent_t ev_start = d->events[0], ev_end = d->events[1];
   const size_t e_idx = P->idx_dtype == DSA_FP8_E4M3 ? 1 : 2;
   const size_t idx_row = (size_t)P->n_idx_heads * P->idx_dim * e_idx;
   const size_t q_row = (size_t)P->n_q_heads * P->head_dim * 2;
@@ -1278,14 +1273,6 @@ dsa_status dsa_prefill_from_host(const dsa_params* P, const dsa_ragged* R,
   auto at = [](const void* base, size_t off) {
     return const_cast<char*>(static_cast<const char*>(base)) + off;
   };
-  // the device buffers may still be in use by earlier work on the caller's stream
-  if (cudaEventRecord(ev_start, st) != cudaSuccess ||
-      cudaStreamWaitEvent(d->s_in, ev_start, 0) != cudaSuccess ||
-      cudaStreamWaitEvent(d->s_out, ev_start, 0) != cudaSuccess)
-    return DSA_ERR_CUDA;
-  DSA_TRY(h2d(at(dev->q_offsets, 0), qo, (size_t)(B + 1) * 4, d->s_in));
-  DSA_TRY(h2d(at(dev->kv_offsets, 0), ko, (size_t)(B + 1) * 4, d->s_in));
-  DSA_TRY(h2d(at(dev->w, 0), host->w, w_bytes, d->s_in));
   // cache rows the queries of rows [a0, a1) see: for every sequence the range touches, up
   // to its last query's position (sequences are packed in order, so this grows with a1)
   auto kv_need_of = [&](int64_t a0, int64_t a1) {
@@ -1310,6 +1297,29 @@ dsa_status dsa_prefill_from_host(const dsa_params* P, const dsa_ragged* R,
   const bool split = (int64_t)ws_bytes > idx_bytes &&
                      (fused ? fused_rows(fg, (int64_t)ws_bytes - idx_bytes) >= TQ
                             : ((int64_t)ws_bytes - idx_bytes) / (scores_ld(R) * 4) >= 1);
+  // Row ranges.  When only the attention runs per range, what follows the last upload is
+  // that range's attention and output read-back: the last range is cut into halves of
+  // halves (at most three cuts, none below 256 rows) so that this tail stays short.
+  std::vector<int64_t> cut;
+  for (int c = 0; c < n_chunks; ++c) cut.push_back(TQ * c / n_chunks);
+  if (split)
+    for (int s = 0; s < 3 && TQ - cut.back() >= 512; ++s)
+      cut.push_back(cut.back() + (TQ - cut.back()) / 2);
+  cut.push_back(TQ);
+  const int n_ranges = (int)cut.size() - 1;
+  // the copy streams and events are shared by the device's calls: one enqueue at a time
+  // (a later call's records do not disturb the waits an earlier call already enqueued).
+  // The event list grows under the same lock, so no call reads it while it is reallocated.
+  std::lock_guard<std::mutex> enqueue_lock(d->enqueue_mu);
+  DSA_TRY(copy_streams(d, 2 * n_ranges + 3));
+  cudaEvent_t ev_start = d->events[0], ev_end = d->events[1];
+  if (cudaEventRecord(ev_start, st) != cudaSuccess ||
+      cudaStreamWaitEvent(d->s_in, ev_start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(d->s_out, ev_start, 0) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  DSA_TRY(h2d(at(dev->q_offsets, 0), qo, (size_t)(B + 1) * 4, d->s_in));
+  DSA_TRY(h2d(at(dev->kv_offsets, 0), ko, (size_t)(B + 1) * 4, d->s_in));
+  DSA_TRY(h2d(at(dev->w, 0), host->w, w_bytes, d->s_in));
   int64_t kv_done = 0;
   if (split) {
     DSA_TRY(check_indexer(P));
@@ -1318,14 +1328,14 @@ dsa_status dsa_prefill_from_host(const dsa_params* P, const dsa_ragged* R,
     void* scratch = static_cast<char*>(workspace) + idx_bytes;
     DSA_TRY(h2d(at(dev->q_idx, 0), host->q_idx, (size_t)TQ * idx_row, d->s_in));
     DSA_TRY(h2d(at(dev->k_idx, 0), host->k_idx, (size_t)R->total_kv * idx_row, d->s_in));
-    cudaEvent_t ev_idx = d->events[2 + 2 * n_chunks];
+    cudaEvent_t ev_idx = d->events[2 + 2 * n_ranges];
     if (cudaEventRecord(ev_idx, d->s_in) != cudaSuccess ||
         cudaStreamWaitEvent(st, ev_idx, 0) != cudaSuccess)
       return DSA_ERR_CUDA;
     DSA_TRY(run_index(*d, P, &Rd, dev->q_idx, dev->k_idx, dev->w, 0, TQ, idx_all, scratch,
                       (size_t)((int64_t)ws_bytes - idx_bytes), st, -1, 0));
-    for (int c = 0; c < n_chunks; ++c) {
-      const int64_t a0 = TQ * c / n_chunks, a1 = TQ * (c + 1) / n_chunks;
+    for (int c = 0; c < n_ranges; ++c) {
+      const int64_t a0 = cut[c], a1 = cut[c + 1];
       if (a0 == a1) continue;
       const int64_t kv_need = std::max(kv_done, kv_need_of(a0, a1));
       cudaEvent_t ev_in = d->events[2 + 2 * c], ev_done = d->events[3 + 2 * c];
@@ -1350,7 +1360,7 @@ dsa_status dsa_prefill_from_host(const dsa_params* P, const dsa_ragged* R,
     }
   } else {
     // the layer per range, each range's inputs uploaded just before it
-    for (int ci = 0; ci < n_chunks; ++ci) {
+    for (int ci = 0; ci < n_ranges; ++ci) {
       const int c = reverse ? n_chunks - 1 - ci : ci;
       const int64_t a0 = TQ * c / n_chunks, a1 = TQ * (c + 1) / n_chunks;
       if (a0 == a1) continue;
