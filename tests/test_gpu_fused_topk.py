@@ -96,6 +96,8 @@ FUSED_CASES = {
     "k1": dict(q_lens=[1500], kv_lens=[1500], K=1),
     "k4096": dict(q_lens=[600], kv_lens=[20000], K=4096),
     "one_head": dict(q_lens=[2000], kv_lens=[5000], Hi=1, K=200),
+    # a full head pair and a pair of one head (each head's accumulator signalled on its own)
+    "three_heads": dict(q_lens=[1800, 700], kv_lens=[6000, 700], Hi=3, K=256),
     # rows of more than 2048 samples (n > 32768): their thresholds come from the one-CTA-per-row
     # kernel
     "long_rows": dict(q_lens=[96], kv_lens=[40000], K=512),
